@@ -1,0 +1,297 @@
+"""Python face of the CPU oracle (``convrot_oracle.c``) plus pure-Python
+references used only on tiny inputs.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py``.  It shares no code with the CUDA path and
+never imports the product package's arithmetic.
+
+Every function cites the passage it follows (page title and section):
+
+* block-diagonal Hadamard rotation -- lehuy.net "Nen mo hinh video khuech tan
+  31B xuong 14B chi voi 6 buoc", section "Cach nen hoat dong";
+* rowwise int8 activation quantisation -- MiniMax-H3-Rung-Omega README,
+  "Technical Architecture Overview", item 2 (Floor 1);
+* per-output-channel F32 weight scales, [output, input] storage -- "MiniMax H3 -
+  pruned INT8 ConvRot - input-major", section "Input-major checkpoint";
+* exact undo of the rotation -- "HyperFlow H3 Flash MLX", section "How to run";
+* W8A8 INT8 -- HyperFlow H3 Flash card, "Choose a Weight Format".
+
+Readings where the pages are silent (all listed in the design doc): Sylvester
+order H[i][j] = (-1)^popcount(i & j); unnormalised transform with the 1/b
+folded into the dequantisation; fp32 butterflies in ascending stage order;
+s = amax/127 and q = rne(z * (127/amax)) in f32; a zero row has s = 0.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from fractions import Fraction
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "convrot_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+__all__ = [
+    "build", "lib", "num_threads", "hadamard", "hadamard_sylvester", "fwht",
+    "quantize_rows", "quantize_act", "pack_weight", "igemm", "igemm_pairs",
+    "dequant", "dequant_pairs", "linear", "rotate_explicit_f64",
+    "bf16_bits", "bf16_bits_to_f32", "py_fwht_exact", "py_quantize_row_exact",
+    "py_igemm",
+]
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", *_CFLAGS, "-o", _LIB_PATH, _SRC, "-lm"])
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I32 = ctypes.c_int
+        L.oracle_hadamard_entry.argtypes = [I64, I64]
+        L.oracle_hadamard_entry.restype = I32
+        L.oracle_num_threads.restype = I32
+        L.oracle_fwht_f32.argtypes = [P, I64, I32]
+        L.oracle_quantize_rows_f32.argtypes = [P, I64, I64, I64, P, I64, P]
+        L.oracle_quantize_act_bf16.argtypes = [P, I64, I64, I64, I32, P, I64, P]
+        L.oracle_pack_weight_f32.argtypes = [P, I64, I64, I32, P, P]
+        L.oracle_igemm_s64.argtypes = [P, I64, P, I64, I64, I64, I64, P, I64]
+        L.oracle_igemm_s64_pairs.argtypes = [P, I64, P, I64, I64, P, P, I64, P]
+        L.oracle_dequant_f64.argtypes = [P, I64, I64, P, P, P, ctypes.c_double, I32, P]
+        L.oracle_dequant_pairs_f64.argtypes = [P, P, P, I64, P, P, P, ctypes.c_double, I32, P]
+        L.oracle_rotate_explicit_f64.argtypes = [P, I64, I64, I32, P]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses."""
+    return int(lib().oracle_num_threads())
+
+
+# ---------------------------------------------------------------- Hadamard
+
+
+def hadamard(b: int) -> np.ndarray:
+    """H_b from its entry definition (-1)^popcount(i & j), via the C oracle."""
+    L = lib()
+    return np.array([[L.oracle_hadamard_entry(i, j) for j in range(b)] for i in range(b)], dtype=np.int64)
+
+
+def hadamard_sylvester(b: int) -> list[list[int]]:
+    """Independent construction: H_1 = [1], H_2n = [[H, H], [H, -H]] (pure Python)."""
+    H = [[1]]
+    while len(H) < b:
+        H = [r + r for r in H] + [r + [-v for v in r] for r in H]
+    if len(H) != b:
+        raise ValueError("b must be a power of two")
+    return H
+
+
+def fwht(x: np.ndarray, b: int) -> np.ndarray:
+    """Block-diagonal FWHT of the last axis of a float32 array (canonical order)."""
+    v = np.ascontiguousarray(x, dtype=np.float32).copy()
+    lib().oracle_fwht_f32(_p(v), v.size, b)
+    return v
+
+
+def rotate_explicit_f64(x: np.ndarray, b: int) -> np.ndarray:
+    """z = blockdiag(H_b) x by the explicit matrix, fp64 accumulation."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    M, K = x.shape
+    z = np.empty((M, K), dtype=np.float64)
+    lib().oracle_rotate_explicit_f64(_p(x), M, K, b, _p(z))
+    return z
+
+
+# ---------------------------------------------------------------- quantisers
+
+
+def bf16_bits(x) -> np.ndarray:
+    """Raw uint16 bits of a torch bfloat16 tensor (CPU)."""
+    import torch
+
+    t = x.detach().to("cpu").contiguous()
+    assert t.dtype == torch.bfloat16
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def quantize_rows(z: np.ndarray):
+    """Rowwise symmetric int8 of already-rotated f32 rows -> (q int8, s f32)."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    M, K = z.shape
+    q = np.empty((M, K), dtype=np.int8)
+    s = np.empty((M,), dtype=np.float32)
+    lib().oracle_quantize_rows_f32(_p(z), M, K, K, _p(q), K, _p(s))
+    return q, s
+
+
+def quantize_act(x_bits: np.ndarray, b: int):
+    """bf16 activations (uint16 bits [M, K]) -> rotate (block b) -> (q, s_x)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    M, K = x_bits.shape
+    q = np.empty((M, K), dtype=np.int8)
+    s = np.empty((M,), dtype=np.float32)
+    lib().oracle_quantize_act_bf16(_p(x_bits), M, K, K, b, _p(q), K, _p(s))
+    return q, s
+
+
+def pack_weight(w: np.ndarray, b: int):
+    """f32 weights [N, K] -> rotate along K -> per-output-channel (q_w, s_w)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    q = np.empty((N, K), dtype=np.int8)
+    s = np.empty((N,), dtype=np.float32)
+    lib().oracle_pack_weight_f32(_p(w), N, K, b, _p(q), _p(s))
+    return q, s
+
+
+# ---------------------------------------------------------------- GEMM + epilogue
+
+
+def igemm(qa: np.ndarray, qb: np.ndarray) -> np.ndarray:
+    """acc = qa @ qb.T exactly in int64 (qa [M, K], qb [N, K], int8)."""
+    qa = np.ascontiguousarray(qa, dtype=np.int8)
+    qb = np.ascontiguousarray(qb, dtype=np.int8)
+    M, K = qa.shape
+    N, K2 = qb.shape
+    assert K == K2
+    c = np.empty((M, N), dtype=np.int64)
+    lib().oracle_igemm_s64(_p(qa), K, _p(qb), K, M, N, K, _p(c), N)
+    return c
+
+
+def igemm_pairs(qa: np.ndarray, qb: np.ndarray, mi: np.ndarray, ni: np.ndarray) -> np.ndarray:
+    """acc[t] = qa[mi[t]] . qb[ni[t]] exactly in int64."""
+    qa = np.ascontiguousarray(qa, dtype=np.int8)
+    qb = np.ascontiguousarray(qb, dtype=np.int8)
+    mi = np.ascontiguousarray(mi, dtype=np.int64)
+    ni = np.ascontiguousarray(ni, dtype=np.int64)
+    K = qa.shape[1]
+    out = np.empty(mi.shape, dtype=np.int64)
+    lib().oracle_igemm_s64_pairs(_p(qa), K, _p(qb), K, K, _p(mi), _p(ni), mi.size, _p(out))
+    return out
+
+
+def _alpha(b: int) -> float:
+    return 1.0 / b if b > 1 else 1.0
+
+
+def dequant(acc: np.ndarray, s_a: np.ndarray, s_b: np.ndarray, bias: np.ndarray | None,
+            b: int, gelu: bool = False) -> np.ndarray:
+    """y = acc * s_a[m] * s_b[n] / b + bias[n] in fp64 (optional exact GELU)."""
+    acc = np.ascontiguousarray(acc, dtype=np.int64)
+    M, N = acc.shape
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_b = np.ascontiguousarray(s_b, dtype=np.float32)
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((M, N), dtype=np.float64)
+    lib().oracle_dequant_f64(_p(acc), M, N, _p(s_a), _p(s_b), _p(bias), _alpha(b), int(gelu), _p(y))
+    return y
+
+
+def dequant_pairs(acc, mi, ni, s_a, s_b, bias, b: int, gelu: bool = False) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, dtype=np.int64)
+    mi = np.ascontiguousarray(mi, dtype=np.int64)
+    ni = np.ascontiguousarray(ni, dtype=np.int64)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_b = np.ascontiguousarray(s_b, dtype=np.float32)
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty(acc.shape, dtype=np.float64)
+    lib().oracle_dequant_pairs_f64(_p(acc), _p(mi), _p(ni), acc.size, _p(s_a), _p(s_b), _p(bias),
+                                   _alpha(b), int(gelu), _p(y))
+    return y
+
+
+def linear(x_bits: np.ndarray, w: np.ndarray, bias: np.ndarray | None, b: int, gelu: bool = False):
+    """Whole path on the CPU: returns (y fp64, q_x, s_x, q_w, s_w, acc)."""
+    qx, sx = quantize_act(x_bits, b)
+    qw, sw = pack_weight(w, b)
+    acc = igemm(qx, qw)
+    y = dequant(acc, sx, sw, bias, b, gelu)
+    return y, qx, sx, qw, sw, acc
+
+
+# ---------------------------------------------------------------- pure-Python references (tiny inputs)
+
+
+def py_fwht_exact(x: list, b: int) -> list:
+    """Explicit H_b x per block with exact rational arithmetic (no rounding)."""
+    H = hadamard_sylvester(b) if b > 1 else [[1]]
+    bb = max(b, 1)
+    out = []
+    for o in range(0, len(x), bb):
+        blk = [Fraction(v) for v in x[o:o + bb]]
+        out.extend(sum(H[i][j] * blk[j] for j in range(bb)) for i in range(bb))
+    return out
+
+
+def _round_to_f32(r: Fraction) -> Fraction:
+    """Round a rational to the nearest float32 value (ties to even), exactly."""
+    if r == 0:
+        return Fraction(0)
+    sign = -1 if r < 0 else 1
+    a = abs(r)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, -126)  # subnormal range keeps the -149 quantum
+    quantum = Fraction(2) ** (e - 23)
+    n = a / quantum
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * quantum
+
+
+def _rne_int(r: Fraction) -> int:
+    fl = r.numerator // r.denominator
+    rem = r - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return fl
+
+
+def py_quantize_row_exact(z: list):
+    """Quantiser of one row with exact rational arithmetic standing in for f32:
+    inv = f32(127/amax), v = f32(z*inv), q = ties-to-even(v) clamped to +-127,
+    s = f32(amax/127).  Returns (codes, scale as Fraction)."""
+    zq = [Fraction(v) for v in z]
+    amax = max((abs(v) for v in zq), default=Fraction(0))
+    if amax == 0:
+        return [0] * len(zq), Fraction(0)
+    inv = _round_to_f32(Fraction(127) / amax)
+    s = _round_to_f32(amax / 127)
+    codes = []
+    for v in zq:
+        c = _rne_int(_round_to_f32(v * inv))
+        codes.append(max(-127, min(127, c)))
+    return codes, s
+
+
+def py_igemm(qa: list, qb: list) -> list:
+    """Brute-force integer dot products in Python ints."""
+    return [[sum(int(a) * int(b) for a, b in zip(ra, rb)) for rb in qb] for ra in qa]

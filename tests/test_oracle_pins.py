@@ -1,0 +1,287 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix.
+
+None of these re-types the oracle's own formula: each compares it with an
+independent construction (Sylvester recursion, exact rational arithmetic,
+pure-Python brute force), a closed form, or an invariant.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(a) -> np.ndarray:
+    t = torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return O.bf16_bits(t)
+
+
+def _is_bf16(v: Fraction) -> bool:
+    f = np.float32(float(v))
+    if Fraction(float(f)) != v:
+        return False
+    return O.bf16_bits_to_f32(_bf16([f]))[0] == f
+
+
+# ------------------------------------------------------------ Hadamard matrix
+
+
+@pytest.mark.parametrize("b", [1, 2, 4, 8, 16, 32, 64, 128, 256])
+def test_hadamard_definition_matches_sylvester_and_is_orthogonal(b):
+    H = O.hadamard(b)
+    S = np.array(O.hadamard_sylvester(b), dtype=np.int64)
+    assert (H == S).all()
+    assert (H == H.T).all()
+    assert (H[0] == 1).all() and (H[:, 0] == 1).all()
+    assert (H @ H.T == b * np.eye(b, dtype=np.int64)).all()
+
+
+# ------------------------------------------------------------ rotation
+
+
+@pytest.mark.parametrize("b", [2, 4, 16, 128, 256])
+def test_fwht_equals_explicit_matrix_on_integers(b):
+    rng = np.random.default_rng(b)
+    x = rng.integers(-1000, 1000, size=3 * b).astype(np.float32)  # every fp32 op exact
+    z = O.fwht(x, b)
+    exact = O.py_fwht_exact([int(v) for v in x], b)
+    assert [Fraction(float(v)) for v in z] == exact
+
+
+@pytest.mark.parametrize("b", [4, 128])
+def test_fwht_is_involution_up_to_b(b):
+    # the pages: the Hadamard rotation can be undone exactly
+    rng = np.random.default_rng(7)
+    x = rng.integers(-500, 500, size=4 * b).astype(np.float32)
+    zz = O.fwht(O.fwht(x, b), b)
+    assert (zz == b * x).all()
+
+
+def test_fwht_f32_within_summation_error_bound():
+    # general bf16 inputs: fp32 butterflies vs the exact product; a depth-7
+    # tree of roundings is bounded by 7 * 2^-24 * sum|x| (first order)
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((8, 256)).astype(np.float32)
+    x[:, 5] *= 20
+    x = O.bf16_bits_to_f32(_bf16(x)).reshape(8, 256)
+    z = np.stack([O.fwht(r, 128) for r in x])
+    exact = O.rotate_explicit_f64(x, 128)
+    absx = np.abs(x).reshape(8, 2, 128).sum(-1)
+    bound = 7 * 2.0 ** -24 * np.repeat(absx, 128, axis=1) * 1.0001
+    assert (np.abs(z - exact) <= bound).all()
+    assert np.abs(z - exact).max() > 0  # the bound is exercised, not vacuous
+
+
+def test_rotation_of_constant_block_is_dc_spike():
+    b, c = 128, 0.75
+    x = np.full((1, 2 * b), c, dtype=np.float32)
+    q, s = O.quantize_act(_bf16(x), b)
+    expect = np.zeros(2 * b, dtype=np.int8)
+    expect[0] = expect[b] = 127
+    assert (q[0] == expect).all()
+    assert s[0] == np.float32(b * c) / np.float32(127)
+
+
+@pytest.mark.parametrize("i", [0, 1, 77, 127])
+def test_rotation_of_spike_gives_hadamard_column_signs(i):
+    b, c = 128, -3.0
+    x = np.zeros((1, b), dtype=np.float32)
+    x[0, i] = c
+    q, s = O.quantize_act(_bf16(x), b)
+    H = np.array(O.hadamard_sylvester(b))
+    assert (q[0] == (-127 * H[:, i])).all()
+    assert s[0] == np.float32(3.0) / np.float32(127)
+
+
+# ------------------------------------------------------------ quantiser
+
+
+def _load_ties():
+    rows = []
+    with open(os.path.join(GOLDEN, "quant_ties.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, codes, scale = [p.strip() for p in line.split("|")]
+            path, block, z = head.split()
+            rows.append((path, int(block), [int(v) for v in z.split(",")],
+                         [int(v) for v in codes.split(",")], Fraction(scale)))
+    return rows
+
+
+@pytest.mark.parametrize("case", _load_ties(), ids=lambda c: f"{c[0]}-b{c[1]}")
+def test_quantiser_ties_round_half_to_even(case):
+    path, b, zlead, codes_lead, scale = case
+    K = max(b, len(zlead))
+    z = zlead + [0] * (K - len(zlead))
+    bb = max(b, 1)
+    H = O.hadamard_sylvester(bb) if bb > 1 else [[1]]
+    x = [Fraction(sum(H[i][j] * z[o + j] for j in range(bb)), bb) for o in range(0, K, bb) for i in range(bb)]
+    expect = codes_lead + [0] * (K - len(codes_lead))
+    if path == "act":
+        assert all(_is_bf16(v) for v in x)
+        q, s = O.quantize_act(_bf16([[float(v) for v in x]]), b)
+    else:
+        assert all(Fraction(float(np.float32(float(v)))) == v for v in x)
+        q, s = O.pack_weight(np.array([[float(v) for v in x]], dtype=np.float32), b)
+    assert q[0].tolist() == expect
+    assert Fraction(float(s[0])) == scale
+
+
+def test_quantiser_matches_exact_rational_arbiter():
+    rng = np.random.default_rng(11)
+    z = (rng.standard_normal((40, 96)) * rng.uniform(0.01, 100, (40, 1))).astype(np.float32)
+    z[3] = 0.0
+    z[5, 7] = 1e4
+    q, s = O.quantize_rows(z)
+    for m in range(z.shape[0]):
+        codes, sc = O.py_quantize_row_exact([Fraction(float(v)) for v in z[m]])
+        assert q[m].tolist() == codes
+        assert Fraction(float(s[m])) == sc
+
+
+def test_quantiser_invariances():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((16, 256)) * 3).astype(np.float32)
+    xb = _bf16(x)
+    q, s = O.quantize_act(xb, 128)
+    qn, sn = O.quantize_act(_bf16(-O.bf16_bits_to_f32(xb)), 128)
+    assert (qn == -q).all() and (sn == s).all()
+    for k in (-6, -1, 3, 9):
+        q2, s2 = O.quantize_act(_bf16(O.bf16_bits_to_f32(xb) * np.float32(2.0 ** k)), 128)
+        assert (q2 == q).all()
+        assert (s2 == s * np.float32(2.0 ** k)).all()
+    assert (np.abs(q).max(axis=1) == 127).all()
+
+
+def test_zero_row_gives_zero_scale_and_codes():
+    x = np.zeros((3, 256), dtype=np.float32)
+    x[1, 9] = 1.0
+    q, s = O.quantize_act(_bf16(x), 128)
+    assert s[0] == 0 and s[2] == 0 and not q[0].any() and not q[2].any()
+    assert s[1] > 0
+
+
+def test_block_one_is_plain_rowwise_absmax():
+    rng = np.random.default_rng(2)
+    x = O.bf16_bits_to_f32(_bf16(rng.standard_normal((6, 64)))).reshape(6, 64)
+    q1, s1 = O.quantize_act(_bf16(x), 1)
+    q0, s0 = O.quantize_act(_bf16(x), 0)
+    for m in range(6):
+        codes, sc = O.py_quantize_row_exact([Fraction(float(v)) for v in x[m]])
+        assert q1[m].tolist() == codes and q0[m].tolist() == codes
+        assert Fraction(float(s1[m])) == sc == Fraction(float(s0[m]))
+
+
+def test_weight_scales_are_per_output_channel():
+    rng = np.random.default_rng(8)
+    w = (rng.standard_normal((5, 256)) * 0.02).astype(np.float32)
+    w[2] *= 100
+    q, s = O.pack_weight(w, 128)
+    for n in range(5):
+        zr = O.fwht(w[n], 128)
+        codes, sc = O.py_quantize_row_exact([Fraction(float(v)) for v in zr])
+        assert q[n].tolist() == codes and Fraction(float(s[n])) == sc
+
+
+# ------------------------------------------------------------ GEMM and epilogue
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 5, 7), (8, 4, 32), (2, 3, 300)])
+def test_igemm_equals_bruteforce(shape):
+    M, N, K = shape
+    rng = np.random.default_rng(M * 100 + N * 10 + K)
+    qa = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    qb = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    qa[0, 0] = -127
+    qb[-1, -1] = 127
+    assert O.igemm(qa, qb).tolist() == O.py_igemm(qa.tolist(), qb.tolist())
+    mi = np.array([0, M - 1, M // 2], dtype=np.int64)
+    ni = np.array([N - 1, 0, N // 2], dtype=np.int64)
+    full = O.py_igemm(qa.tolist(), qb.tolist())
+    assert O.igemm_pairs(qa, qb, mi, ni).tolist() == [full[m][n] for m, n in zip(mi, ni)]
+
+
+def test_igemm_extreme_accumulator_fits_int32_at_largest_k():
+    K = 21504
+    qa = np.full((1, K), -127, dtype=np.int8)
+    qb = np.full((2, K), 127, dtype=np.int8)
+    qb[1] = -127
+    acc = O.igemm(qa, qb)
+    assert acc[0, 0] == -127 * 127 * K and acc[0, 1] == 127 * 127 * K
+    assert abs(acc).max() < 2 ** 31
+
+
+def test_dequant_exact_rational():
+    rng = np.random.default_rng(4)
+    acc = rng.integers(-10 ** 6, 10 ** 6, (3, 4))
+    sa = rng.uniform(0.01, 1, 3).astype(np.float32)
+    sb = rng.uniform(0.001, 0.1, 4).astype(np.float32)
+    bias = rng.standard_normal(4).astype(np.float32)
+    y = O.dequant(acc, sa, sb, bias, 128)
+    for m in range(3):
+        for n in range(4):
+            ex = Fraction(int(acc[m, n])) * Fraction(float(sa[m])) * Fraction(float(sb[n])) / 128 + Fraction(float(bias[n]))
+            assert abs(Fraction(y[m, n]) - ex) <= abs(ex) * Fraction(1, 2 ** 50)
+    y0 = O.dequant(acc, sa, sb, None, 0)
+    assert np.allclose(y0, acc * sa[:, None].astype(np.float64) * sb[None, :].astype(np.float64), rtol=1e-15)
+
+
+def test_gelu_closed_forms():
+    acc = np.array([[0, 10 ** 6, -10 ** 6]], dtype=np.int64)
+    y = O.dequant(acc, np.array([1e-3], np.float32), np.array([1.0, 1.0, 1.0], np.float32), None, 0, gelu=True)
+    assert y[0, 0] == 0.0
+    x1 = float(np.float32(1e-3)) * 1e6
+    assert abs(y[0, 1] - x1) < 1e-12 * x1  # gelu(x) -> x for large x
+    assert abs(y[0, 2]) < 1e-12           # gelu(x) -> 0 for large negative x
+
+
+# ------------------------------------------------------------ the whole linear
+
+
+def _tiny():
+    from w8a8_int8_quantized_block_b200 import workloads as W
+    x, w, bias = W.linear_inputs(W.TINY)
+    return x, w.numpy(), bias.numpy()
+
+
+def test_linear_close_to_unquantised_product():
+    # The pages accept a block when its cosine to the reference is >= 0.995
+    # ("HyperFlow H3 Flash MLX", "How they were checked"); one quantised linear
+    # must sit well inside that.
+    x, w, bias = _tiny()
+    xb = O.bf16_bits(x)
+    y, *_ = O.linear(xb, w, bias, 128)
+    ref = O.bf16_bits_to_f32(xb).astype(np.float64) @ w.T.astype(np.float64) + bias
+    cos = (y * ref).sum() / np.sqrt((y * y).sum() * (ref * ref).sum())
+    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert cos > 0.999 and rel < 0.03
+
+
+def test_rotation_reduces_error_with_outlier_channels():
+    x, w, bias = _tiny()
+    xb = O.bf16_bits(x)
+    ref = O.bf16_bits_to_f32(xb).astype(np.float64) @ w.T.astype(np.float64) + bias
+    err = {}
+    for b in (0, 128):
+        y, *_ = O.linear(xb, w, bias, b)
+        err[b] = np.linalg.norm(y - ref)
+    assert err[128] < 0.8 * err[0]
+
+
+def test_rotated_linear_equals_unrotated_math_on_exact_inputs():
+    # With integer inputs every step before rounding is exact, and
+    # (H x) . (H w) / b = x . w: the rotation cancels in the product.
+    rng = np.random.default_rng(12)
+    b = 128
+    xz = rng.integers(-3, 4, (2, b)).astype(np.float32)
+    wz = rng.integers(-3, 4, (3, b)).astype(np.float32)
+    zx = np.stack([O.fwht(r, b) for r in xz]).astype(np.int64)
+    zw = np.stack([O.fwht(r, b) for r in wz]).astype(np.int64)
+    assert ((zx @ zw.T) == b * (xz.astype(np.int64) @ wz.astype(np.int64).T)).all()
