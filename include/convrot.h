@@ -1,0 +1,164 @@
+/*
+ * convrot.h -- C ABI of libconvrot.so, the B200 (sm_100a) ConvRot W8A8 INT8
+ * linear projection.
+ *
+ * The operation (the pages' "int8_convrot" linear):
+ *   1. rotate: z = blockdiag(H_b) x for every token, H_b the Sylvester Hadamard
+ *      matrix H[i][j] = (-1)^popcount(i & j), b = 128 ("180 linear layers
+ *      quantized to INT8 behind a block-diagonal Hadamard rotation" -- lehuy.net,
+ *      "Nen mo hinh video khuech tan 31B xuong 14B chi voi 6 buoc", section
+ *      "Cach nen hoat dong");
+ *   2. quantise each token row to symmetric int8 with one F32 scale
+ *      ("Rowwise INT8 Quantize" -- MiniMax-H3-Rung-Omega README, "Technical
+ *      Architecture Overview", item 2, Floor 1):
+ *      s = amax/127, q = clamp(rne(z * (127/amax)), -127, 127);
+ *   3. multiply with int8 weights that were rotated the same way and quantised
+ *      per output channel offline ("per-output F32 scales", "ConvRot metadata",
+ *      [output, input] storage -- "MiniMax H3 - pruned INT8 ConvRot -
+ *      input-major", section "Input-major checkpoint"), accumulating in int32;
+ *   4. dequantise: y = acc * s_x[m] * s_w[n] / b + bias[n], stored as bf16
+ *      (bf16, not fp16: "the residual stream reaches 2.4e5" -- "HyperFlow H3
+ *      Flash MLX", section "How to run").
+ * The 1/b folds the 1/sqrt(b) of both orthonormal rotations into one exact
+ * power-of-two factor.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except
+ *     where a name ends in `_host`.  The library never allocates or frees.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) on the current device, which must be sm_100 (B200).
+ *   - Argument errors are detected on the host and returned before anything is
+ *     launched: CONVROT_EINVAL (null pointer, non-positive or oversized size,
+ *     bad stride, pointer not 16-byte aligned), CONVROT_EUNSUPPORTED (block
+ *     size, device), CONVROT_ELAYOUT (weight descriptor mismatch).
+ *     CONVROT_ECUDA reports a failed CUDA call (launch, attribute, copy).
+ *   - Every device-side wait is bounded; a wait that gives up records a code
+ *     in the library's device error word, which convrot_last_device_status()
+ *     reports as CONVROT_ETIMEOUT.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Row-major everywhere: element (r, c) of a matrix with leading dimension
+ *     ld is at offset r*ld + c.
+ */
+#ifndef CONVROT_H
+#define CONVROT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum convrot_status {
+    CONVROT_OK = 0,
+    CONVROT_EINVAL = 1,
+    CONVROT_EUNSUPPORTED = 2,
+    CONVROT_ELAYOUT = 3,
+    CONVROT_ECUDA = 4,
+    CONVROT_ETIMEOUT = 5
+} convrot_status;
+
+/* Packed-weight descriptor.  Plays the role of the pages' "versioned layout
+ * marker" that is validated before the pipeline is built ("MiniMax H3 -
+ * pruned INT8 ConvRot - input-major", section "Input-major checkpoint"). */
+#define CONVROT_WDESC_MAGIC 0x52564E43u   /* "CNVR" */
+#define CONVROT_WDESC_VERSION 1u
+#define CONVROT_LAYOUT_OUTPUT_MAJOR 1u    /* int8 [N][K], K contiguous */
+
+typedef struct convrot_wdesc {
+    uint32_t magic;    /* CONVROT_WDESC_MAGIC */
+    uint32_t version;  /* CONVROT_WDESC_VERSION */
+    uint32_t layout;   /* CONVROT_LAYOUT_OUTPUT_MAJOR */
+    int32_t block;     /* Hadamard block used when packing: 128, or 0 = none */
+    int64_t N;         /* output channels */
+    int64_t K;         /* input channels */
+} convrot_wdesc;
+
+/* Epilogue selector of the linear entry points. */
+#define CONVROT_EPI_NONE 0  /* y = acc*s_x*s_w/b + bias */
+#define CONVROT_EPI_GELU 1  /* then exact-erf GELU: 0.5*y*(1 + erf(y/sqrt(2))) */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* convrot_status_string(int status);
+
+/* ABI version of this header/library pair (currently 1). */
+int convrot_abi_version(void);
+
+/* Offline weight packing (step 3's weights).
+ * w: f32 [N][K] row-major.  block: 128 (rotate) or 0 (no rotation).
+ * Writes q: int8 [N][K] (K contiguous, "output-major") and s_w: f32 [N], and
+ * fills *desc (HOST pointer) synchronously.  Requires K % 64 == 0,
+ * K % block == 0, K <= 32768, N <= 2^31-1, 16-byte aligned pointers. */
+convrot_status convrot_pack_weight(const float* w, int64_t N, int64_t K, int32_t block, int8_t* q,
+                                   float* s_w, convrot_wdesc* desc, void* stream);
+
+/* Steps 1-2: x: bf16 [M][K] with row stride ldx (elements) ->
+ * q: int8 [M][K] (contiguous) and s_x: f32 [M].  block: 128 or 0.
+ * Requires K % 64 == 0, K % block == 0, K <= 32768, ldx >= K, ldx % 8 == 0,
+ * 0 < M <= 2^31-1.  A row of zeros gives s_x = 0 and zero codes. */
+convrot_status convrot_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int32_t block,
+                                    int8_t* q, float* s_x, void* stream);
+
+/* Steps 3-4 on already quantised activations.
+ * qx: int8 [M][K], s_x: f32 [M]; qw/s_w/desc from convrot_pack_weight;
+ * bias: f32 [N] or NULL; epilogue: CONVROT_EPI_*; y: bf16 [M][N] with row
+ * stride ldy (ldy >= N, ldy % 8 == 0).  K is desc->K (K % 16 == 0). */
+convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int8_t* qw, const float* s_w,
+                                   const convrot_wdesc* desc, const float* bias, int32_t epilogue, int64_t M,
+                                   uint16_t* y, int64_t ldy, void* stream);
+
+/* Bytes of device workspace convrot_linear_fused needs: the int8 codes
+ * (M*K, rounded up to 256) plus the scales (4*M, rounded up to 256). */
+size_t convrot_workspace_bytes(int64_t M, int64_t K);
+
+/* The whole linear, steps 1-4, in two kernels on `stream` (the GEMM starts
+ * while the quantiser drains).  x: bf16 [M][K] (row stride ldx); the codes and
+ * scales go to `workspace` (>= convrot_workspace_bytes(M, K) bytes, 256-byte
+ * aligned, caller-owned, must not be shared by calls that overlap). */
+convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw,
+                                    const float* s_w, const convrot_wdesc* desc, const float* bias,
+                                    int32_t epilogue, void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy,
+                                    void* stream);
+
+/* End-to-end form of convrot_linear_fused for callers whose activations live
+ * in host memory: copies x_host (bf16 [M][K], contiguous; pinned for overlap)
+ * into the caller's device buffer x_dev, runs the fused linear into y_dev
+ * (bf16 [M][N], contiguous) and copies it back to y_host.  All enqueued on
+ * `stream`; the host buffers must stay valid until the stream reaches the end
+ * of the call. */
+convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, const int8_t* qw, const float* s_w,
+                                         const convrot_wdesc* desc, const float* bias, int32_t epilogue,
+                                         uint16_t* x_dev, void* workspace, size_t ws_bytes, uint16_t* y_dev,
+                                         uint16_t* y_host, void* stream);
+
+/* Batched int8 GEMM with per-row scales on both operands and no rotation:
+ * y[b][m][n] = bf16(sum_k qa[b][m][k]*qb[b][n][k] * sa[b*M+m] * sb[b*N+n]).
+ * Shapes like attention's Q K^T over heads.  All contiguous; K % 16 == 0. */
+convrot_status convrot_w8a8_bmm(const int8_t* qa, const float* sa, const int8_t* qb, const float* sb,
+                                int64_t batch, int64_t M, int64_t N, int64_t K, uint16_t* y, void* stream);
+
+/* Test hook: raw int32 accumulators acc[b][m][n] = sum_k qa[b][m][k]*qb[b][n][k]
+ * from the same tensor-core main loop (N % 4 == 0, K % 16 == 0). */
+convrot_status convrot_igemm_s32(const int8_t* qa, const int8_t* qb, int64_t batch, int64_t M, int64_t N,
+                                 int64_t K, int32_t* acc, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: CONVROT_ETIMEOUT if any bounded wait gave up since the last
+ * call, CONVROT_ECUDA if the synchronisation failed, else CONVROT_OK.
+ * *code (may be NULL) receives the raw site code (0 = none). */
+convrot_status convrot_last_device_status(void* stream, uint32_t* code);
+
+/* Bound, in nanoseconds, on every device-side wait of later launches
+ * (default 2e9; 0 restores the default). */
+void convrot_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook for the failure path: launches one CTA whose wait can never be
+ * satisfied, bounded by limit_ns; afterwards convrot_last_device_status()
+ * must report CONVROT_ETIMEOUT with code 6.  Faults nothing. */
+convrot_status convrot_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H */

@@ -1,0 +1,120 @@
+"""Host-side tests of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_int8_quantized_block_b200 import convrot as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "convrot.h")
+
+
+def _declared_symbols():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(convrot_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    L = C.load()
+    declared = _declared_symbols()
+    assert len(declared) >= 13
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(C.EXPORTS) == declared
+
+
+def test_abi_version_and_status_strings():
+    L = C.load()
+    assert L.convrot_abi_version() == 1
+    for st in range(6):
+        s = L.convrot_status_string(st)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert L.convrot_status_string(99) == b"unknown status"
+
+
+def test_workspace_bytes():
+    L = C.load()
+    assert L.convrot_workspace_bytes(38656, 5376) == 38656 * 5376 + ((38656 * 4 + 255) // 256) * 256
+    assert L.convrot_workspace_bytes(1, 128) == 256 + 256
+    assert L.convrot_workspace_bytes(0, 128) == 0
+
+
+FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("M,K,ldx,block,expect", [
+    (0, 512, 512, 128, C.EINVAL),
+    (-3, 512, 512, 128, C.EINVAL),
+    (4, 100, 100, 0, C.EINVAL),        # K % 64
+    (4, 192, 192, 128, C.EINVAL),      # K % block
+    (4, 512, 500, 128, C.EINVAL),      # ldx < K
+    (4, 512, 516, 128, C.EINVAL),      # ldx % 8
+    (4, 65536, 65536, 128, C.EINVAL),  # K too large
+    (4, 512, 512, 64, C.EUNSUPPORTED),
+])
+def test_quantize_act_rejects_bad_arguments(M, K, ldx, block, expect):
+    st = C.load().convrot_quantize_act(FAKE, M, K, ldx, block, FAKE, FAKE, None)
+    assert st == expect
+
+
+def test_null_pointers_rejected():
+    L = C.load()
+    assert L.convrot_quantize_act(None, 4, 512, 512, 128, FAKE, FAKE, None) == C.EINVAL
+    assert L.convrot_pack_weight(FAKE, 4, 512, 128, FAKE, FAKE, None, None) == C.EINVAL
+    assert L.convrot_igemm_s32(None, FAKE, 1, 4, 4, 16, FAKE, None) == C.EINVAL
+    assert L.convrot_w8a8_bmm(FAKE, None, FAKE, FAKE, 1, 4, 8, 16, FAKE, None) == C.EINVAL
+
+
+def test_misaligned_pointer_rejected():
+    L = C.load()
+    bad = ctypes.c_void_p(0x100008)
+    assert L.convrot_quantize_act(bad, 4, 512, 512, 128, FAKE, FAKE, None) == C.EINVAL
+    assert L.convrot_igemm_s32(FAKE, bad, 1, 4, 4, 16, FAKE, None) == C.EINVAL
+
+
+def _desc(**kw):
+    d = C.WDesc(C.WDESC_MAGIC, C.WDESC_VERSION, C.LAYOUT_OUTPUT_MAJOR, 128, 512, 512)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("field,value", [("magic", 0x12345678), ("version", 2), ("layout", 0), ("block", 64),
+                                         ("N", 0), ("K", 100)])
+def test_bad_weight_descriptor_is_a_layout_error(field, value):
+    d = _desc(**{field: value})
+    st = C.load().convrot_w8a8_linear(FAKE, FAKE, FAKE, FAKE, ctypes.byref(d), None, 0, 16, FAKE, 512, None)
+    assert st == C.ELAYOUT
+
+
+def test_linear_rejects_bad_output_stride_and_epilogue():
+    L = C.load()
+    d = _desc()
+    assert L.convrot_w8a8_linear(FAKE, FAKE, FAKE, FAKE, ctypes.byref(d), None, 0, 16, FAKE, 500, None) == C.EINVAL
+    assert L.convrot_w8a8_linear(FAKE, FAKE, FAKE, FAKE, ctypes.byref(d), None, 7, 16, FAKE, 512, None) == C.EINVAL
+    ws = ctypes.c_void_p(0x100000)
+    assert L.convrot_linear_fused(FAKE, 16, 512, FAKE, FAKE, ctypes.byref(d), None, 0, ws, 10, FAKE, 512,
+                                  None) == C.EINVAL
+
+
+def test_bmm_and_igemm_shape_rules():
+    L = C.load()
+    assert L.convrot_w8a8_bmm(FAKE, FAKE, FAKE, FAKE, 1, 4, 12, 16, FAKE, None) == C.EINVAL   # N % 8
+    assert L.convrot_w8a8_bmm(FAKE, FAKE, FAKE, FAKE, 1, 4, 16, 24, FAKE, None) == C.EINVAL   # K % 16
+    assert L.convrot_igemm_s32(FAKE, FAKE, 0, 4, 4, 16, FAKE, None) == C.EINVAL
+    assert L.convrot_igemm_s32(FAKE, FAKE, 1, 4, 6, 16, FAKE, None) == C.EINVAL               # N % 4
+
+
+def test_valid_call_without_a_gpu_reports_cuda_error():
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present")
+    except ImportError:
+        pass
+    st = C.load().convrot_quantize_act(FAKE, 4, 512, 512, 128, FAKE, FAKE, None)
+    assert st == C.ECUDA

@@ -1,0 +1,205 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, element
+by element, on seeded inputs that span several tiles and a ragged tail."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from w8a8_int8_quantized_block_b200 import convrot as C
+from w8a8_int8_quantized_block_b200 import workloads as W
+
+from helpers import assert_close_bf16, assert_codes_match, bits, f32_of_bf16
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _act(M, K, seed, n_out=0, out_scale=10.0, token_scale=False):
+    spec, (x, _, _) = W.custom_linear(M, K, 8, seed, n_out=n_out, out_scale=out_scale, token_scale=token_scale)
+    return x
+
+
+# ------------------------------------------------------------------ rotate + quantise
+
+
+@pytest.mark.parametrize("M,K,block", [
+    (256, 512, 128), (1, 5376, 128), (127, 5376, 128), (129, 512, 128), (300, 21504, 128),
+    (200, 128, 128), (64, 128, 0), (77, 1024, 128), (33, 384, 128), (5, 640, 0), (3, 32768, 128),
+])
+def test_quantize_act_bitexact(M, K, block):
+    x = _act(M, K, seed=M + K, n_out=max(1, K // 100), token_scale=True)
+    q, s = C.quantize_act(x.to(DEV), block)
+    torch.cuda.synchronize()
+    qr, sr = O.quantize_act(bits(x), block)
+    assert_codes_match(q.cpu().numpy(), s.cpu().numpy(), qr, sr, f32_of_bf16(x), block)
+    assert C.last_device_status() == (C.OK, 0)
+
+
+def test_quantize_act_strided_rows():
+    x = _act(150, 5376 + 64, seed=9, n_out=20)
+    xs = x[:, 32:32 + 5376]  # row stride 5440, offset 64 bytes
+    q, s = C.quantize_act(x.to(DEV)[:, 32:32 + 5376], 128)
+    qr, sr = O.quantize_act(bits(xs.contiguous()), 128)
+    assert_codes_match(q.cpu().numpy(), s.cpu().numpy(), qr, sr, f32_of_bf16(xs.contiguous()), 128)
+
+
+def test_quantize_act_special_rows():
+    K = 1024
+    x = torch.randn(16, K, generator=torch.Generator().manual_seed(3))
+    x[0] = 0.0                              # zero row
+    x[1] = 0.0
+    x[1, 517] = -7.5                        # spike
+    x[2] = 1.0                              # constant row (DC of every block)
+    x[3] = 1e-30                            # tiny values
+    x[4] = 3.0e38 / 2 ** 10                 # large values, no overflow after 128-sums
+    x[5, ::2] *= -1
+    x = x.to(torch.bfloat16)
+    q, s = C.quantize_act(x.to(DEV), 128)
+    qr, sr = O.quantize_act(bits(x), 128)
+    assert_codes_match(q.cpu().numpy(), s.cpu().numpy(), qr, sr, f32_of_bf16(x), 128)
+    assert s[0].item() == 0.0 and not q[0].any()
+
+
+@pytest.mark.parametrize("N,K", [(512, 512), (384, 5376), (5376, 5376), (1000, 21504), (3, 128)])
+def test_pack_weight_bitexact(N, K):
+    w = torch.randn(N, K, generator=torch.Generator().manual_seed(N + K)) * 0.02
+    w[:, 7] *= 30
+    pw = C.pack_weight(w.to(DEV), 128)
+    qr, sr = O.pack_weight(w.numpy(), 128)
+    assert (pw.desc.magic, pw.desc.version, pw.desc.layout, pw.desc.block, pw.desc.N, pw.desc.K) == (
+        C.WDESC_MAGIC, C.WDESC_VERSION, C.LAYOUT_OUTPUT_MAJOR, 128, N, K)
+    assert_codes_match(pw.q.cpu().numpy(), pw.s.cpu().numpy(), qr, sr)
+
+
+# ------------------------------------------------------------------ int8 GEMM accumulators
+
+
+def _codes(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(-127, 128, shape, generator=g, dtype=torch.int8)
+
+
+@pytest.mark.parametrize("B,M,N,K", [
+    (1, 128, 256, 128), (1, 1, 8, 16), (1, 127, 260, 528), (1, 129, 512, 512), (1, 300, 1000, 5376),
+    (3, 200, 264, 128), (1, 1024, 768, 1024), (1, 64, 4, 48),
+])
+def test_igemm_s32_bitexact(B, M, N, K):
+    qa = _codes((B, M, K), M * 7 + K)
+    qb = _codes((B, N, K), N * 3 + K + 1)
+    acc = C.igemm_s32(qa.to(DEV), qb.to(DEV))
+    torch.cuda.synchronize()
+    for b in range(B):
+        ref = O.igemm(qa[b].numpy(), qb[b].numpy())
+        assert (acc[b].cpu().numpy().astype(np.int64) == ref).all()
+
+
+def test_igemm_s32_extreme_accumulators():
+    K = 21504
+    qa = torch.full((1, 130, K), -127, dtype=torch.int8)
+    qa[0, 1] = 127
+    qa[0, 2, ::2] = 127
+    qb = torch.full((1, 260, K), 127, dtype=torch.int8)
+    acc = C.igemm_s32(qa.to(DEV), qb.to(DEV)).cpu().numpy().astype(np.int64)
+    assert (acc[0, 0] == -127 * 127 * K).all()
+    assert (acc[0, 1] == 127 * 127 * K).all()
+    assert (acc[0, 2] == 0).all()
+
+
+# ------------------------------------------------------------------ the linear
+
+
+def _run_linear(spec_or_args, fused=True, gelu=False):
+    x, w, bias = spec_or_args
+    pw = C.pack_weight(w.to(DEV), 128)
+    b = None if bias is None else bias.to(DEV)
+    if fused:
+        y = C.linear_fused(x.to(DEV), pw, b, gelu=gelu)
+    else:
+        q, s = C.quantize_act(x.to(DEV), 128)
+        y = C.w8a8_linear(q, s, pw, b, gelu=gelu)
+    torch.cuda.synchronize()
+    return y, pw
+
+
+def test_linear_tiny_matches_oracle():
+    x, w, bias = W.linear_inputs(W.TINY)
+    y, pw = _run_linear((x, w, bias), fused=True)
+    yr, qx, sx, qw, sw, acc = O.linear(bits(x), w.numpy(), bias.numpy(), 128)
+    assert_codes_match(pw.q.cpu().numpy(), pw.s.cpu().numpy(), qw, sw)
+    assert_close_bf16(f32_of_bf16(y), yr, "tiny linear")
+    assert C.last_device_status() == (C.OK, 0)
+
+
+def test_linear_fused_equals_two_step_bitwise():
+    x, w, bias = W.linear_inputs(W.TINY)
+    y1, _ = _run_linear((x, w, bias), fused=True)
+    y2, _ = _run_linear((x, w, bias), fused=False)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 128, 8), (127, 512, 384), (129, 640, 264), (257, 5376, 520),
+                                   (1000, 1024, 2048)])
+def test_linear_ragged_shapes(M, K, N):
+    spec, (x, w, bias) = W.custom_linear(M, K, N, seed=M + N, n_out=max(1, K // 100))
+    y, pw = _run_linear((x, w, bias), fused=True)
+    yr, *_ = O.linear(bits(x), w.numpy(), bias.numpy(), 128)
+    assert_close_bf16(f32_of_bf16(y), yr, f"linear {M}x{K}x{N}")
+
+
+def test_linear_gelu_epilogue():
+    spec, (x, w, bias) = W.custom_linear(300, 1024, 768, seed=5, n_out=10)
+    y, pw = _run_linear((x, w, bias), fused=True, gelu=True)
+    yr, *_ = O.linear(bits(x), w.numpy(), bias.numpy(), 128, gelu=True)
+    assert_close_bf16(f32_of_bf16(y), yr, "gelu linear")
+
+
+def test_linear_epilogue_on_identical_codes_is_tight():
+    # Same codes on both sides: the only error left is the f32 epilogue and the
+    # final bf16 rounding (<= 2^-8 relative per element plus f32 noise).
+    x, w, bias = W.linear_inputs(W.TINY)
+    pw = C.pack_weight(w.to(DEV), 128)
+    q, s = C.quantize_act(x.to(DEV), 128)
+    y = C.w8a8_linear(q, s, pw, bias.to(DEV))
+    acc = O.igemm(q.cpu().numpy(), pw.q.cpu().numpy())
+    yr = O.dequant(acc, s.cpu().numpy(), pw.s.cpu().numpy(), bias.numpy(), 128)
+    err = np.abs(f32_of_bf16(y).astype(np.float64) - yr)
+    assert (err <= np.abs(yr) * 2.0 ** -8 + 1e-6).all()
+
+
+# ------------------------------------------------------------------ batched skinny-K GEMM
+
+
+def test_bmm_small_batch_matches_oracle():
+    spec = W.QK_BMM
+    q, k = W.bmm_inputs(spec, M=512, N=384)
+    q = q[:3]
+    k = k[:3]
+    B, M, K = q.shape
+    N = k.shape[1]
+    qa, sa = C.quantize_act(q.to(DEV).reshape(B * M, K), 0)
+    qb, sb = C.quantize_act(k.to(DEV).reshape(B * N, K), 0)
+    y = C.w8a8_bmm(qa.view(B, M, K), sa, qb.view(B, N, K), sb)
+    torch.cuda.synchronize()
+    qar, sar = O.quantize_act(bits(q.reshape(B * M, K)), 0)
+    qbr, sbr = O.quantize_act(bits(k.reshape(B * N, K)), 0)
+    assert_codes_match(qa.cpu().numpy(), sa.cpu().numpy(), qar, sar)
+    assert_codes_match(qb.cpu().numpy(), sb.cpu().numpy(), qbr, sbr)
+    for b in range(B):
+        acc = O.igemm(qar[b * M:(b + 1) * M], qbr[b * N:(b + 1) * N])
+        yr = O.dequant(acc, sar[b * M:(b + 1) * M], sbr[b * N:(b + 1) * N], None, 0)
+        assert_close_bf16(f32_of_bf16(y[b]), yr, f"bmm head {b}")
+
+
+# ------------------------------------------------------------------ failure path
+
+
+def test_bounded_wait_times_out_cleanly():
+    assert C.last_device_status() == (C.OK, 0)
+    C.selftest_wait_timeout(2_000_000)  # 2 ms
+    st, code = C.last_device_status()
+    assert st == C.ETIMEOUT and code == 6
+    assert C.last_device_status() == (C.OK, 0)  # cleared, context still usable
+    x = torch.ones(4, 128, dtype=torch.bfloat16, device=DEV)
+    q, s = C.quantize_act(x, 128)
+    torch.cuda.synchronize()
+    assert q[:, 0].tolist() == [127] * 4

@@ -1,0 +1,239 @@
+"""Thin ctypes binding over ``libconvrot.so`` (include/convrot.h).
+
+Argument marshalling only: every step of the path runs in the library's
+sm_100a kernels.  Tensors are torch CUDA tensors (torch supplies device memory
+and streams); outputs are allocated here when not given.  There is no CPU
+fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libconvrot.so")
+
+OK, EINVAL, EUNSUPPORTED, ELAYOUT, ECUDA, ETIMEOUT = range(6)
+EPI_NONE, EPI_GELU = 0, 1
+WDESC_MAGIC = 0x52564E43
+WDESC_VERSION = 1
+LAYOUT_OUTPUT_MAJOR = 1
+
+# Every symbol include/convrot.h declares.
+EXPORTS = (
+    "convrot_status_string", "convrot_abi_version", "convrot_pack_weight", "convrot_quantize_act",
+    "convrot_w8a8_linear", "convrot_workspace_bytes", "convrot_linear_fused", "convrot_linear_fused_host",
+    "convrot_w8a8_bmm", "convrot_igemm_s32", "convrot_last_device_status", "convrot_set_wait_limit_ns",
+    "convrot_selftest_wait_timeout",
+)
+
+
+class ConvrotError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+class WDesc(ctypes.Structure):
+    _fields_ = [("magic", ctypes.c_uint32), ("version", ctypes.c_uint32), ("layout", ctypes.c_uint32),
+                ("block", ctypes.c_int32), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load (building first if it is missing or stale) the CUDA library."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if path is None:
+        from . import build as _build
+        try:
+            _build.build()
+        except (OSError, RuntimeError) as e:  # no nvcc: only an existing library will do
+            if not os.path.exists(p):
+                raise RuntimeError(f"libconvrot.so is missing and could not be built: {e}") from e
+    if not os.path.exists(p):
+        raise RuntimeError(f"libconvrot.so not found at {p}; run `python -m w8a8_int8_quantized_block_b200.build`")
+    L = ctypes.CDLL(p)
+    P, I64, I32, U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64
+    sig = {
+        "convrot_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "convrot_abi_version": ([], ctypes.c_int),
+        "convrot_pack_weight": ([P, I64, I64, I32, P, P, ctypes.POINTER(WDesc), P], ctypes.c_int),
+        "convrot_quantize_act": ([P, I64, I64, I64, I32, P, P, P], ctypes.c_int),
+        "convrot_w8a8_linear": ([P, P, P, P, ctypes.POINTER(WDesc), P, I32, I64, P, I64, P], ctypes.c_int),
+        "convrot_workspace_bytes": ([I64, I64], ctypes.c_size_t),
+        "convrot_linear_fused": ([P, I64, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, ctypes.c_size_t, P, I64, P],
+                                 ctypes.c_int),
+        "convrot_linear_fused_host": ([P, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, P, ctypes.c_size_t, P, P, P],
+                                      ctypes.c_int),
+        "convrot_w8a8_bmm": ([P, P, P, P, I64, I64, I64, I64, P, P], ctypes.c_int),
+        "convrot_igemm_s32": ([P, P, I64, I64, I64, I64, P, P], ctypes.c_int),
+        "convrot_last_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+        "convrot_set_wait_limit_ns": ([U64], None),
+        "convrot_selftest_wait_timeout": ([U64, P], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _check(fn: str, st: int):
+    if st != OK:
+        raise ConvrotError(fn, st, load().convrot_status_string(st).decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str, cuda: bool = True):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if cuda and not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+
+
+@dataclass
+class PackedWeight:
+    """Offline-packed weights: int8 codes [N, K], f32 scales [N], descriptor."""
+    q: torch.Tensor
+    s: torch.Tensor
+    desc: WDesc
+
+    @property
+    def N(self) -> int:
+        return int(self.desc.N)
+
+    @property
+    def K(self) -> int:
+        return int(self.desc.K)
+
+    @property
+    def block(self) -> int:
+        return int(self.desc.block)
+
+
+def pack_weight(w: torch.Tensor, block: int = 128, stream=None) -> PackedWeight:
+    _need(w, torch.float32, "w")
+    w = w.contiguous()
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    s = torch.empty((N,), dtype=torch.float32, device=w.device)
+    d = WDesc()
+    _check("convrot_pack_weight", load().convrot_pack_weight(_ptr(w), N, K, block, _ptr(q), _ptr(s),
+                                                             ctypes.byref(d), _stream(stream)))
+    return PackedWeight(q, s, d)
+
+
+def quantize_act(x: torch.Tensor, block: int = 128, q: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                 stream=None):
+    _need(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device) if q is None else q
+    s = torch.empty((M,), dtype=torch.float32, device=x.device) if s is None else s
+    _check("convrot_quantize_act", load().convrot_quantize_act(_ptr(x), M, K, x.stride(0), block, _ptr(q), _ptr(s),
+                                                               _stream(stream)))
+    return q, s
+
+
+def w8a8_linear(qx: torch.Tensor, sx: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None,
+                gelu: bool = False, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(qx, torch.int8, "qx")
+    M = qx.shape[0]
+    y = torch.empty((M, pw.N), dtype=torch.bfloat16, device=qx.device) if out is None else out
+    _check("convrot_w8a8_linear", load().convrot_w8a8_linear(
+        _ptr(qx.contiguous()), _ptr(sx), _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias),
+        EPI_GELU if gelu else EPI_NONE, M, _ptr(y), y.stride(0), _stream(stream)))
+    return y
+
+
+def workspace_bytes(M: int, K: int) -> int:
+    return int(load().convrot_workspace_bytes(M, K))
+
+
+def alloc_workspace(M: int, K: int, device=None) -> torch.Tensor:
+    """Caller-owned workspace for linear_fused (torch allocations are 512-byte aligned)."""
+    return torch.empty((workspace_bytes(M, K),), dtype=torch.uint8, device=device or "cuda")
+
+
+def linear_fused(x: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None, gelu: bool = False,
+                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    M = x.shape[0]
+    ws = alloc_workspace(M, pw.K, x.device) if workspace is None else workspace
+    y = torch.empty((M, pw.N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("convrot_linear_fused", load().convrot_linear_fused(
+        _ptr(x), M, x.stride(0), _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias),
+        EPI_GELU if gelu else EPI_NONE, _ptr(ws), ws.numel(), _ptr(y), y.stride(0), _stream(stream)))
+    return y
+
+
+def linear_fused_host(x_host: torch.Tensor, pw: PackedWeight, bias, gelu: bool, x_dev: torch.Tensor,
+                      workspace: torch.Tensor, y_dev: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
+    """Host bf16 activations in, host bf16 outputs out (copies enqueued on `stream`)."""
+    _need(x_host, torch.bfloat16, "x_host", cuda=False)
+    _need(y_host, torch.bfloat16, "y_host", cuda=False)
+    M = x_host.shape[0]
+    _check("convrot_linear_fused_host", load().convrot_linear_fused_host(
+        _ptr(x_host), M, _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias), EPI_GELU if gelu else EPI_NONE,
+        _ptr(x_dev), _ptr(workspace), workspace.numel(), _ptr(y_dev), _ptr(y_host), _stream(stream)))
+
+
+def w8a8_bmm(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need(qa, torch.int8, "qa")
+    _need(qb, torch.int8, "qb")
+    B, M, K = qa.shape
+    N = qb.shape[1]
+    y = torch.empty((B, M, N), dtype=torch.bfloat16, device=qa.device) if out is None else out
+    _check("convrot_w8a8_bmm", load().convrot_w8a8_bmm(_ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), B, M, N, K, _ptr(y),
+                                                       _stream(stream)))
+    return y
+
+
+def igemm_s32(qa: torch.Tensor, qb: torch.Tensor, stream=None) -> torch.Tensor:
+    """Raw int32 accumulators (test hook); qa [B, M, K] or [M, K], qb likewise."""
+    _need(qa, torch.int8, "qa")
+    _need(qb, torch.int8, "qb")
+    squeeze = qa.dim() == 2
+    a = qa.unsqueeze(0) if squeeze else qa
+    b = qb.unsqueeze(0) if squeeze else qb
+    B, M, K = a.shape
+    N = b.shape[1]
+    acc = torch.empty((B, M, N), dtype=torch.int32, device=qa.device)
+    _check("convrot_igemm_s32", load().convrot_igemm_s32(_ptr(a.contiguous()), _ptr(b.contiguous()), B, M, N, K,
+                                                         _ptr(acc), _stream(stream)))
+    return acc[0] if squeeze else acc
+
+
+def last_device_status(stream=None):
+    code = ctypes.c_uint32(0)
+    st = load().convrot_last_device_status(_stream(stream), ctypes.byref(code))
+    return st, code.value
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load().convrot_set_wait_limit_ns(ns)
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check("convrot_selftest_wait_timeout", load().convrot_selftest_wait_timeout(limit_ns, _stream(stream)))

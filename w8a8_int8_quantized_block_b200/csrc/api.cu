@@ -1,0 +1,327 @@
+// api.cu -- the C ABI of libconvrot.so: argument validation, TMA descriptor
+// encoding and kernel launches.  The library owns no memory apart from one
+// 4-byte device error word per device.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/convrot.h"
+#include "kernels.h"
+
+namespace convrot {
+
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultLimitNs = 2000000000ull;
+
+std::atomic<uint64_t> g_limit_ns{kDefaultLimitNs};
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int num_sms = 0;
+    unsigned int* err = nullptr;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+const DeviceInfo* device_info() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return nullptr;
+        if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return nullptr;
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+        d.supported = (major == 10 && minor == 0);
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        d.err = static_cast<unsigned int*>(p);
+        d.ready = true;
+    }
+    return &d;
+}
+
+bool encoder_ready() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 3D tiled tensor map: dims {d0 (contiguous), d1, d2}, byte strides of dims 1
+// and 2, box {b0, b1, b2}.
+bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw) {
+    if (!encoder_ready()) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    std::memset(map, 0, sizeof(*map));
+    CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+constexpr int64_t kMaxI32 = 2147483647;
+
+convrot_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CONVROT_OK : CONVROT_ECUDA; }
+
+// Shared by activations (bf16) and weights (f32).
+convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t K, int64_t ldx, int32_t block,
+                            int8_t* q, float* s, cudaStream_t stream) {
+    if (!x || !q || !s) return CONVROT_EINVAL;
+    if (M <= 0 || M > kMaxI32 || K <= 0) return CONVROT_EINVAL;
+    if (block != 0 && block != 1 && block != 128) return CONVROT_EUNSUPPORTED;
+    if (K % 64 != 0 || K > 32768 || (block > 1 && K % block != 0)) return CONVROT_EINVAL;
+    if (ldx < K || (ldx * in_elem_bytes) % 16 != 0) return CONVROT_EINVAL;
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u) != 0) return CONVROT_EINVAL;
+    const DeviceInfo* d = device_info();
+    if (!d) return CONVROT_ECUDA;
+    if (!d->supported) return CONVROT_EUNSUPPORTED;
+    RqGeometry g;
+    if (!rq_geometry(K, in_elem_bytes, &g)) return CONVROT_EINVAL;
+    CUtensorMap xmap;
+    const uint32_t inner = 128u / static_cast<uint32_t>(in_elem_bytes);
+    const CUtensorMapDataType dt =
+        in_elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (!encode_3d(&xmap, dt, x, inner, static_cast<uint64_t>(g.rows128), static_cast<uint64_t>(M), 128,
+                   static_cast<uint64_t>(ldx) * in_elem_bytes, inner, static_cast<uint32_t>(g.box1),
+                   static_cast<uint32_t>(g.rows_per_cta), CU_TENSOR_MAP_SWIZZLE_128B))
+        return CONVROT_ECUDA;
+    return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, block, M, K, g, q, K, s, g_limit_ns.load(),
+                                           d->err, stream));
+}
+
+convrot_status check_desc(const convrot_wdesc* desc) {
+    if (!desc) return CONVROT_EINVAL;
+    if (desc->magic != CONVROT_WDESC_MAGIC || desc->version != CONVROT_WDESC_VERSION ||
+        desc->layout != CONVROT_LAYOUT_OUTPUT_MAJOR)
+        return CONVROT_ELAYOUT;
+    if (desc->N <= 0 || desc->N > kMaxI32 || desc->K <= 0 || desc->K % 16 != 0 || desc->K > kMaxI32)
+        return CONVROT_ELAYOUT;
+    if (desc->block != 0 && desc->block != 1 && desc->block != 128) return CONVROT_ELAYOUT;
+    return CONVROT_OK;
+}
+
+// GEMM + epilogue over [batch][M][K] x [batch][N][K] -> [batch][M][N].
+convrot_status gemm(const int8_t* qa, const int8_t* qb, const float* sa, const float* sb, const float* bias,
+                    float alpha, int epi, int64_t batch, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
+                    bool pdl, cudaStream_t stream) {
+    const DeviceInfo* d = device_info();
+    if (!d) return CONVROT_ECUDA;
+    if (!d->supported) return CONVROT_EUNSUPPORTED;
+    const bool s32 = epi == kEpiS32;
+    const int ebytes = s32 ? 4 : 2;
+    CUtensorMap amap, bmap, ymap;
+    if (!encode_3d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                   static_cast<uint64_t>(batch), static_cast<uint64_t>(K), static_cast<uint64_t>(M * K), kGemmBK,
+                   kGemmBM, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+        return CONVROT_ECUDA;
+    if (!encode_3d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                   static_cast<uint64_t>(batch), static_cast<uint64_t>(K), static_cast<uint64_t>(N * K), kGemmBK,
+                   kGemmBN, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+        return CONVROT_ECUDA;
+    if (!encode_3d(&ymap, s32 ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y,
+                   static_cast<uint64_t>(N), static_cast<uint64_t>(M), static_cast<uint64_t>(batch),
+                   static_cast<uint64_t>(ldy) * ebytes, static_cast<uint64_t>(M * ldy) * ebytes, kEpiCols, kEpiRows,
+                   1, s32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+        return CONVROT_ECUDA;
+    GemmArgs a;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.batch = static_cast<int>(batch);
+    a.s_a = sa;
+    a.s_b = sb;
+    a.bias = bias;
+    a.alpha = alpha;
+    a.limit_ns = g_limit_ns.load();
+    a.err = d->err;
+    return cuda_status(launch_igemm(amap, bmap, ymap, a, epi, d->num_sms, pdl, stream));
+}
+
+float alpha_for_block(int32_t block) { return block > 1 ? 1.0f / static_cast<float>(block) : 1.0f; }
+
+bool tiles_fit_int(int64_t batch, int64_t M, int64_t N) {
+    const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + kGemmBN - 1) / kGemmBN) * batch;
+    return tiles <= kMaxI32;
+}
+
+convrot_status linear_checks(const int8_t* qw, const float* s_w, const convrot_wdesc* desc, int32_t epilogue,
+                             int64_t M, const void* y, int64_t ldy, const float* bias) {
+    convrot_status st = check_desc(desc);
+    if (st != CONVROT_OK) return st;
+    if (!qw || !s_w || !y) return CONVROT_EINVAL;
+    if (epilogue != CONVROT_EPI_NONE && epilogue != CONVROT_EPI_GELU) return CONVROT_EINVAL;
+    if (M <= 0 || M > kMaxI32 || !tiles_fit_int(1, M, desc->N)) return CONVROT_EINVAL;
+    if (ldy < desc->N || ldy % 8 != 0) return CONVROT_EINVAL;
+    if (!aligned16(qw) || !aligned16(y) || (reinterpret_cast<uintptr_t>(s_w) & 3u) != 0) return CONVROT_EINVAL;
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u) != 0) return CONVROT_EINVAL;
+    return CONVROT_OK;
+}
+
+}  // namespace
+}  // namespace convrot
+
+using namespace convrot;
+
+extern "C" {
+
+const char* convrot_status_string(int status) {
+    switch (status) {
+        case CONVROT_OK: return "ok";
+        case CONVROT_EINVAL: return "invalid argument";
+        case CONVROT_EUNSUPPORTED: return "unsupported (block size or device)";
+        case CONVROT_ELAYOUT: return "weight descriptor does not match this library's layout";
+        case CONVROT_ECUDA: return "CUDA call failed";
+        case CONVROT_ETIMEOUT: return "a device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int convrot_abi_version(void) { return 1; }
+
+void convrot_set_wait_limit_ns(uint64_t ns) { g_limit_ns.store(ns == 0 ? kDefaultLimitNs : ns); }
+
+convrot_status convrot_pack_weight(const float* w, int64_t N, int64_t K, int32_t block, int8_t* q, float* s_w,
+                                   convrot_wdesc* desc, void* stream) {
+    if (!desc) return CONVROT_EINVAL;
+    convrot_status st = rotate_quant(w, 4, N, K, K, block, q, s_w, static_cast<cudaStream_t>(stream));
+    if (st != CONVROT_OK) return st;
+    desc->magic = CONVROT_WDESC_MAGIC;
+    desc->version = CONVROT_WDESC_VERSION;
+    desc->layout = CONVROT_LAYOUT_OUTPUT_MAJOR;
+    desc->block = block > 1 ? block : 0;
+    desc->N = N;
+    desc->K = K;
+    return CONVROT_OK;
+}
+
+convrot_status convrot_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int32_t block,
+                                    int8_t* q, float* s_x, void* stream) {
+    return rotate_quant(x, 2, M, K, ldx, block, q, s_x, static_cast<cudaStream_t>(stream));
+}
+
+convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int8_t* qw, const float* s_w,
+                                   const convrot_wdesc* desc, const float* bias, int32_t epilogue, int64_t M,
+                                   uint16_t* y, int64_t ldy, void* stream) {
+    convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y, ldy, bias);
+    if (st != CONVROT_OK) return st;
+    if (!qx || !s_x || !aligned16(qx) || (reinterpret_cast<uintptr_t>(s_x) & 3u) != 0) return CONVROT_EINVAL;
+    return gemm(qx, qw, s_x, s_w, bias, alpha_for_block(desc->block),
+                epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16, 1, M, desc->N, desc->K, y, ldy, false,
+                static_cast<cudaStream_t>(stream));
+}
+
+size_t convrot_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) + round256(static_cast<size_t>(M) * 4);
+}
+
+convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
+                                    const convrot_wdesc* desc, const float* bias, int32_t epilogue,
+                                    void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy, void* stream) {
+    convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y, ldy, bias);
+    if (st != CONVROT_OK) return st;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CONVROT_EINVAL;
+    if (ws_bytes < convrot_workspace_bytes(M, desc->K)) return CONVROT_EINVAL;
+    int8_t* qx = static_cast<int8_t*>(workspace);
+    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         round256(static_cast<size_t>(M) * static_cast<size_t>(desc->K)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = rotate_quant(x, 2, M, desc->K, ldx, desc->block, qx, sx, s);
+    if (st != CONVROT_OK) return st;
+    return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block),
+                epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16, 1, M, desc->N, desc->K, y, ldy, true, s);
+}
+
+convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, const int8_t* qw, const float* s_w,
+                                         const convrot_wdesc* desc, const float* bias, int32_t epilogue,
+                                         uint16_t* x_dev, void* workspace, size_t ws_bytes, uint16_t* y_dev,
+                                         uint16_t* y_host, void* stream) {
+    convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y_dev, desc ? desc->N : 0, bias);
+    if (st != CONVROT_OK) return st;
+    if (!x_host || !y_host || !x_dev || !aligned16(x_dev)) return CONVROT_EINVAL;
+    if (desc->N % 8 != 0) return CONVROT_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t xbytes = static_cast<size_t>(M) * static_cast<size_t>(desc->K) * 2;
+    const size_t ybytes = static_cast<size_t>(M) * static_cast<size_t>(desc->N) * 2;
+    if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return CONVROT_ECUDA;
+    st = convrot_linear_fused(x_dev, M, desc->K, qw, s_w, desc, bias, epilogue, workspace, ws_bytes, y_dev,
+                              desc->N, stream);
+    if (st != CONVROT_OK) return st;
+    if (cudaMemcpyAsync(y_host, y_dev, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return CONVROT_ECUDA;
+    return CONVROT_OK;
+}
+
+convrot_status convrot_w8a8_bmm(const int8_t* qa, const float* sa, const int8_t* qb, const float* sb,
+                                int64_t batch, int64_t M, int64_t N, int64_t K, uint16_t* y, void* stream) {
+    if (!qa || !sa || !qb || !sb || !y) return CONVROT_EINVAL;
+    if (batch <= 0 || M <= 0 || N <= 0 || K <= 0 || K % 16 != 0 || N % 8 != 0) return CONVROT_EINVAL;
+    if (batch > kMaxI32 || M > kMaxI32 || N > kMaxI32 || K > kMaxI32 || !tiles_fit_int(batch, M, N))
+        return CONVROT_EINVAL;
+    if (!aligned16(qa) || !aligned16(qb) || !aligned16(y)) return CONVROT_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(sa) & 3u) != 0 || (reinterpret_cast<uintptr_t>(sb) & 3u) != 0)
+        return CONVROT_EINVAL;
+    return gemm(qa, qb, sa, sb, nullptr, 1.0f, kEpiBf16, batch, M, N, K, y, N, false,
+                static_cast<cudaStream_t>(stream));
+}
+
+convrot_status convrot_igemm_s32(const int8_t* qa, const int8_t* qb, int64_t batch, int64_t M, int64_t N, int64_t K,
+                                 int32_t* acc, void* stream) {
+    if (!qa || !qb || !acc) return CONVROT_EINVAL;
+    if (batch <= 0 || M <= 0 || N <= 0 || K <= 0 || K % 16 != 0 || N % 4 != 0) return CONVROT_EINVAL;
+    if (batch > kMaxI32 || M > kMaxI32 || N > kMaxI32 || K > kMaxI32 || !tiles_fit_int(batch, M, N))
+        return CONVROT_EINVAL;
+    if (!aligned16(qa) || !aligned16(qb) || !aligned16(acc)) return CONVROT_EINVAL;
+    return gemm(qa, qb, nullptr, nullptr, nullptr, 1.0f, kEpiS32, batch, M, N, K, acc, N, false,
+                static_cast<cudaStream_t>(stream));
+}
+
+convrot_status convrot_last_device_status(void* stream, uint32_t* code) {
+    if (code) *code = 0;
+    const DeviceInfo* d = device_info();
+    if (!d) return CONVROT_ECUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONVROT_ECUDA;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, d->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return CONVROT_ECUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(d->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return CONVROT_ECUDA;
+    }
+    if (code) *code = v;
+    return v ? CONVROT_ETIMEOUT : CONVROT_OK;
+}
+
+convrot_status convrot_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+    const DeviceInfo* d = device_info();
+    if (!d) return CONVROT_ECUDA;
+    if (!d->supported) return CONVROT_EUNSUPPORTED;
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return CONVROT_EINVAL;
+    return cuda_status(launch_wait_selftest(limit_ns, d->err, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// kernels.h -- host-side launchers of the sm_100a kernels (internal to the
+// library; the public surface is include/convrot.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace convrot {
+
+// ---------------------------------------------------------------- rotate + quantise
+
+// Launch geometry of the rotate+quantise kernel for one row length.
+struct RqGeometry {
+    int tpr;           // threads holding data in one row (K / 32)
+    int tpr_pad;       // threads per row including idle ones
+    int rows_per_cta;  // rows one CTA handles
+    int threads;       // CTA size
+    int rows128;       // 128-byte shared-memory rows per input row
+    int box1;          // TMA box extent along the 128-byte-row dimension
+    int nbox;          // TMA boxes per input row
+    size_t smem_bytes; // dynamic shared memory requested
+};
+
+// in_elem_bytes: 2 for bf16 activations, 4 for f32 weights.
+bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g);
+
+// x: bf16 (bits) or f32 rows, described by `xmap` (3D: 128-byte inner rows,
+// rows128, M) with 128-byte swizzling.  block: 0/1 (no rotation) or 128.
+cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int block, int64_t M, int64_t K,
+                                const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
+                                unsigned int* err, cudaStream_t stream);
+
+// One CTA waits on an mbarrier that nothing arrives on, so its bounded wait
+// must give up after `limit_ns` and record kErrTimeoutSelfTest.
+cudaError_t launch_wait_selftest(uint64_t limit_ns, unsigned int* err, cudaStream_t stream);
+
+// ---------------------------------------------------------------- int8 GEMM
+
+enum EpilogueKind : int {
+    kEpiBf16 = 0,      // y = acc * s_a[m] * s_b[n] * alpha + bias[n] -> bf16
+    kEpiBf16Gelu = 1,  // same, then exact-erf GELU
+    kEpiS32 = 2,       // raw int32 accumulators
+};
+
+struct GemmArgs {
+    int M, N, K, batch;
+    const float* s_a;   // [batch * M] (bf16 epilogues)
+    const float* s_b;   // [batch * N] (bf16 epilogues)
+    const float* bias;  // [N] or null
+    float alpha;        // 1/b for a rotated pair, else 1
+    uint64_t limit_ns;  // bound on every wait
+    unsigned int* err;  // device error word
+};
+
+// amap: int8 [batch][M][K]; bmap: int8 [batch][N][K]; ymap: output
+// [batch][M][N] (bf16, or int32 for kEpiS32).  `pdl` lets the kernel start
+// while the previous kernel on the stream drains.
+cudaError_t launch_igemm(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
+                         const GemmArgs& a, int epilogue, int num_sms, bool pdl, cudaStream_t stream);
+
+// Box sizes the GEMM's tensor maps must use.
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 128;     // bytes of K per stage (= int8 elements)
+constexpr int kEpiCols = 32;     // output columns per epilogue store
+constexpr int kEpiRows = 32;     // rows per epilogue store (one warp)
+
+}  // namespace convrot
