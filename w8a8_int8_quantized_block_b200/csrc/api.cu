@@ -112,7 +112,7 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
                    static_cast<uint32_t>(g.rows_per_cta), CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
     return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, block, M, K, g, q, K, s, g_limit_ns.load(),
-                                           d->err, stream));
+                                           d->err, d->num_sms, stream));
 }
 
 convrot_status check_desc(const convrot_wdesc* desc) {

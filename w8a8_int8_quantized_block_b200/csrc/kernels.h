@@ -19,6 +19,7 @@ struct RqGeometry {
     int rows128;       // 128-byte shared-memory rows per input row
     int box1;          // TMA box extent along the 128-byte-row dimension
     int nbox;          // TMA boxes per input row
+    int nstage;        // shared-memory ring slots (row groups in flight per CTA)
     size_t smem_bytes; // dynamic shared memory requested
 };
 
@@ -29,7 +30,7 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g);
 // rows128, M) with 128-byte swizzling.  block: 0/1 (no rotation) or 128.
 cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int block, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
-                                unsigned int* err, cudaStream_t stream);
+                                unsigned int* err, int num_sms, cudaStream_t stream);
 
 // One CTA waits on an mbarrier that nothing arrives on, so its bounded wait
 // must give up after `limit_ns` and record kErrTimeoutSelfTest.

@@ -11,13 +11,28 @@
 //   z = blockdiag(H_128) x            (fp32 butterflies, stages 1, 2, ..., 64)
 //   amax = max |z|;  s = amax / 127;  q = clamp(rne(z * (127 / amax)), +-127)
 //
-// Design (B200): one CTA owns `rows_per_cta` rows.  A single TMA load brings
-// the rows into shared memory with 128-byte swizzling, so every thread's
-// 16-byte reads are bank-conflict free.  Each thread holds 32 consecutive
-// elements in registers: the first five butterfly stages (h = 1..16) run in
-// registers and the last two (h = 32, 64) by shuffles with lanes t^1 and t^2.
-// The row's absmax is reduced by shuffles (and shared memory when a row spans
-// several warps), then each thread writes its 32 codes as one 32-byte store.
+// Design (B200).  A persistent CTA walks over groups of rows; each group is
+// brought into one slot of a 2-3 slot shared-memory ring by TMA (128-byte
+// swizzle, so the 16-byte reads below are bank-conflict free) while the
+// previous group is computed.  Each thread owns 32 consecutive elements of a
+// row, held as 16 packed f32x2 register pairs (element j with element j+16):
+//   - butterfly stages h = 1, 2, 4, 8 are packed add/sub (two lanes of work
+//     per instruction), stage h = 16 is inside each pair;
+//   - stages h = 32 and 64 pair lanes t^1 and t^2: a shuffle brings the
+//     partner's values and one packed FMA with a +-1 sign computes
+//     self + partner on the lower side and partner - self on the upper side,
+//     each rounded once exactly like the add or subtract it replaces;
+//   - the row absmax is reduced with shuffles (and shared memory when a row
+//     spans several warps);
+//   - codes: v = z * (127/amax) (packed multiply, rounded), then a
+//     round-to-nearest-even conversion to int32 (|v| <= 127*(1+2^-24) < 127.5,
+//     so no clamp can bind); byte permutes pack four codes per word and one
+//     32-byte store writes the thread's 32 codes.  (The product must be rounded
+//     on its own before the integer rounding: adding 1.5*2^23 to round was
+//     contracted with the packed multiply into one FMA, which rounds the exact
+//     product instead and moves values that sit within half an ulp of a tie.)
+// The arithmetic is therefore the same sequence of IEEE single-precision
+// operations as the plain definition, in the same order.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -28,176 +43,278 @@ namespace convrot {
 namespace {
 
 constexpr int kPerThread = 32;  // elements each thread owns
+#ifndef CONVROT_RQ_LONG_ROWS
+#define CONVROT_RQ_LONG_ROWS 1  // rows per group when a row spans more than one warp
+#endif
+constexpr int kMaxStages = 3;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     const uint32_t a = smem_u32(p);
     return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// Load this thread's 32 elements from the swizzled stage into registers.
-// `R0` is the index of the 128-byte shared row holding element 0 of the
-// thread's input row.
+// ---- packed single-precision pairs (one 64-bit register pair)
+
+__device__ __forceinline__ uint64_t pk(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Load this thread's 32 elements from the swizzled slot into pairs
+// P[j] = (element j, element j + 16).  `R0` is the 128-byte shared row holding
+// element 0 of the thread's input row.
 template <typename Tin>
-__device__ __forceinline__ void load_row_piece(const uint8_t* stage, int R0, int t, float (&v)[kPerThread]) {
+__device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, uint64_t (&P)[16]) {
     if constexpr (sizeof(Tin) == 2) {
         // 32 bf16 = 64 bytes = half of a 128-byte row: row t/2, chunks 4*(t&1) .. +3
         const int R = R0 + (t >> 1);
         const int c0 = (t & 1) * 4;
+        uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint4 w = *reinterpret_cast<const uint4*>(stage + R * 128 + (((c0 + j) ^ (R & 7)) << 4));
-            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            const uint4 v = *reinterpret_cast<const uint4*>(slot + R * 128 + (((c0 + j) ^ (R & 7)) << 4));
+            w[4 * j] = v.x;
+            w[4 * j + 1] = v.y;
+            w[4 * j + 2] = v.z;
+            w[4 * j + 3] = v.w;
+        }
+        // word k holds elements 2k (low half) and 2k+1 (high half)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[8 * j + 2 * i] = __uint_as_float(u[i] << 16);
-                v[8 * j + 2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
-            }
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t lo = w[j >> 1], hi = w[8 + (j >> 1)];
+            const float a = __uint_as_float((j & 1) ? (lo & 0xFFFF0000u) : (lo << 16));
+            const float b = __uint_as_float((j & 1) ? (hi & 0xFFFF0000u) : (hi << 16));
+            P[j] = pk(a, b);
         }
     } else {
         // 32 f32 = one whole 128-byte row: row t, chunks 0..7
         const int R = R0 + t;
+        float e[32];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 w = *reinterpret_cast<const float4*>(stage + R * 128 + ((j ^ (R & 7)) << 4));
-            v[4 * j + 0] = w.x;
-            v[4 * j + 1] = w.y;
-            v[4 * j + 2] = w.z;
-            v[4 * j + 3] = w.w;
+            const float4 v = *reinterpret_cast<const float4*>(slot + R * 128 + ((j ^ (R & 7)) << 4));
+            e[4 * j] = v.x;
+            e[4 * j + 1] = v.y;
+            e[4 * j + 2] = v.z;
+            e[4 * j + 3] = v.w;
         }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) P[j] = pk(e[j], e[j + 16]);
     }
 }
 
-// Stages h = 1, 2, 4, 8, 16 of the 128-point transform, on the thread's
-// 32 consecutive elements.  Each butterfly (u, w) -> (u + w, u - w).
-__device__ __forceinline__ void fwht_in_registers(float (&v)[kPerThread]) {
+// Stages h = 1, 2, 4, 8 (packed, both halves at once) then h = 16 (inside
+// each pair).  Butterfly (u, w) -> (u + w, u - w), u the lower index.
+__device__ __forceinline__ void fwht_in_registers(uint64_t (&P)[16]) {
 #pragma unroll
-    for (int h = 1; h < kPerThread; h <<= 1) {
+    for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
-        for (int e = 0; e < kPerThread; ++e) {
-            if ((e & h) == 0) {
-                const float u = v[e];
-                const float w = v[e + h];
-                v[e] = __fadd_rn(u, w);
-                v[e + h] = __fsub_rn(u, w);
+        for (int j = 0; j < 16; ++j) {
+            if ((j & h) == 0) {
+                const uint64_t u = P[j], w = P[j + h];
+                P[j] = add2(u, w);
+                P[j + h] = sub2(u, w);
             }
         }
     }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        float u, w;
+        upk(P[j], u, w);
+        P[j] = pk(__fadd_rn(u, w), __fsub_rn(u, w));
+    }
 }
 
-// Stage across lanes: the partner lane (lane ^ sh) holds the elements `sh*32`
-// positions away.  The lower-index side keeps u + w, the upper side u - w,
-// where u is always the lower-index element.
-__device__ __forceinline__ void fwht_across_lanes(float (&v)[kPerThread], int sh, bool upper) {
+// Stage across lanes: the partner (lane ^ sh) holds the elements sh*32
+// positions away.  sign = +1 on the lower side (self + partner), -1 on the
+// upper side (partner - self); fma(sign, self, partner) rounds once, exactly
+// like that add or subtract.
+__device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[16], int sh, bool upper) {
+    const float sg = upper ? -1.0f : 1.0f;
+    const uint64_t S = pk(sg, sg);
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-        const float p = __shfl_xor_sync(0xFFFFFFFFu, v[e], sh);
-        v[e] = upper ? __fsub_rn(p, v[e]) : __fadd_rn(v[e], p);
+    for (int j = 0; j < 16; ++j) {
+        float a, b;
+        upk(P[j], a, b);
+        const float pa = __shfl_xor_sync(0xFFFFFFFFu, a, sh);
+        const float pb = __shfl_xor_sync(0xFFFFFFFFu, b, sh);
+        P[j] = fma2(S, P[j], pk(pa, pb));
     }
 }
 
 template <typename Tin, int BLOCK>
 __global__ void __launch_bounds__(1024) rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
-                                                            int K, int tpr, int tpr_pad, int rows_per_cta,
-                                                            int rows128, int box1, int nbox, int8_t* __restrict__ q,
-                                                            int64_t ldq, float* __restrict__ s,
-                                                            uint64_t limit_ns, unsigned int* err) {
+                                                            int tpr, int tpr_pad, int rows_per_cta, int rows128,
+                                                            int box1, int nbox, int nstage, int64_t num_groups,
+                                                            int8_t* __restrict__ q, int64_t ldq,
+                                                            float* __restrict__ s, uint64_t limit_ns,
+                                                            unsigned int* err) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bar;
-    __shared__ float red[32];
+    __shared__ uint64_t full[kMaxStages];
+    __shared__ float red[2][32];  // warp maxima, double-buffered across iterations
     __shared__ int abort_flag;
-    uint8_t* stage = align1024(smem_raw);
+    uint8_t* ring = align1024(smem_raw);
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
     const int rloc = tid / tpr_pad;
     const int t = tid - rloc * tpr_pad;
+    const uint32_t slot_bytes = static_cast<uint32_t>(nbox) * box1 * 128u * rows_per_cta;
+    const int row_pitch = nbox * box1;  // 128-byte shared rows between consecutive input rows of a group
+    (void)rows128;
+
+    auto issue = [&](int64_t g, int slot) {
+        // Full boxes are credited even where they run past the tensor (zero fill).
+        mbar_arrive_expect_tx(&full[slot], slot_bytes);
+        uint8_t* dst = ring + static_cast<size_t>(slot) * slot_bytes;
+        for (int b = 0; b < nbox; ++b)
+            tma_load_3d(dst + static_cast<size_t>(b) * box1 * 128, &xmap, &full[slot], 0, b * box1,
+                        static_cast<int>(g * rows_per_cta));
+    };
 
     if (tid == 0) {
         abort_flag = 0;
-        mbar_init(&bar, 1);
+        for (int i = 0; i < nstage; ++i) mbar_init(&full[i], 1);
         fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-        // Full boxes are credited even where they run past the tensor (zero fill).
-        const uint32_t bytes = static_cast<uint32_t>(nbox) * box1 * 128u * rows_per_cta;
-        mbar_arrive_expect_tx(&bar, bytes);
-        for (int b = 0; b < nbox; ++b)
-            tma_load_3d(stage + static_cast<size_t>(b) * box1 * 128, &xmap, &bar, 0, b * box1,
-                        static_cast<int>(row0));
-        if (!mbar_wait_bounded(&bar, 0, limit_ns, kErrTimeoutLoad, err)) abort_flag = 1;
-    }
-    __syncthreads();
-    if (abort_flag) return;  // uniform across the CTA
-
-    float v[kPerThread];
-    if (t < tpr) {
-        load_row_piece<Tin>(stage, rloc * rows128, t, v);
-    } else {
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) v[e] = 0.0f;
-    }
-
-    if constexpr (BLOCK == 128) {
-        fwht_in_registers(v);
-        fwht_across_lanes(v, 1, (t & 1) != 0);  // h = 32
-        fwht_across_lanes(v, 2, (t & 2) != 0);  // h = 64
-    }
-
-    float amax = 0.0f;
-#pragma unroll
-    for (int e = 0; e < kPerThread; ++e) amax = fmaxf(amax, fabsf(v[e]));
-
-    if (tpr_pad <= 32) {
-        for (int o = tpr_pad >> 1; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    } else {
-        // one row per CTA: warp maxima through shared memory
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        if (lane == 0) red[warp] = amax;
-        __syncthreads();
-        const int nw = tpr_pad >> 5;
-        amax = red[0];
-        for (int i = 1; i < nw; ++i) amax = fmaxf(amax, red[i]);
-    }
-
-    const int64_t row = row0 + rloc;
-    if (row >= M || t >= tpr) return;
-
-    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-    uint32_t packed[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            int c = __float2int_rn(__fmul_rn(v[4 * w + b], inv));
-            c = max(-127, min(127, c));
-            word |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * b);
+        for (int i = 0; i < nstage; ++i) {
+            const int64_t g = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+            if (g < num_groups) issue(g, i);
         }
-        packed[w] = word;
     }
-    int8_t* dst = q + row * ldq + static_cast<int64_t>(t) * kPerThread;
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(packed[0]),
-                 "r"(packed[1]), "r"(packed[2]), "r"(packed[3]), "r"(packed[4]), "r"(packed[5]), "r"(packed[6]),
-                 "r"(packed[7])
-                 : "memory");
-    if (t == 0) s[row] = __fdiv_rn(amax, 127.0f);
+    __syncthreads();
+
+    int it = 0;
+    for (int64_t g = blockIdx.x; g < num_groups; g += gridDim.x, ++it) {
+        const int slot = it % nstage;
+        const uint32_t parity = static_cast<uint32_t>(it / nstage) & 1u;
+        // Every thread waits for the slot itself; a time-out is acted on after
+        // the next CTA barrier so that all threads leave the loop together.
+        if (!mbar_wait_bounded(&full[slot], parity, limit_ns, kErrTimeoutLoad, err)) abort_flag = 1;
+
+        uint64_t P[16];
+        if (t < tpr) {
+            load_pairs<Tin>(ring + static_cast<size_t>(slot) * slot_bytes, rloc * row_pitch, t, P);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) P[j] = 0ull;
+        }
+
+        if constexpr (BLOCK == 128) {
+            fwht_in_registers(P);
+            fwht_across_lanes(P, 1, (t & 1) != 0);  // h = 32
+            fwht_across_lanes(P, 2, (t & 2) != 0);  // h = 64
+        }
+
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float a, b;
+            upk(P[j], a, b);
+            amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+        }
+        float* rbuf = red[it & 1];
+        if (tpr_pad <= 32) {
+            for (int o = tpr_pad >> 1; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        } else {
+            // rows span whole warps: warp maxima through shared memory
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            if (lane == 0) rbuf[warp] = amax;
+        }
+        // The one CTA barrier per group: every thread has read the slot (so it
+        // can be refilled) and has published its warp maximum.
+        __syncthreads();
+        if (abort_flag) break;  // uniform across the CTA
+        if (tid == 0) {
+            const int64_t gn = g + static_cast<int64_t>(nstage) * gridDim.x;
+            if (gn < num_groups) {
+                fence_proxy_async_smem();
+                issue(gn, slot);
+            }
+        }
+        if (tpr_pad > 32) {
+            const int nw = tpr_pad >> 5;  // warps per row
+            amax = rbuf[rloc * nw];
+            for (int i = 1; i < nw; ++i) amax = fmaxf(amax, rbuf[rloc * nw + i]);
+        }
+
+        const int64_t row = g * rows_per_cta + rloc;
+        if (row < M && t < tpr) {
+            const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+            const uint64_t inv2 = pk(inv, inv);
+            uint32_t lo[16], hi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float a, b;
+                upk(mul2(P[j], inv2), a, b);
+                lo[j] = static_cast<uint32_t>(__float2int_rn(a));
+                hi[j] = static_cast<uint32_t>(__float2int_rn(b));
+            }
+            uint32_t word[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                word[i] = prmt(prmt(lo[4 * i], lo[4 * i + 1], 0x0040u), prmt(lo[4 * i + 2], lo[4 * i + 3], 0x0040u),
+                               0x5410u);
+                word[4 + i] = prmt(prmt(hi[4 * i], hi[4 * i + 1], 0x0040u),
+                                   prmt(hi[4 * i + 2], hi[4 * i + 3], 0x0040u), 0x5410u);
+            }
+            int8_t* dst = q + row * ldq + static_cast<int64_t>(t) * kPerThread;
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(word[0]),
+                         "r"(word[1]), "r"(word[2]), "r"(word[3]), "r"(word[4]), "r"(word[5]), "r"(word[6]),
+                         "r"(word[7])
+                         : "memory");
+            if (t == 0) s[row] = __fdiv_rn(amax, 127.0f);
+        }
+    }
 }
 
 template <typename Tin, int BLOCK>
-cudaError_t launch_typed(const CUtensorMap& xmap, int64_t M, int64_t K, const RqGeometry& g, int8_t* q,
-                         int64_t ldq, float* s, uint64_t limit_ns, unsigned int* err, cudaStream_t stream) {
+cudaError_t launch_typed(const CUtensorMap& xmap, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
+                         float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
     auto kern = rotate_quant_kernel<Tin, BLOCK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(g.smem_bytes));
     if (e != cudaSuccess) return e;
-    const int64_t grid = (M + g.rows_per_cta - 1) / g.rows_per_cta;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem_bytes);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t groups = (M + g.rows_per_cta - 1) / g.rows_per_cta;
+    const int64_t cap = static_cast<int64_t>(per_sm) * num_sms;
+    const int64_t grid = groups < cap ? groups : cap;
     kern<<<static_cast<unsigned>(grid), g.threads, g.smem_bytes, stream>>>(
-        xmap, M, static_cast<int>(K), g.tpr, g.tpr_pad, g.rows_per_cta, g.rows128, g.box1, g.nbox, q, ldq, s,
-        limit_ns, err);
+        xmap, M, g.tpr, g.tpr_pad, g.rows_per_cta, g.rows128, g.box1, g.nbox, g.nstage, groups, q, ldq, s, limit_ns,
+        err);
     return cudaGetLastError();
 }
 
@@ -213,38 +330,46 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
     if (K <= 0 || K % 64 != 0 || K > 32768) return false;
     if ((K * in_elem_bytes) % 128 != 0) return false;
     g->tpr = static_cast<int>(K / kPerThread);
+    g->rows128 = static_cast<int>(K * in_elem_bytes / 128);
     if (g->tpr <= 32) {
+        // Short rows: a power-of-two lane group per row, 256 threads per CTA.
         g->tpr_pad = next_pow2(g->tpr);
         g->rows_per_cta = 256 / g->tpr_pad;
+        g->nbox = 1;
+        g->box1 = g->rows128;  // <= 32; the slot size is a multiple of 1024 bytes
     } else {
+        // Long rows: whole warps per row; boxes padded to 8 rows of 128 bytes
+        // so every box and slot starts on a 1024-byte boundary.
         g->tpr_pad = (g->tpr + 31) / 32 * 32;
-        g->rows_per_cta = 1;
+        g->nbox = (g->rows128 + 255) / 256;
+        const int per = (g->rows128 + g->nbox - 1) / g->nbox;
+        g->box1 = (per + 7) / 8 * 8;
+        if (g->box1 > 256) return false;
+        // Several rows per group share the CTA's barriers (at most 1024 threads).
+        g->rows_per_cta = g->nbox == 1 ? CONVROT_RQ_LONG_ROWS : 1;
+        while (g->rows_per_cta > 1 && g->tpr_pad * g->rows_per_cta > 1024) --g->rows_per_cta;
     }
     g->threads = g->tpr_pad * g->rows_per_cta;
-    g->rows128 = static_cast<int>(K * in_elem_bytes / 128);
-    if (g->rows_per_cta > 1) {
-        g->nbox = 1;
-        g->box1 = g->rows128;  // <= 32 here
-    } else {
-        g->nbox = (g->rows128 + 255) / 256;
-        int per = (g->rows128 + g->nbox - 1) / g->nbox;
-        g->box1 = (per + 7) / 8 * 8;  // keep every box 1024-byte aligned
-        if (g->box1 > 256) return false;
-    }
-    const size_t stage = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
-    g->smem_bytes = stage + 1024;  // slack for 1024-byte alignment
-    return g->smem_bytes <= 200 * 1024;
+    const size_t slot = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
+    if (slot % 1024 != 0) return false;  // slots must stay 1024-byte aligned for the swizzle
+    const size_t budget = 200 * 1024;
+    g->nstage = 3;
+    while (g->nstage > 1 && slot * g->nstage + 1024 > budget) --g->nstage;
+    if (g->nstage == 3 && slot * 3 > 96 * 1024) g->nstage = 2;  // leave room for a second CTA
+    g->smem_bytes = slot * g->nstage + 1024;  // slack for 1024-byte alignment
+    return g->smem_bytes <= budget;
 }
 
 cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int block, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
-                                unsigned int* err, cudaStream_t stream) {
+                                unsigned int* err, int num_sms, cudaStream_t stream) {
+    (void)K;
     const bool rot = block == 128;
     if (in_elem_bytes == 2)
-        return rot ? launch_typed<__nv_bfloat16, 128>(xmap, M, K, g, q, ldq, s, limit_ns, err, stream)
-                   : launch_typed<__nv_bfloat16, 0>(xmap, M, K, g, q, ldq, s, limit_ns, err, stream);
-    return rot ? launch_typed<float, 128>(xmap, M, K, g, q, ldq, s, limit_ns, err, stream)
-               : launch_typed<float, 0>(xmap, M, K, g, q, ldq, s, limit_ns, err, stream);
+        return rot ? launch_typed<__nv_bfloat16, 128>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream)
+                   : launch_typed<__nv_bfloat16, 0>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+    return rot ? launch_typed<float, 128>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream)
+               : launch_typed<float, 0>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
 }
 
 namespace {
