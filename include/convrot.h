@@ -55,7 +55,8 @@ typedef enum convrot_status {
     CONVROT_EUNSUPPORTED = 2,
     CONVROT_ELAYOUT = 3,
     CONVROT_ECUDA = 4,
-    CONVROT_ETIMEOUT = 5
+    CONVROT_ETIMEOUT = 5,
+    CONVROT_ETOOLARGE = 6  /* exceeds the fixed scratch of convrot_linear_fused_noalloc */
 } convrot_status;
 
 /* Packed-weight descriptor.  Plays the role of the pages' "versioned layout
@@ -130,6 +131,29 @@ convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, cons
                                          const convrot_wdesc* desc, const float* bias, int32_t epilogue,
                                          uint16_t* x_dev, void* workspace, size_t ws_bytes, uint16_t* y_dev,
                                          uint16_t* y_host, void* stream);
+
+/* Allocation-free form of convrot_linear_fused, for callers that cannot call
+ * cudaMalloc: a plugin or embedded runtime whose host owns every device
+ * allocation (a pre-planned pool, an ABI that hands out no allocator), or a
+ * per-batch loop that cannot afford cudaMalloc's latency and implicit
+ * device-wide synchronisation.  (The pages have no counterpart; this is a
+ * property of this library's interface, not of the method.)
+ * The caller still passes x and y exactly as for convrot_linear_fused; the
+ * int8 codes and scales go to a scratch array built into the library instead
+ * of a caller workspace.  That array is 32 MiB per device, held by every GPU
+ * that loads the library until the process exits: the call accepts
+ * convrot_workspace_bytes(M, desc->K) <= 33554432 (M <= 6236 at K = 5376) and
+ * returns CONVROT_ETOOLARGE, launching nothing, beyond that.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the previous call's contents
+ * (every byte a call reads was written earlier in the same call, so nothing
+ * needs clearing); calls whose kernels overlap on the GPU (different streams,
+ * or different host threads) race on it and must be serialised by the caller.
+ * Allocates nothing, on the host or the device. */
+convrot_status convrot_linear_fused_noalloc(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw,
+                                            const float* s_w, const convrot_wdesc* desc, const float* bias,
+                                            int32_t epilogue, uint16_t* y, int64_t ldy, void* stream);
 
 /* Batched int8 GEMM with per-row scales on both operands and no rotation:
  * y[b][m][n] = bf16(sum_k qa[b][m][k]*qb[b][n][k] * sa[b*M+m] * sb[b*N+n]).

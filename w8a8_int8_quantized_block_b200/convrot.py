@@ -16,7 +16,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libconvrot.so")
 
-OK, EINVAL, EUNSUPPORTED, ELAYOUT, ECUDA, ETIMEOUT = range(6)
+OK, EINVAL, EUNSUPPORTED, ELAYOUT, ECUDA, ETIMEOUT, ETOOLARGE = range(7)
 EPI_NONE, EPI_GELU = 0, 1
 WDESC_MAGIC = 0x52564E43
 WDESC_VERSION = 1
@@ -27,7 +27,7 @@ EXPORTS = (
     "convrot_status_string", "convrot_abi_version", "convrot_pack_weight", "convrot_quantize_act",
     "convrot_w8a8_linear", "convrot_workspace_bytes", "convrot_linear_fused", "convrot_linear_fused_host",
     "convrot_w8a8_bmm", "convrot_igemm_s32", "convrot_last_device_status", "convrot_set_wait_limit_ns",
-    "convrot_selftest_wait_timeout",
+    "convrot_selftest_wait_timeout", "convrot_linear_fused_noalloc",
 )
 
 
@@ -78,6 +78,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "convrot_last_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
         "convrot_set_wait_limit_ns": ([U64], None),
         "convrot_selftest_wait_timeout": ([U64, P], ctypes.c_int),
+        "convrot_linear_fused_noalloc": ([P, I64, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, I64, P],
+                                         ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -184,6 +186,23 @@ def linear_fused(x: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = 
     _check("convrot_linear_fused", load().convrot_linear_fused(
         _ptr(x), M, x.stride(0), _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias),
         EPI_GELU if gelu else EPI_NONE, _ptr(ws), ws.numel(), _ptr(y), y.stride(0), _stream(stream)))
+    return y
+
+
+def linear_fused_noalloc(x: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None, gelu: bool = False,
+                         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The fused linear without a workspace, for callers that cannot allocate
+    device scratch (the codes and scales go to the library's fixed 32 MiB
+    array; the output tensor is still the caller's).  Raises ConvrotError with
+    status ETOOLARGE beyond that size.  Calls that overlap on the GPU race."""
+    _need(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    M = x.shape[0]
+    y = torch.empty((M, pw.N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("convrot_linear_fused_noalloc", load().convrot_linear_fused_noalloc(
+        _ptr(x), M, x.stride(0), _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias),
+        EPI_GELU if gelu else EPI_NONE, _ptr(y), y.stride(0), _stream(stream)))
     return y
 
 

@@ -198,6 +198,7 @@ const char* convrot_status_string(int status) {
         case CONVROT_ELAYOUT: return "weight descriptor does not match this library's layout";
         case CONVROT_ECUDA: return "CUDA call failed";
         case CONVROT_ETIMEOUT: return "a device-side wait timed out";
+        case CONVROT_ETOOLARGE: return "problem exceeds the fixed scratch of the allocation-free entry point";
         default: return "unknown status";
     }
 }
@@ -275,6 +276,53 @@ convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, cons
     if (st != CONVROT_OK) return st;
     if (cudaMemcpyAsync(y_host, y_dev, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return CONVROT_ECUDA;
     return CONVROT_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free fused linear
+//
+// For callers that cannot allocate device memory (see the header): the codes
+// and scales that convrot_linear_fused keeps in the caller's workspace live in
+// this fixed array instead.  Host code must not hand `g_noalloc_scratch`
+// itself to a kernel -- on the host that name is only a stand-in for the
+// device symbol -- so its device address is looked up once per device.
+namespace convrot {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on the
+// first call per device, with that device current), or null on failure.
+void* noalloc_scratch() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace convrot
+
+extern "C" {
+
+convrot_status convrot_linear_fused_noalloc(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw,
+                                            const float* s_w, const convrot_wdesc* desc, const float* bias,
+                                            int32_t epilogue, uint16_t* y, int64_t ldy, void* stream) {
+    convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y, ldy, bias);
+    if (st != CONVROT_OK) return st;
+    if (convrot_workspace_bytes(M, desc->K) > kNoAllocScratchBytes) return CONVROT_ETOOLARGE;
+    void* scratch = noalloc_scratch();
+    if (scratch == nullptr) return CONVROT_ECUDA;
+    return convrot_linear_fused(x, M, ldx, qw, s_w, desc, bias, epilogue, scratch, kNoAllocScratchBytes, y, ldy,
+                                stream);
 }
 
 convrot_status convrot_w8a8_bmm(const int8_t* qa, const float* sa, const int8_t* qb, const float* sb,
