@@ -14,20 +14,21 @@
 // Design (B200).  A persistent CTA walks over groups of rows; each group is
 // brought into one slot of a 2-3 slot shared-memory ring by TMA (128-byte
 // swizzle, so the 16-byte reads below are bank-conflict free) while the
-// previous group is computed.  Each thread owns 32 consecutive elements of a
-// row, held as 16 packed f32x2 register pairs (element j with element j+16):
-//   - butterfly stages h = 1, 2, 4, 8 are packed add/sub (two lanes of work
-//     per instruction), stage h = 16 is inside each pair;
-//   - stages h = 32 and 64 pair lanes t^1 and t^2: a shuffle brings the
-//     partner's values and one packed FMA with a +-1 sign computes
-//     self + partner on the lower side and partner - self on the upper side,
-//     each rounded once exactly like the add or subtract it replaces;
+// previous group is computed.  Each thread owns 64 consecutive elements of a
+// row (half a Hadamard block), held as 32 packed f32x2 register pairs
+// (element j with element j+32):
+//   - butterfly stages h = 1, 2, 4, 8, 16 are packed add/sub (two lanes of
+//     work per instruction), stage h = 32 is inside each pair;
+//   - stage h = 64 pairs lanes t and t^1: a shuffle brings the partner's
+//     values and one packed FMA with a +-1 sign computes self + partner on
+//     the lower side and partner - self on the upper side, each rounded once
+//     exactly like the add or subtract it replaces;
 //   - the row absmax is reduced with shuffles (and shared memory when a row
 //     spans several warps);
 //   - codes: v = z * (127/amax) (packed multiply, rounded), then a
 //     round-to-nearest-even conversion to int32 (|v| <= 127*(1+2^-24) < 127.5,
-//     so no clamp can bind); byte permutes pack four codes per word and one
-//     32-byte store writes the thread's 32 codes.  (The product must be rounded
+//     so no clamp can bind); byte permutes pack four codes per word and two
+//     32-byte stores write the thread's 64 codes.  (The product must be rounded
 //     on its own before the integer rounding: adding 1.5*2^23 to round was
 //     contracted with the packed multiply into one FMA, which rounds the exact
 //     product instead and moves values that sit within half an ulp of a tie.)
@@ -42,7 +43,14 @@ namespace convrot {
 
 namespace {
 
-constexpr int kPerThread = 32;  // elements each thread owns
+#ifndef CONVROT_RQ_EPT
+#define CONVROT_RQ_EPT 64  // elements each thread owns (32 or 64)
+#endif
+constexpr int kPerThread = CONVROT_RQ_EPT;
+static_assert(kPerThread == 32 || kPerThread == 64, "32 or 64 elements per thread");
+constexpr int kPairs = kPerThread / 2;          // P[j] = (element j, element j + kPairs)
+constexpr int kLanesPerBlock = 128 / kPerThread;  // lanes sharing one Hadamard block
+constexpr int kMaxThreads = kPerThread == 32 ? 1024 : 512;
 #ifndef CONVROT_RQ_LONG_ROWS
 #define CONVROT_RQ_LONG_ROWS 1  // rows per group when a row spans more than one warp
 #endif
@@ -89,56 +97,50 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-// Load this thread's 32 elements from the swizzled slot into pairs
-// P[j] = (element j, element j + 16).  `R0` is the 128-byte shared row holding
-// element 0 of the thread's input row.
+// Load this thread's kPerThread consecutive elements from the swizzled slot
+// into pairs P[j] = (element j, element j + kPairs).  `R0` is the 128-byte
+// shared row holding element 0 of the thread's input row.  A 16-byte chunk c
+// of 128-byte row R sits at chunk position c ^ (R & 7) (128-byte swizzle).
 template <typename Tin>
-__device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, uint64_t (&P)[16]) {
-    if constexpr (sizeof(Tin) == 2) {
-        // 32 bf16 = 64 bytes = half of a 128-byte row: row t/2, chunks 4*(t&1) .. +3
-        const int R = R0 + (t >> 1);
-        const int c0 = (t & 1) * 4;
-        uint32_t w[16];
+__device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, uint64_t (&P)[kPairs]) {
+    constexpr int kBytes = kPerThread * static_cast<int>(sizeof(Tin));
+    constexpr int kChunks = kBytes / 16;
+    const int off = t * kBytes;  // byte offset of the thread's span in its row
+    uint32_t w[kBytes / 4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(slot + R * 128 + (((c0 + j) ^ (R & 7)) << 4));
-            w[4 * j] = v.x;
-            w[4 * j + 1] = v.y;
-            w[4 * j + 2] = v.z;
-            w[4 * j + 3] = v.w;
+    for (int c = 0; c < kChunks; ++c) {
+        const int cc = (off >> 4) + c;  // chunk index counted from the row start
+        const int R = R0 + (cc >> 3);
+        const uint4 v = *reinterpret_cast<const uint4*>(slot + R * 128 + (((cc & 7) ^ (R & 7)) << 4));
+        w[4 * c] = v.x;
+        w[4 * c + 1] = v.y;
+        w[4 * c + 2] = v.z;
+        w[4 * c + 3] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        if constexpr (sizeof(Tin) == 2) {
+            // word k holds elements 2k (low half) and 2k+1 (high half)
+            const uint32_t lo = w[j >> 1], hi = w[(j + kPairs) >> 1];
+            a = __uint_as_float((j & 1) ? (lo & 0xFFFF0000u) : (lo << 16));
+            b = __uint_as_float((j & 1) ? (hi & 0xFFFF0000u) : (hi << 16));
+        } else {
+            a = __uint_as_float(w[j]);
+            b = __uint_as_float(w[j + kPairs]);
         }
-        // word k holds elements 2k (low half) and 2k+1 (high half)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint32_t lo = w[j >> 1], hi = w[8 + (j >> 1)];
-            const float a = __uint_as_float((j & 1) ? (lo & 0xFFFF0000u) : (lo << 16));
-            const float b = __uint_as_float((j & 1) ? (hi & 0xFFFF0000u) : (hi << 16));
-            P[j] = pk(a, b);
-        }
-    } else {
-        // 32 f32 = one whole 128-byte row: row t, chunks 0..7
-        const int R = R0 + t;
-        float e[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 v = *reinterpret_cast<const float4*>(slot + R * 128 + ((j ^ (R & 7)) << 4));
-            e[4 * j] = v.x;
-            e[4 * j + 1] = v.y;
-            e[4 * j + 2] = v.z;
-            e[4 * j + 3] = v.w;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) P[j] = pk(e[j], e[j + 16]);
+        P[j] = pk(a, b);
     }
 }
 
-// Stages h = 1, 2, 4, 8 (packed, both halves at once) then h = 16 (inside
-// each pair).  Butterfly (u, w) -> (u + w, u - w), u the lower index.
-__device__ __forceinline__ void fwht_in_registers(uint64_t (&P)[16]) {
+// Stages h = 1, 2, ..., kPairs/2 (packed, both halves at once) then
+// h = kPairs (inside each pair).  Butterfly (u, w) -> (u + w, u - w), u the
+// lower index.
+__device__ __forceinline__ void fwht_in_registers(uint64_t (&P)[kPairs]) {
 #pragma unroll
-    for (int h = 1; h < 16; h <<= 1) {
+    for (int h = 1; h < kPairs; h <<= 1) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < kPairs; ++j) {
             if ((j & h) == 0) {
                 const uint64_t u = P[j], w = P[j + h];
                 P[j] = add2(u, w);
@@ -147,22 +149,22 @@ __device__ __forceinline__ void fwht_in_registers(uint64_t (&P)[16]) {
         }
     }
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < kPairs; ++j) {
         float u, w;
         upk(P[j], u, w);
         P[j] = pk(__fadd_rn(u, w), __fsub_rn(u, w));
     }
 }
 
-// Stage across lanes: the partner (lane ^ sh) holds the elements sh*32
-// positions away.  sign = +1 on the lower side (self + partner), -1 on the
+// Stage across lanes: the partner (lane ^ sh) holds the elements
+// sh*kPerThread positions away.  sign = +1 on the lower side (self + partner), -1 on the
 // upper side (partner - self); fma(sign, self, partner) rounds once, exactly
 // like that add or subtract.
-__device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[16], int sh, bool upper) {
+__device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[kPairs], int sh, bool upper) {
     const float sg = upper ? -1.0f : 1.0f;
     const uint64_t S = pk(sg, sg);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < kPairs; ++j) {
         float a, b;
         upk(P[j], a, b);
         const float pa = __shfl_xor_sync(0xFFFFFFFFu, a, sh);
@@ -172,7 +174,7 @@ __device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[16], int sh, boo
 }
 
 template <typename Tin, int BLOCK>
-__global__ void __launch_bounds__(1024) rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
+__global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
                                                             int tpr, int tpr_pad, int rows_per_cta, int rows128,
                                                             int box1, int nbox, int nstage, int64_t num_groups,
                                                             int8_t* __restrict__ q, int64_t ldq,
@@ -221,23 +223,24 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const __grid_constan
         // the next CTA barrier so that all threads leave the loop together.
         if (!mbar_wait_bounded(&full[slot], parity, limit_ns, kErrTimeoutLoad, err)) abort_flag = 1;
 
-        uint64_t P[16];
+        uint64_t P[kPairs];
         if (t < tpr) {
             load_pairs<Tin>(ring + static_cast<size_t>(slot) * slot_bytes, rloc * row_pitch, t, P);
         } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) P[j] = 0ull;
+            for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
         }
 
         if constexpr (BLOCK == 128) {
             fwht_in_registers(P);
-            fwht_across_lanes(P, 1, (t & 1) != 0);  // h = 32
-            fwht_across_lanes(P, 2, (t & 2) != 0);  // h = 64
+#pragma unroll
+            for (int sh = 1; sh < kLanesPerBlock; sh <<= 1)  // h = kPerThread * sh
+                fwht_across_lanes(P, sh, (t & sh) != 0);
         }
 
         float amax = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < kPairs; ++j) {
             float a, b;
             upk(P[j], a, b);
             amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
@@ -272,27 +275,27 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(const __grid_constan
         if (row < M && t < tpr) {
             const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
             const uint64_t inv2 = pk(inv, inv);
-            uint32_t lo[16], hi[16];
+            uint32_t c[kPerThread];  // codes in element order, one per 32-bit word
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < kPairs; ++j) {
                 float a, b;
                 upk(mul2(P[j], inv2), a, b);
-                lo[j] = static_cast<uint32_t>(__float2int_rn(a));
-                hi[j] = static_cast<uint32_t>(__float2int_rn(b));
+                c[j] = static_cast<uint32_t>(__float2int_rn(a));
+                c[j + kPairs] = static_cast<uint32_t>(__float2int_rn(b));
             }
-            uint32_t word[8];
+            uint32_t word[kPerThread / 4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                word[i] = prmt(prmt(lo[4 * i], lo[4 * i + 1], 0x0040u), prmt(lo[4 * i + 2], lo[4 * i + 3], 0x0040u),
+            for (int i = 0; i < kPerThread / 4; ++i)
+                word[i] = prmt(prmt(c[4 * i], c[4 * i + 1], 0x0040u), prmt(c[4 * i + 2], c[4 * i + 3], 0x0040u),
                                0x5410u);
-                word[4 + i] = prmt(prmt(hi[4 * i], hi[4 * i + 1], 0x0040u),
-                                   prmt(hi[4 * i + 2], hi[4 * i + 3], 0x0040u), 0x5410u);
-            }
             int8_t* dst = q + row * ldq + static_cast<int64_t>(t) * kPerThread;
-            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(word[0]),
-                         "r"(word[1]), "r"(word[2]), "r"(word[3]), "r"(word[4]), "r"(word[5]), "r"(word[6]),
-                         "r"(word[7])
-                         : "memory");
+#pragma unroll
+            for (int i = 0; i < kPerThread / 32; ++i)
+                asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 32 * i),
+                             "r"(word[8 * i]), "r"(word[8 * i + 1]), "r"(word[8 * i + 2]), "r"(word[8 * i + 3]),
+                             "r"(word[8 * i + 4]), "r"(word[8 * i + 5]), "r"(word[8 * i + 6]),
+                             "r"(word[8 * i + 7])
+                             : "memory");
             if (t == 0) s[row] = __fdiv_rn(amax, 127.0f);
         }
     }
@@ -347,7 +350,7 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
         if (g->box1 > 256) return false;
         // Several rows per group share the CTA's barriers (at most 1024 threads).
         g->rows_per_cta = g->nbox == 1 ? CONVROT_RQ_LONG_ROWS : 1;
-        while (g->rows_per_cta > 1 && g->tpr_pad * g->rows_per_cta > 1024) --g->rows_per_cta;
+        while (g->rows_per_cta > 1 && g->tpr_pad * g->rows_per_cta > kMaxThreads) --g->rows_per_cta;
     }
     g->threads = g->tpr_pad * g->rows_per_cta;
     const size_t slot = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
