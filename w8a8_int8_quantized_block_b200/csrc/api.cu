@@ -142,7 +142,7 @@ convrot_status gemm(const int8_t* qa, const int8_t* qb, const float* sa, const f
         return CONVROT_ECUDA;
     if (!encode_3d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                    static_cast<uint64_t>(batch), static_cast<uint64_t>(K), static_cast<uint64_t>(N * K), kGemmBK,
-                   kGemmBN, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint32_t>(gemm_b_box_rows()), 1, CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
     if (!encode_3d(&ymap, s32 ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y,
                    static_cast<uint64_t>(N), static_cast<uint64_t>(M), static_cast<uint64_t>(batch),

@@ -11,42 +11,69 @@
 // is bf16 because "the residual stream reaches 2.4e5, beyond fp16's range"
 // ("HyperFlow H3 Flash MLX", section "How to run").
 //
-// Design (B200, one CTA per SM, persistent):
-//   warp 0      TMA producer: 128x128-byte A and 256x128-byte B tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (mbarrier per stage)
-//   warp 1      MMA issuer: one thread issues tcgen05.mma kind::i8
-//               (M=128, N=256, K=32) into a TMEM accumulator; tcgen05.commit
+// Two kernels share the roles and the epilogue; both are persistent,
+// warp-specialised, one CTA per SM:
+//   warp 0      TMA producer into a shared-memory ring (mbarrier per stage,
+//               128-byte swizzle)
+//   warp 1      MMA issuer: one thread issues tcgen05.mma kind::i8 (K = 32
+//               per instruction) into a TMEM accumulator; tcgen05.commit
 //               frees each stage and, per tile, signals the epilogue
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, scale + bias
 //               (+ GELU), bf16, swizzled shared staging, TMA store
 // Two 256-column accumulators (all 512 TMEM columns) let the epilogue of one
-// tile overlap the main loop of the next.  Tiles run n-fastest so the A panel
-// of a 128-row block is read from HBM once and reused from L2 across N.
-// No load uses cluster multicast.
+// tile overlap the main loop of the next.  Tiles run n-fastest so an A panel
+// is read from HBM once and reused from L2 across N.
+//
+//   igemm_kernel       one CTA per 128 x 256 tile (M = 128, N = 256 MMAs),
+//                      A 16 KB + B 32 KB per stage, 4 stages.
+//   igemm_pair_kernel  a cluster of two CTAs per 256 x 256 tile
+//                      (cta_group::2, M = 256, N = 256 MMAs issued by the
+//                      pair's leader): each CTA stages 128 rows of A and half
+//                      of B's 256 rows (32 KB per stage, 6 stages), so per
+//                      output element the pair moves a third less operand data
+//                      through shared memory and L2 than the single-CTA tile.
+// No load uses cluster multicast (the pair's commits do, which is allowed).
 #include <cuda_bf16.h>
 
 #include "kernels.h"
 #include "ptx.cuh"
 
+#ifndef CONVROT_GEMM_PAIR
+#define CONVROT_GEMM_PAIR 1  // 1: CTA-pair tiles, 0: single-CTA tiles
+#endif
+
 namespace convrot {
 
 namespace {
 
-constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
-constexpr int kStages = 4;
+constexpr int BN = kGemmBN, BK = kGemmBK;
 constexpr int kAccBufs = 2;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kAStage = BM * BK;                 // 16 KB
-constexpr int kBStage = BN * BK;                 // 32 KB
-constexpr int kEpiBufBytes = 4096;               // per epilogue warp
-constexpr int kSmemRing = kStages * (kAStage + kBStage);
+constexpr int kEpiBufBytes = 4096;                 // per epilogue warp
 constexpr int kSmemEpi = kEpiWarps * kEpiBufBytes;
 constexpr int kSmemCols = kEpiWarps * 2 * BN * 4;  // per-warp column scale and bias
-constexpr int kSmemBars = 8 * (2 * kStages + 2 * kAccBufs) + 16;
-constexpr int kSmemTotal = kSmemRing + kSmemEpi + kSmemCols + kSmemBars + 1024;
-static_assert(kSmemTotal <= 227 * 1024, "shared memory budget");
+
+// single-CTA tiles
+constexpr int BM1 = kGemmBM;  // 128
+constexpr int kStages1 = 4;
+constexpr int kAStage1 = BM1 * BK;  // 16 KB
+constexpr int kBStage1 = BN * BK;   // 32 KB
+constexpr int kSmemRing1 = kStages1 * (kAStage1 + kBStage1);
+constexpr int kSmemBars1 = 8 * (2 * kStages1 + 2 * kAccBufs) + 16;
+constexpr int kSmemTotal1 = kSmemRing1 + kSmemEpi + kSmemCols + kSmemBars1 + 1024;
+static_assert(kSmemTotal1 <= 227 * 1024, "shared memory budget");
+
+// CTA-pair tiles
+constexpr int BMP = 2 * kGemmBM;         // 256 rows per pair, 128 per CTA
+constexpr int kStagesP = 6;
+constexpr int kAStageP = kGemmBM * BK;   // 16 KB: this CTA's 128 rows of A
+constexpr int kBStageP = (BN / 2) * BK;  // 16 KB: this CTA's half of B
+constexpr int kSmemRingP = kStagesP * (kAStageP + kBStageP);
+constexpr int kSmemBarsP = 8 * (2 * kStagesP + 2 * kAccBufs) + 16;
+constexpr int kSmemTotalP = kSmemRingP + kSmemEpi + kSmemCols + kSmemBarsP + 1024;
+static_assert(kSmemTotalP <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     const uint32_t a = smem_u32(p);
@@ -64,13 +91,98 @@ struct TileCoord {
     int m0, n0, b;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n) {
+// Tile t of a [batch][tiles_m][tiles_n] grid of bm x BN tiles, n fastest.
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bm) {
     const int per_batch = tiles_m * tiles_n;
     const int b = t / per_batch;
     const int r = t - b * per_batch;
     const int mb = r / tiles_n;
-    return {mb * BM, (r - mb * tiles_n) * BN, b};
+    return {mb * bm, (r - mb * tiles_n) * BN, b};
 }
+
+// Column scale (s_b * alpha) and bias of one tile's BN columns into this
+// warp's private copy (no cross-warp waits anywhere in the epilogue).
+template <int EPI>
+__device__ __forceinline__ void load_tile_columns(const GemmArgs& p, const TileCoord& c, float* sColScale,
+                                                  float* sColBias, int lane) {
+    if constexpr (EPI != kEpiS32) {
+        __syncwarp();  // every lane is done with the previous tile's columns
+        for (int i = lane; i < BN; i += 32) {
+            const int n = c.n0 + i;
+            const bool in = n < p.N;
+            sColScale[i] = in ? p.s_b[static_cast<int64_t>(c.b) * p.N + n] * p.alpha : 0.0f;
+            sColBias[i] = (in && p.bias != nullptr) ? p.bias[n] : 0.0f;
+        }
+        __syncwarp();
+    }
+}
+
+// Drain one 32-row x BN accumulator slice of TMEM (lane quadrant `quad`,
+// columns from `tmem_col`) into y rows [row0, row0 + 32), columns from n0.
+template <int EPI>
+__device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensorMap* ymap, uint32_t tmem_base,
+                                               int quad, uint32_t tmem_col, int row0, int n0, int b, float sa,
+                                               const float* sColScale, const float* sColBias, uint8_t* ebuf,
+                                               int lane) {
+    for (int cc = 0; cc < BN / 32; ++cc) {
+        if (n0 + cc * 32 >= p.N) break;  // whole chunk past the last column
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(
+            tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tmem_col + static_cast<uint32_t>(cc * 32), r);
+        tmem_ld_wait();
+        if constexpr (EPI == kEpiS32) {
+            // 32 int32 = 128 bytes per row, 128-byte swizzle, single buffer
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            uint8_t* rowp = ebuf + lane * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(ymap, ebuf, n0 + cc * 32, row0, b);
+                bulk_commit_group();
+            }
+        } else {
+            // 32 bf16 = 64 bytes per row, 64-byte swizzle, two buffers
+            uint8_t* buf = ebuf + (cc & 1) * 2048;
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i0 = cc * 32 + 2 * j;
+                float y0 =
+                    fmaf(static_cast<float>(static_cast<int32_t>(r[2 * j])), sa * sColScale[i0], sColBias[i0]);
+                float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * j + 1])), sa * sColScale[i0 + 1],
+                                sColBias[i0 + 1]);
+                if constexpr (EPI == kEpiBf16Gelu) {
+                    y0 = gelu_erf(y0);
+                    y1 = gelu_erf(y1);
+                }
+                w[j] = pack_bf16x2(y0, y1);
+            }
+            uint8_t* rowp = buf + lane * 64;
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
+                    make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(ymap, buf, n0 + cc * 32, row0, b);
+                bulk_commit_group();
+            }
+        }
+    }
+}
+
+// ============================================================================ single-CTA tiles
 
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -79,18 +191,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kStages * kAStage;
-    uint8_t* sEpi = smem + kSmemRing;
+    uint8_t* sB = smem + kStages1 * kAStage1;
+    uint8_t* sEpi = smem + kSmemRing1;
     float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);  // [warp][scale | bias][BN]
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);
-    uint64_t* empty_bar = full_bar + kStages;
-    uint64_t* accf_bar = empty_bar + kStages;
+    uint64_t* empty_bar = full_bar + kStages1;
+    uint64_t* accf_bar = empty_bar + kStages1;
     uint64_t* acce_bar = accf_bar + kAccBufs;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + kAccBufs);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int tiles_m = (p.M + BM - 1) / BM;
+    const int tiles_m = (p.M + BM1 - 1) / BM1;
     const int tiles_n = (p.N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n * p.batch;
     const int k_blocks = (p.K + BK - 1) / BK;
@@ -99,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&amap);
         tma_prefetch_desc(&bmap);
         tma_prefetch_desc(&ymap);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStages1; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
@@ -128,16 +240,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const TileCoord c = tile_coord(t, tiles_m, tiles_n);
+                const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, p.limit_ns, kErrTimeoutEmpty, p.err)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full_bar[stage], kAStage + kBStage);
-                    tma_load_3d(sA + stage * kAStage, &amap, &full_bar[stage], kb * BK, c.m0, c.b);
-                    tma_load_3d(sB + stage * kBStage, &bmap, &full_bar[stage], kb * BK, c.n0, c.b);
-                    if (++stage == kStages) {
+                    mbar_arrive_expect_tx(&full_bar[stage], kAStage1 + kBStage1);
+                    tma_load_3d(sA + stage * kAStage1, &amap, &full_bar[stage], kb * BK, c.m0, c.b);
+                    tma_load_3d(sB + stage * kBStage1, &bmap, &full_bar[stage], kb * BK, c.n0, c.b);
+                    if (++stage == kStages1) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -147,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = umma_idesc_i8(BM, BN);
+            constexpr uint32_t idesc = umma_idesc_i8(BM1, BN);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -166,15 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(sA + stage * kAStage);
-                    const uint32_t b_addr = smem_u32(sB + stage * kBStage);
+                    const uint32_t a_addr = smem_u32(sA + stage * kAStage1);
+                    const uint32_t b_addr = smem_u32(sB + stage * kBStage1);
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
                         mma_i8(d_tmem, umma_desc_sw128_kmajor(a_addr + k * 32),
                                umma_desc_sw128_kmajor(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit(&empty_bar[stage]);
-                    if (++stage == kStages) {
+                    if (++stage == kStages1) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -188,95 +300,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue
-        // Each warp keeps its own copy of the tile's column scales, so the four
-        // epilogue warps never wait on one another.
-        const int ew = warp - 2;             // 0..3
-        const int quad = warp & 3;           // TMEM lane quadrant this warp may read
+        const int ew = warp - 2;    // 0..3
+        const int quad = warp & 3;  // TMEM lane quadrant this warp may read
         uint8_t* ebuf = sEpi + ew * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            const TileCoord c = tile_coord(t, tiles_m, tiles_n);
-            if constexpr (EPI != kEpiS32) {
-                __syncwarp();  // every lane is done with the previous tile's columns
-                for (int i = lane; i < BN; i += 32) {
-                    const int n = c.n0 + i;
-                    const bool in = n < p.N;
-                    sColScale[i] = in ? p.s_b[static_cast<int64_t>(c.b) * p.N + n] * p.alpha : 0.0f;
-                    sColBias[i] = (in && p.bias != nullptr) ? p.bias[n] : 0.0f;
-                }
-                __syncwarp();
-            }
+            const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1);
+            load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
             const bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
             tc_fence_after_sync();
-            const int row_in_tile = quad * 32 + lane;
-            const int m = c.m0 + row_in_tile;
+            const int row0 = c.m0 + quad * 32;
             float sa = 0.0f;
             if constexpr (EPI != kEpiS32) {
-                if (m < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + m];
+                if (row0 + lane < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + row0 + lane];
             }
-            const bool rows_in = c.m0 + quad * 32 < p.M;  // else this warp's rows are all past M
-            if (ok && rows_in) {
-                for (int cc = 0; cc < BN / 32; ++cc) {
-                    if (c.n0 + cc * 32 >= p.N) break;  // whole chunk past the last column
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                           static_cast<uint32_t>(acc * BN + cc * 32),
-                                       r);
-                    tmem_ld_wait();
-                    if constexpr (EPI == kEpiS32) {
-                        // 32 int32 = 128 bytes per row, 128-byte swizzle, single buffer
-                        if (lane == 0) bulk_wait_group_read<0>();
-                        __syncwarp();
-                        uint8_t* rowp = ebuf + lane * 128;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
-                                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_3d(&ymap, ebuf, c.n0 + cc * 32, c.m0 + quad * 32, c.b);
-                            bulk_commit_group();
-                        }
-                    } else {
-                        // 32 bf16 = 64 bytes per row, 64-byte swizzle, two buffers
-                        uint8_t* buf = ebuf + (cc & 1) * 2048;
-                        if (lane == 0) bulk_wait_group_read<1>();
-                        __syncwarp();
-                        uint32_t w[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int i0 = cc * 32 + 2 * j;
-                            float y0 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * j])),
-                                            sa * sColScale[i0], sColBias[i0]);
-                            float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * j + 1])),
-                                            sa * sColScale[i0 + 1], sColBias[i0 + 1]);
-                            if constexpr (EPI == kEpiBf16Gelu) {
-                                y0 = gelu_erf(y0);
-                                y1 = gelu_erf(y1);
-                            }
-                            w[j] = pack_bf16x2(y0, y1);
-                        }
-                        uint8_t* rowp = buf + lane * 64;
-                        const int sw = (lane >> 1) & 3;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
-                                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_3d(&ymap, buf, c.n0 + cc * 32, c.m0 + quad * 32, c.b);
-                            bulk_commit_group();
-                        }
-                    }
-                }
-            }
+            if (ok && row0 < p.M)
+                epilogue_slice<EPI>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0, c.b, sa,
+                                    sColScale, sColBias, ebuf, lane);
             tc_fence_before_sync();
             mbar_arrive(&acce_bar[acc]);
             if (!ok) break;
@@ -294,18 +337,185 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// ============================================================================ CTA-pair tiles
+
 template <int EPI>
-cudaError_t launch_epi(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
-                       const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+__global__ void __launch_bounds__(kThreads, 1)
+    igemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                      const __grid_constant__ CUtensorMap ymap, const GemmArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    // The same layout in both CTAs: the pair's MMAs and commits address the
+    // peer's shared memory at the same offsets as the leader's.
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStagesP * kAStageP;
+    uint8_t* sEpi = smem + kSmemRingP;
+    float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);  // used in the leader
+    uint64_t* empty_bar = full_bar + kStagesP;                                       // in both CTAs
+    uint64_t* accf_bar = empty_bar + kStagesP;                                       // in both CTAs
+    uint64_t* acce_bar = accf_bar + kAccBufs;                                        // used in the leader
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + kAccBufs);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+    const int tiles_m = (p.M + BMP - 1) / BMP;
+    const int tiles_n = (p.N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n * p.batch;
+    const int k_blocks = (p.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
+        tma_prefetch_desc(&ymap);
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full_bar[s], 1);   // the leader's producer arrives; both CTAs' loads complete bytes
+            mbar_init(&empty_bar[s], 1);  // the leader's commit arrives (multicast)
+        }
+        for (int a = 0; a < kAccBufs; ++a) {
+            mbar_init(&accf_bar[a], 1);              // the leader's commit arrives (multicast)
+            mbar_init(&acce_bar[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_wait_primary();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- producer (both CTAs)
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP);
+                const int a_row = c.m0 + static_cast<int>(rank) * kGemmBM;
+                const int b_row = c.n0 + static_cast<int>(rank) * (BN / 2);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, p.limit_ns, kErrTimeoutEmpty, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    // The leader expects both CTAs' bytes on its own barrier.
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (kAStageP + kBStageP));
+                    const uint32_t leader_full = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                    tma_load_3d_pair(sA + stage * kAStageP, &amap, leader_full, kb * BK, a_row, c.b);
+                    tma_load_3d_pair(sB + stage * kBStageP, &bmap, leader_full, kb * BK, b_row, c.b);
+                    if (++stage == kStagesP) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------------------------------------------------- MMA issuer (leader only)
+            constexpr uint32_t idesc = umma_idesc_i8(BMP, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                if (!mbar_wait_bounded(&acce_bar[acc], acc_phase ^ 1u, p.limit_ns, kErrTimeoutAccEmpty, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(&full_bar[stage], phase, p.limit_ns, kErrTimeoutMmaFull, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(sA + stage * kAStageP);
+                    const uint32_t b_addr = smem_u32(sB + stage * kBStageP);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k) {
+                        mma_i8_pair(d_tmem, umma_desc_sw128_kmajor(a_addr + k * 32),
+                                    umma_desc_sw128_kmajor(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit_pair(&empty_bar[stage], 0x3);  // frees this stage in both CTAs
+                    if (++stage == kStagesP) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                mma_commit_pair(&accf_bar[acc], 0x3);  // both CTAs' accumulators are ready
+                if (++acc == kAccBufs) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int quad = warp & 3;
+        uint8_t* ebuf = sEpi + ew * kEpiBufBytes;
+        float* sColScale = sCols + ew * 2 * BN;
+        float* sColBias = sColScale + BN;
+        const uint32_t leader_acce0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair; t < num_tiles; t += num_pairs) {
+            const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP);
+            load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
+            const bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
+            tc_fence_after_sync();
+            const int row0 = c.m0 + static_cast<int>(rank) * kGemmBM + quad * 32;
+            float sa = 0.0f;
+            if constexpr (EPI != kEpiS32) {
+                if (row0 + lane < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + row0 + lane];
+            }
+            if (ok && row0 < p.M)
+                epilogue_slice<EPI>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0, c.b, sa,
+                                    sColScale, sColBias, ebuf, lane);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acce0 + static_cast<uint32_t>(acc * 8));
+            if (!ok) break;
+            if (++acc == kAccBufs) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) bulk_wait_group<0>();
+    }
+
+    tc_fence_before_sync();
+    cluster_sync();  // no CTA leaves while its peer may still signal it or read its TMEM
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+// ============================================================================ launchers
+
+template <int EPI>
+cudaError_t launch_single(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
+                          const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
     auto kern = igemm_kernel<EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal1);
     if (e != cudaSuccess) return e;
-    const int64_t tiles = static_cast<int64_t>((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN) * a.batch;
+    const int64_t tiles = static_cast<int64_t>((a.M + BM1 - 1) / BM1) * ((a.N + BN - 1) / BN) * a.batch;
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemTotal;
+    cfg.dynamicSmemBytes = kSmemTotal1;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -317,7 +527,50 @@ cudaError_t launch_epi(const CUtensorMap& amap, const CUtensorMap& bmap, const C
     return cudaGetLastError();
 }
 
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
+                        const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+    auto kern = igemm_pair_kernel<EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalP);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = static_cast<int64_t>((a.M + BMP - 1) / BMP) * ((a.N + BN - 1) / BN) * a.batch;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemTotalP;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    int max_clusters = 0;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
+    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+    const int64_t pairs = tiles < max_clusters ? tiles : max_clusters;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    e = cudaLaunchKernelEx(&cfg, kern, amap, bmap, ymap, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_epi(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
+                       const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+    if (gemm_uses_pair()) return launch_pair<EPI>(amap, bmap, ymap, a, num_sms, pdl, stream);
+    return launch_single<EPI>(amap, bmap, ymap, a, num_sms, pdl, stream);
+}
+
 }  // namespace
+
+bool gemm_uses_pair() { return CONVROT_GEMM_PAIR != 0; }
+
+int gemm_b_box_rows() { return gemm_uses_pair() ? BN / 2 : BN; }
 
 cudaError_t launch_igemm(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
                          const GemmArgs& a, int epilogue, int num_sms, bool pdl, cudaStream_t stream) {

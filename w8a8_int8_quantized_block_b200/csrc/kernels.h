@@ -60,6 +60,11 @@ struct GemmArgs {
 cudaError_t launch_igemm(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
                          const GemmArgs& a, int epilogue, int num_sms, bool pdl, cudaStream_t stream);
 
+// Whether the GEMM runs as CTA pairs (256 x 256 tiles, cta_group::2).
+bool gemm_uses_pair();
+// Rows of B one CTA loads per stage: BN for single-CTA tiles, BN/2 for pairs.
+int gemm_b_box_rows();
+
 // Box sizes the GEMM's tensor maps must use.
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;

@@ -51,6 +51,14 @@ static_assert(kPerThread == 32 || kPerThread == 64, "32 or 64 elements per threa
 constexpr int kPairs = kPerThread / 2;          // P[j] = (element j, element j + kPairs)
 constexpr int kLanesPerBlock = 128 / kPerThread;  // lanes sharing one Hadamard block
 constexpr int kMaxThreads = kPerThread == 32 ? 1024 : 512;
+#ifdef CONVROT_RQ_MAXREG
+#define CONVROT_RQ_BOUNDS __maxnreg__(CONVROT_RQ_MAXREG)
+#else
+#define CONVROT_RQ_BOUNDS __launch_bounds__(kMaxThreads)
+#endif
+#ifndef CONVROT_RQ_STAGES
+#define CONVROT_RQ_STAGES 3  // ring slots (row groups in flight) per CTA
+#endif
 #ifndef CONVROT_RQ_LONG_ROWS
 #define CONVROT_RQ_LONG_ROWS 1  // rows per group when a row spans more than one warp
 #endif
@@ -174,7 +182,7 @@ __device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[kPairs], int sh,
 }
 
 template <typename Tin, int BLOCK>
-__global__ void __launch_bounds__(kMaxThreads) rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
+__global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
                                                             int tpr, int tpr_pad, int rows_per_cta, int rows128,
                                                             int box1, int nbox, int nstage, int64_t num_groups,
                                                             int8_t* __restrict__ q, int64_t ldq,
@@ -356,9 +364,9 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
     const size_t slot = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
     if (slot % 1024 != 0) return false;  // slots must stay 1024-byte aligned for the swizzle
     const size_t budget = 200 * 1024;
-    g->nstage = 3;
+    g->nstage = CONVROT_RQ_STAGES;
     while (g->nstage > 1 && slot * g->nstage + 1024 > budget) --g->nstage;
-    if (g->nstage == 3 && slot * 3 > 96 * 1024) g->nstage = 2;  // leave room for a second CTA
+    if (g->nstage > 2 && slot * g->nstage > 96 * 1024) g->nstage = 2;  // leave room for a second CTA
     g->smem_bytes = slot * g->nstage + 1024;  // slack for 1024-byte alignment
     return g->smem_bytes <= budget;
 }
