@@ -12,7 +12,7 @@
 //   amax = max |z|;  s = amax / 127;  q = clamp(rne(z * (127 / amax)), +-127)
 //
 // Design (B200).  A persistent CTA walks over groups of rows; each group is
-// brought into one slot of a 2-3 slot shared-memory ring by TMA (128-byte
+// brought into one slot of a two-slot shared-memory ring by TMA (128-byte
 // swizzle, so the 16-byte reads below are bank-conflict free) while the
 // previous group is computed.  Each thread owns 64 consecutive elements of a
 // row (half a Hadamard block), held as 32 packed f32x2 register pairs
@@ -51,13 +51,14 @@ static_assert(kPerThread == 32 || kPerThread == 64, "32 or 64 elements per threa
 constexpr int kPairs = kPerThread / 2;          // P[j] = (element j, element j + kPairs)
 constexpr int kLanesPerBlock = 128 / kPerThread;  // lanes sharing one Hadamard block
 constexpr int kMaxThreads = kPerThread == 32 ? 1024 : 512;
-#ifdef CONVROT_RQ_MAXREG
-#define CONVROT_RQ_BOUNDS __maxnreg__(CONVROT_RQ_MAXREG)
-#else
-#define CONVROT_RQ_BOUNDS __launch_bounds__(kMaxThreads)
+// 80 registers and two ring slots let eight 96-thread CTAs share an SM (the
+// kernel is latency-bound; more rows in flight beat more registers per thread).
+#ifndef CONVROT_RQ_MAXREG
+#define CONVROT_RQ_MAXREG 80
 #endif
+#define CONVROT_RQ_BOUNDS __maxnreg__(CONVROT_RQ_MAXREG)
 #ifndef CONVROT_RQ_STAGES
-#define CONVROT_RQ_STAGES 3  // ring slots (row groups in flight) per CTA
+#define CONVROT_RQ_STAGES 2  // ring slots (row groups in flight) per CTA
 #endif
 #ifndef CONVROT_RQ_LONG_ROWS
 #define CONVROT_RQ_LONG_ROWS 1  // rows per group when a row spans more than one warp
