@@ -30,9 +30,9 @@ if ROOT not in sys.path:
 METRIC = "ConvRot W8A8 linear TOPS at M=38656,K=N=5376 and % of B200 INT8 peak"
 UNIT = "TOPS"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-GEMM_PROFILE = os.path.join(ROOT, "profiles", "igemm_tcgen05_proj_m38656_k5376_n5376.txt")
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "igemm_pair_proj_m38656_k5376_n5376.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "w8a8_int8_quantized_block_b200", "csrc", f)
-                  for f in ("igemm_tcgen05.cu", "ptx.cuh", "kernels.h")]
+                  for f in ("igemm_tcgen05.cu", "gemm_core.cuh", "ptx.cuh", "kernels.h")]
 INT8_PER_BF16 = 2.0  # nominal dense ratio of 8-bit to bf16 tensor throughput (4.5 vs 2.25 PFLOP/s)
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
@@ -173,9 +173,11 @@ def cpu_baseline(spec, target_s: float = 12.0):
     xb = O.bf16_bits(x)
     qw, sw = O.pack_weight(w.numpy(), spec.block)  # offline on both sides: not timed
     b = bias.numpy().astype(np.float32)
-    t = oracle_sample(xb, qw, sw, b, 8, spec.block)
-    rows = int(min(spec.M, max(8, round(8 * target_s / max(t, 1e-3)))))
+    rows = 16
     t = oracle_sample(xb, qw, sw, b, rows, spec.block)
+    while t < 0.5 * target_s and rows < spec.M:  # grow the sample until it takes about target_s
+        rows = int(min(spec.M, max(2 * rows, round(rows * target_s / max(t, 1e-3)))))
+        t = oracle_sample(xb, qw, sw, b, rows, spec.block)
     ops = 2.0 * rows * spec.N * spec.K
     return {"value": ops / t / 1e12, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle",
             "sample": f"{rows} of {spec.M} token rows through the whole path (rotate+quantise, int64 GEMM vs all "

@@ -47,8 +47,9 @@ def test_proj_768p_full_size():
     torch.cuda.synchronize()
     assert C.last_device_status() == (C.OK, 0)
     qx = ws[:spec.M * spec.K].view(torch.int8).view(spec.M, spec.K).cpu().numpy()
-    sx = ws[C.workspace_bytes(spec.M, spec.K) - ((spec.M * 4 + 255) // 256) * 256:].view(torch.float32)[:spec.M]
-    sx = sx.cpu().numpy()
+    # workspace layout: codes [M][K], then the scales, each region rounded up to 256 bytes
+    off = (spec.M * spec.K + 255) // 256 * 256
+    sx = ws[off:off + spec.M * 4].view(torch.float32).cpu().numpy()
     xb = bits(x)
     qxr, sxr = O.quantize_act(xb, spec.block)
     assert_codes_match(qx, sx, qxr, sxr, None, spec.block)

@@ -183,6 +183,53 @@ convrot_status linear_checks(const int8_t* qw, const float* s_w, const convrot_w
     return CONVROT_OK;
 }
 
+// The one-kernel linear covers rotated (block 128) or unrotated rows whose
+// length fits one quantiser group.
+bool fused_eligible(int64_t K, int32_t block) {
+    return (block == 128 || block == 0) && K % 128 == 0 && K >= 128 && K <= kFusedMaxK;
+}
+
+convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
+                                 const convrot_wdesc* desc, const float* bias, int epi, int8_t* qx, float* sx,
+                                 unsigned int* ready, uint16_t* y, int64_t ldy, cudaStream_t stream) {
+    const DeviceInfo* d = device_info();
+    if (!d) return CONVROT_ECUDA;
+    if (!d->supported) return CONVROT_EUNSUPPORTED;
+    const int64_t K = desc->K, N = desc->N;
+    CUtensorMap xmap, amap, bmap, ymap;
+    if (!encode_3d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 64, static_cast<uint64_t>(K / 64),
+                   static_cast<uint64_t>(M), 128, static_cast<uint64_t>(ldx) * 2, 64,
+                   static_cast<uint32_t>(fused_box1(K)), 1, CU_TENSOR_MAP_SWIZZLE_128B))
+        return CONVROT_ECUDA;
+    if (!encode_3d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, static_cast<uint64_t>(K), static_cast<uint64_t>(M), 1,
+                   static_cast<uint64_t>(K), static_cast<uint64_t>(M * K), kGemmBK, kGemmBM, 1,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return CONVROT_ECUDA;
+    if (!encode_3d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, static_cast<uint64_t>(K), static_cast<uint64_t>(N), 1,
+                   static_cast<uint64_t>(K), static_cast<uint64_t>(N * K), kGemmBK, kGemmBN / 2, 1,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return CONVROT_ECUDA;
+    if (!encode_3d(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, static_cast<uint64_t>(N), static_cast<uint64_t>(M), 1,
+                   static_cast<uint64_t>(ldy) * 2, static_cast<uint64_t>(M * ldy) * 2, kEpiCols, kEpiRows, 1,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+        return CONVROT_ECUDA;
+    const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
+    if (cudaMemsetAsync(ready, 0, panels * 4, stream) != cudaSuccess) return CONVROT_ECUDA;
+    GemmArgs a;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.batch = 1;
+    a.s_a = sx;
+    a.s_b = s_w;
+    a.bias = bias;
+    a.alpha = alpha_for_block(desc->block);
+    a.limit_ns = g_limit_ns.load();
+    a.err = d->err;
+    return cuda_status(launch_linear_fused(xmap, amap, bmap, ymap, a, qx, sx, ready, desc->block > 1 ? 128 : 0, epi,
+                                           d->num_sms, true, stream));
+}
+
 }  // namespace
 }  // namespace convrot
 
@@ -239,7 +286,9 @@ convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int
 
 size_t convrot_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
-    return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) + round256(static_cast<size_t>(M) * 4);
+    const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
+    return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) + round256(static_cast<size_t>(M) * 4) +
+           round256(panels * 4);
 }
 
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
@@ -252,11 +301,18 @@ convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, c
     int8_t* qx = static_cast<int8_t*>(workspace);
     float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                          round256(static_cast<size_t>(M) * static_cast<size_t>(desc->K)));
+    unsigned int* ready = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(sx) +
+                                                          round256(static_cast<size_t>(M) * 4));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int epi = epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16;
+    if (fused_eligible(desc->K, desc->block)) {
+        // One kernel: the quantiser warps run ahead of the tensor cores.
+        if (!aligned16(x) || ldx < desc->K || ldx % 8 != 0) return CONVROT_EINVAL;
+        return linear_one_kernel(x, M, ldx, qw, s_w, desc, bias, epi, qx, sx, ready, y, ldy, s);
+    }
     st = rotate_quant(x, 2, M, desc->K, ldx, desc->block, qx, sx, s);
     if (st != CONVROT_OK) return st;
-    return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block),
-                epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16, 1, M, desc->N, desc->K, y, ldy, true, s);
+    return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block), epi, 1, M, desc->N, desc->K, y, ldy, true, s);
 }
 
 convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, const int8_t* qw, const float* s_w,

@@ -1,0 +1,132 @@
+// gemm_core.cuh -- pieces shared by the int8 GEMM kernels: tile
+// coordinates, the per-warp column scales and the TMEM-draining epilogue
+// (scale, bias, optional GELU, bf16 or raw int32, swizzled staging, TMA store).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace convrot {
+namespace gcore {
+
+constexpr int BN = kGemmBN, BK = kGemmBK;
+constexpr int kAccBufs = 2;
+constexpr int kEpiWarps = 4;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kEpiBufBytes = 4096;                 // per epilogue warp
+constexpr int kSmemEpi = kEpiWarps * kEpiBufBytes;
+constexpr int kSmemCols = kEpiWarps * 2 * BN * 4;  // per-warp column scale and bias
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    const uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float gelu_erf(float y) { return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f)); }
+
+struct TileCoord {
+    int m0, n0, b;
+};
+
+// Tile t of a [batch][tiles_m][tiles_n] grid of bm x BN tiles, n fastest.
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bm) {
+    const int per_batch = tiles_m * tiles_n;
+    const int b = t / per_batch;
+    const int r = t - b * per_batch;
+    const int mb = r / tiles_n;
+    return {mb * bm, (r - mb * tiles_n) * BN, b};
+}
+
+// Column scale (s_b * alpha) and bias of one tile's BN columns into this
+// warp's private copy (no cross-warp waits anywhere in the epilogue).
+template <int EPI>
+__device__ __forceinline__ void load_tile_columns(const GemmArgs& p, const TileCoord& c, float* sColScale,
+                                                  float* sColBias, int lane) {
+    if constexpr (EPI != kEpiS32) {
+        __syncwarp();  // every lane is done with the previous tile's columns
+        for (int i = lane; i < BN; i += 32) {
+            const int n = c.n0 + i;
+            const bool in = n < p.N;
+            sColScale[i] = in ? p.s_b[static_cast<int64_t>(c.b) * p.N + n] * p.alpha : 0.0f;
+            sColBias[i] = (in && p.bias != nullptr) ? p.bias[n] : 0.0f;
+        }
+        __syncwarp();
+    }
+}
+
+// Drain one 32-row x BN accumulator slice of TMEM (lane quadrant `quad`,
+// columns from `tmem_col`) into y rows [row0, row0 + 32), columns from n0.
+template <int EPI>
+__device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensorMap* ymap, uint32_t tmem_base,
+                                               int quad, uint32_t tmem_col, int row0, int n0, int b, float sa,
+                                               const float* sColScale, const float* sColBias, uint8_t* ebuf,
+                                               int lane) {
+    for (int cc = 0; cc < BN / 32; ++cc) {
+        if (n0 + cc * 32 >= p.N) break;  // whole chunk past the last column
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(
+            tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tmem_col + static_cast<uint32_t>(cc * 32), r);
+        tmem_ld_wait();
+        if constexpr (EPI == kEpiS32) {
+            // 32 int32 = 128 bytes per row, 128-byte swizzle, single buffer
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            uint8_t* rowp = ebuf + lane * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(ymap, ebuf, n0 + cc * 32, row0, b);
+                bulk_commit_group();
+            }
+        } else {
+            // 32 bf16 = 64 bytes per row, 64-byte swizzle, two buffers
+            uint8_t* buf = ebuf + (cc & 1) * 2048;
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i0 = cc * 32 + 2 * j;
+                float y0 =
+                    fmaf(static_cast<float>(static_cast<int32_t>(r[2 * j])), sa * sColScale[i0], sColBias[i0]);
+                float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * j + 1])), sa * sColScale[i0 + 1],
+                                sColBias[i0 + 1]);
+                if constexpr (EPI == kEpiBf16Gelu) {
+                    y0 = gelu_erf(y0);
+                    y1 = gelu_erf(y1);
+                }
+                w[j] = pack_bf16x2(y0, y1);
+            }
+            uint8_t* rowp = buf + lane * 64;
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
+                    make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(ymap, buf, n0 + cc * 32, row0, b);
+                bulk_commit_group();
+            }
+        }
+    }
+}
+
+}  // namespace gcore
+}  // namespace convrot

@@ -1,0 +1,387 @@
+// linear_fused.cu -- the whole ConvRot W8A8 linear in one persistent kernel:
+// rotate + quantise the activations while the tensor cores run the int8 GEMM
+// on the rows that are already quantised.
+//
+// The steps are those of rotate_quant.cu (block-diagonal Hadamard rotation,
+// rowwise int8: lehuy.net "Nen mo hinh video khuech tan 31B xuong 14B",
+// section "Cach nen hoat dong"; MiniMax-H3-Rung-Omega README, "Technical
+// Architecture Overview", item 2) and igemm_tcgen05.cu (int8 GEMM, per-token x
+// per-output-channel dequantisation, bf16 out); the arithmetic and its order
+// are identical, so the codes, scales and outputs equal the two-kernel path
+// bit for bit.
+//
+// Why one kernel: the GEMM is tensor-bound and leaves most of the SM's issue
+// slots and HBM bandwidth idle, while the quantiser is memory- and
+// latency-bound.  Here each CTA of the CTA-pair GEMM (cta_group::2, 256 x 256
+// tiles, see igemm_tcgen05.cu) also runs three quantiser groups of three warps.
+// Rows are dealt round-robin to the groups of all CTAs; each group keeps a
+// two-slot TMA ring of input rows, quantises a row, writes its codes and scale
+// to global memory and adds the row to its 256-row panel's ready count
+// (release).  The GEMM producer of a tile acquires its panel's count before it
+// loads A by TMA; the epilogue does the same before it reads the panel's
+// scales.  Panels become ready in order, the tiles walk the panels in order,
+// and every CTA is resident (the grid is sized to what fits), so every wait
+// ends; each wait is bounded all the same.
+//
+// Shared memory per CTA: a 4-stage GEMM ring (128 KB), epilogue staging and
+// column scales (24 KB) and 3 groups x 2 slots of one input row each
+// (<= 72 KB for K <= 6144).
+#include <cuda_bf16.h>
+
+#include "gemm_core.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "quant_core.cuh"
+
+namespace convrot {
+
+namespace {
+
+using namespace gcore;
+using qcore::kPairs;
+using qcore::kPerThread;
+
+constexpr int kQGroups = 3;                    // quantiser groups per CTA
+constexpr int kQWarps = 3;                     // warps per group: one row of K <= 6144
+constexpr int kQThreads = kQWarps * 32;
+constexpr int kQSlots = 2;                     // input rows in flight per group
+constexpr int kFirstQWarp = 2 + kEpiWarps;
+constexpr int kThreadsF = (kFirstQWarp + kQGroups * kQWarps) * 32;
+constexpr int kPanelRows = 2 * kGemmBM;        // 256: the pair's tile height
+constexpr int kStagesF = 4;
+constexpr int kAStageF = kGemmBM * BK;
+constexpr int kBStageF = (BN / 2) * BK;
+constexpr int kSmemRingF = kStagesF * (kAStageF + kBStageF);
+constexpr int kMaxRow128 = kFusedMaxK * 2 / 128;  // 128-byte rows of one bf16 input row
+constexpr int kSmemQ = kQGroups * kQSlots * kMaxRow128 * 128;
+constexpr int kSmemBarsF = 8 * (2 * kStagesF + 2 * kAccBufs + kQGroups * kQSlots) + 16;
+constexpr int kSmemRedF = kQGroups * 2 * kQWarps * 4;
+constexpr int kSmemTotalF = kSmemRingF + kSmemEpi + kSmemCols + kSmemQ + kSmemBarsF + kSmemRedF + 1024;
+static_assert(kSmemTotalF <= 227 * 1024, "shared memory budget");
+static_assert(kQThreads * kPerThread >= kFusedMaxK, "a group must cover a row");
+
+struct FusedArgs {
+    GemmArgs g;             // the GEMM and its epilogue (s_a = the scales below)
+    int8_t* q;              // [M][K] codes (workspace)
+    float* s;               // [M] scales (workspace)
+    unsigned int* ready;    // [ceil(M/256)] rows of each panel already quantised (zeroed)
+    int tpr;                // K / 64: threads of a group holding data
+    int box1;               // 128-byte rows per input-row box (multiple of 8)
+    int block;              // 128 = rotate, 0 = no rotation
+};
+
+__device__ __forceinline__ uint32_t panel_rows(int panel, int M) {
+    const int r = M - panel * kPanelRows;
+    return static_cast<uint32_t>(r < kPanelRows ? r : kPanelRows);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreadsF, 1)
+    linear_fused_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap amap,
+                        const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap ymap,
+                        const FusedArgs f) {
+    const GemmArgs& p = f.g;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStagesF * kAStageF;
+    uint8_t* sQ = smem + kSmemRingF;  // [group][slot][input row]
+    uint8_t* sEpi = sQ + kSmemQ;
+    float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);
+    uint64_t* empty_bar = full_bar + kStagesF;
+    uint64_t* accf_bar = empty_bar + kStagesF;
+    uint64_t* acce_bar = accf_bar + kAccBufs;
+    uint64_t* qfull = acce_bar + kAccBufs;  // [group][slot]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + kQGroups * kQSlots);
+    float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [group][2][warp]
+    __shared__ int abort_q[kQGroups];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+    const int tiles_m = (p.M + kPanelRows - 1) / kPanelRows;
+    const int tiles_n = (p.N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n;
+    const int k_blocks = (p.K + BK - 1) / BK;
+    const uint32_t qslot_bytes = static_cast<uint32_t>(f.box1) * 128u;
+
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&xmap);
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
+        tma_prefetch_desc(&ymap);
+        for (int s = 0; s < kStagesF; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < kAccBufs; ++a) {
+            mbar_init(&accf_bar[a], 1);
+            mbar_init(&acce_bar[a], 2 * kEpiWarps);
+        }
+        for (int i = 0; i < kQGroups * kQSlots; ++i) mbar_init(&qfull[i], 1);
+        for (int g = 0; g < kQGroups; ++g) abort_q[g] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_wait_primary();
+
+    if (warp >= kFirstQWarp) {
+        // ================================================================ quantiser groups
+        const int qg = (warp - kFirstQWarp) / kQWarps;
+        const int qw = (warp - kFirstQWarp) % kQWarps;
+        const int t = (warp - kFirstQWarp - qg * kQWarps) * 32 + lane;  // 0..95 within the group
+        const int64_t stride = static_cast<int64_t>(gridDim.x) * kQGroups;
+        const int64_t first = blockIdx.x + static_cast<int64_t>(gridDim.x) * qg;
+        uint8_t* ring = sQ + static_cast<size_t>(qg) * kQSlots * kMaxRow128 * 128;
+        uint64_t* bars = qfull + qg * kQSlots;
+        float* gred = red + qg * 2 * kQWarps;
+        auto issue = [&](int64_t row, int slot) {
+            mbar_arrive_expect_tx(&bars[slot], qslot_bytes);
+            tma_load_3d(ring + static_cast<size_t>(slot) * kMaxRow128 * 128, &xmap, &bars[slot], 0, 0,
+                        static_cast<int>(row));
+        };
+        if (t == 0) {
+            for (int i = 0; i < kQSlots; ++i) {
+                const int64_t r = first + i * stride;
+                if (r < p.M) issue(r, i);
+            }
+        }
+        int it = 0;
+        for (int64_t row = first; row < p.M; row += stride, ++it) {
+            const int slot = it & (kQSlots - 1);
+            const uint32_t parity = static_cast<uint32_t>(it / kQSlots) & 1u;
+            if (!mbar_wait_bounded(&bars[slot], parity, p.limit_ns, kErrTimeoutLoad, p.err)) abort_q[qg] = 1;
+            uint64_t P[kPairs];
+            if (t < f.tpr) {
+                qcore::load_pairs<__nv_bfloat16>(ring + static_cast<size_t>(slot) * kMaxRow128 * 128, 0, t, P);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
+            }
+            if (f.block == 128) qcore::fwht128(P, t);
+            float amax = qcore::piece_absmax(P);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            if (lane == 0) gred[(it & 1) * kQWarps + qw] = amax;
+            named_bar_sync(1 + qg, kQThreads);  // slot read, warp maxima published
+            if (abort_q[qg]) break;
+            if (t == 0) {
+                const int64_t rn = row + kQSlots * stride;
+                if (rn < p.M) {
+                    fence_proxy_async_smem();
+                    issue(rn, slot);
+                }
+            }
+            amax = gred[(it & 1) * kQWarps];
+            for (int i = 1; i < kQWarps; ++i) amax = fmaxf(amax, gred[(it & 1) * kQWarps + i]);
+            if (t < f.tpr) {
+                const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+                qcore::quantize_store(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
+                if (t == 0) f.s[row] = __fdiv_rn(amax, 127.0f);
+            }
+            __threadfence();                    // this thread's codes are visible device-wide
+            named_bar_sync(1 + qg, kQThreads);  // ... and so are the whole group's
+            if (t == 0) {
+                fence_proxy_async_global();
+                red_release_gpu_add(f.ready + row / kPanelRows, 1u);
+            }
+        }
+    } else if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- producer (both CTAs)
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int ready_panel = -1;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows);
+                const int panel = c.m0 / kPanelRows;
+                if (panel != ready_panel) {
+                    if (!wait_count_bounded(f.ready + panel, panel_rows(panel, p.M), p.limit_ns, kErrTimeoutPanel,
+                                            p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();  // the TMA reads below see the quantised panel
+                    ready_panel = panel;
+                }
+                const int a_row = c.m0 + static_cast<int>(rank) * kGemmBM;
+                const int b_row = c.n0 + static_cast<int>(rank) * (BN / 2);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, p.limit_ns, kErrTimeoutEmpty, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (kAStageF + kBStageF));
+                    const uint32_t leader_full = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                    tma_load_3d_pair(sA + stage * kAStageF, &amap, leader_full, kb * BK, a_row, 0);
+                    tma_load_3d_pair(sB + stage * kBStageF, &bmap, leader_full, kb * BK, b_row, 0);
+                    if (++stage == kStagesF) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------------------------------------------------- MMA issuer (leader only)
+            constexpr uint32_t idesc = umma_idesc_i8(kPanelRows, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                if (!mbar_wait_bounded(&acce_bar[acc], acc_phase ^ 1u, p.limit_ns, kErrTimeoutAccEmpty, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(&full_bar[stage], phase, p.limit_ns, kErrTimeoutMmaFull, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(sA + stage * kAStageF);
+                    const uint32_t b_addr = smem_u32(sB + stage * kBStageF);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k) {
+                        mma_i8_pair(d_tmem, umma_desc_sw128_kmajor(a_addr + k * 32),
+                                    umma_desc_sw128_kmajor(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit_pair(&empty_bar[stage], 0x3);
+                    if (++stage == kStagesF) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                mma_commit_pair(&accf_bar[acc], 0x3);
+                if (++acc == kAccBufs) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int quad = warp & 3;
+        uint8_t* ebuf = sEpi + ew * kEpiBufBytes;
+        float* sColScale = sCols + ew * 2 * BN;
+        float* sColBias = sColScale + BN;
+        const uint32_t leader_acce0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair; t < num_tiles; t += num_pairs) {
+            const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows);
+            load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
+            bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
+            tc_fence_after_sync();
+            // The accumulator is done, so the panel was ready; acquire it again
+            // here so that this warp's reads of the panel's scales see them.
+            const int panel = c.m0 / kPanelRows;
+            if (ok && lane == 0)
+                ok = wait_count_bounded(f.ready + panel, panel_rows(panel, p.M), p.limit_ns, kErrTimeoutPanel, p.err);
+            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+            __syncwarp();  // orders lane 0's acquire before every lane's reads of the scales
+            const int row0 = c.m0 + static_cast<int>(rank) * kGemmBM + quad * 32;
+            float sa = 0.0f;
+            if (ok && row0 + lane < p.M) sa = f.s[row0 + lane];
+            if (ok && row0 < p.M)
+                epilogue_slice<EPI>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0, 0, sa,
+                                    sColScale, sColBias, ebuf, lane);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acce0 + static_cast<uint32_t>(acc * 8));
+            if (!ok) break;
+            if (++acc == kAccBufs) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) bulk_wait_group<0>();
+    }
+
+    tc_fence_before_sync();
+    cluster_sync();
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+template <int EPI>
+cudaError_t launch_fused_epi(const CUtensorMap& xmap, const CUtensorMap& amap, const CUtensorMap& bmap,
+                             const CUtensorMap& ymap, const FusedArgs& f, int num_sms, bool pdl,
+                             cudaStream_t stream) {
+    auto kern = linear_fused_kernel<EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalF);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreadsF);
+    cfg.dynamicSmemBytes = kSmemTotalF;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    int max_clusters = 0;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
+    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+    // Every CTA quantises rows other CTAs wait for, so all of them must be
+    // resident at once: never launch more clusters than fit.
+    const int64_t tiles = static_cast<int64_t>((f.g.M + kPanelRows - 1) / kPanelRows) * ((f.g.N + BN - 1) / BN);
+    const int64_t pairs = tiles < max_clusters ? tiles : max_clusters;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    e = cudaLaunchKernelEx(&cfg, kern, xmap, amap, bmap, ymap, f);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int fused_box1(int64_t K) { return static_cast<int>(((K * 2 / 128) + 7) / 8 * 8); }
+
+cudaError_t launch_linear_fused(const CUtensorMap& xmap, const CUtensorMap& amap, const CUtensorMap& bmap,
+                                const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
+                                unsigned int* ready, int block, int epilogue, int num_sms, bool pdl,
+                                cudaStream_t stream) {
+    FusedArgs f;
+    f.g = g;
+    f.q = q;
+    f.s = s;
+    f.ready = ready;
+    f.tpr = g.K / kPerThread;
+    f.box1 = fused_box1(g.K);
+    f.block = block;
+    if (f.box1 > kMaxRow128 || f.tpr > kQThreads) return cudaErrorInvalidValue;
+    switch (epilogue) {
+        case kEpiBf16:
+            return launch_fused_epi<kEpiBf16>(xmap, amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kEpiBf16Gelu:
+            return launch_fused_epi<kEpiBf16Gelu>(xmap, amap, bmap, ymap, f, num_sms, pdl, stream);
+        default:
+            return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace convrot

@@ -21,6 +21,7 @@ enum : unsigned int {
     kErrTimeoutAccFull = 4,   // the epilogue waited for an accumulator too long
     kErrTimeoutAccEmpty = 5,  // the MMA issuer waited for a drained accumulator
     kErrTimeoutSelfTest = 6,  // the deliberate time-out of the wait self-test
+    kErrTimeoutPanel = 7,     // the fused linear waited too long for a quantised panel
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -310,6 +311,46 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
             smem_u32(bar)),
         "h"(cta_mask)
         : "memory");
+}
+
+}  // namespace convrot
+
+// ------------------------------------------------------------------ cross-CTA signalling through global memory
+namespace convrot {
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned int* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(unsigned int* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy view of global memory with later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Spin until *p >= target (acquire), giving up after limit_ns.
+__device__ __forceinline__ bool wait_count_bounded(const unsigned int* p, uint32_t target, uint64_t limit_ns,
+                                                   unsigned int code, unsigned int* err) {
+    if (ld_acquire_gpu(p) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(p) >= target) return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_error(err, code);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace convrot

@@ -1,0 +1,190 @@
+// quant_core.cuh -- the per-thread pieces of the rotate + quantise pipeline,
+// shared by the standalone quantiser and the fused quantise-ahead linear.
+//
+// A thread owns kPerThread consecutive elements of a row (half a 128-point
+// Hadamard block), held as packed f32x2 register pairs P[j] = (element j,
+// element j + kPairs).  All arithmetic is IEEE single precision with
+// round-to-nearest-even, in the order of the textbook in-place fast
+// Walsh-Hadamard transform (stages h = 1, 2, ..., 64).
+#pragma once
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace convrot {
+namespace qcore {
+
+#ifndef CONVROT_RQ_EPT
+#define CONVROT_RQ_EPT 64  // elements each thread owns (32 or 64)
+#endif
+constexpr int kPerThread = CONVROT_RQ_EPT;
+static_assert(kPerThread == 32 || kPerThread == 64, "32 or 64 elements per thread");
+constexpr int kPairs = kPerThread / 2;          // P[j] = (element j, element j + kPairs)
+constexpr int kLanesPerBlock = 128 / kPerThread;  // lanes sharing one Hadamard block
+
+// ---- packed single-precision pairs (one 64-bit register pair)
+
+__device__ __forceinline__ uint64_t pk(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Load this thread's kPerThread consecutive elements from the swizzled slot
+// into pairs P[j] = (element j, element j + kPairs).  `R0` is the 128-byte
+// shared row holding element 0 of the thread's input row.  A 16-byte chunk c
+// of 128-byte row R sits at chunk position c ^ (R & 7) (128-byte swizzle).
+template <typename Tin>
+__device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, uint64_t (&P)[kPairs]) {
+    constexpr int kBytes = kPerThread * static_cast<int>(sizeof(Tin));
+    constexpr int kChunks = kBytes / 16;
+    const int off = t * kBytes;  // byte offset of the thread's span in its row
+    uint32_t w[kBytes / 4];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+        const int cc = (off >> 4) + c;  // chunk index counted from the row start
+        const int R = R0 + (cc >> 3);
+        const uint4 v = *reinterpret_cast<const uint4*>(slot + R * 128 + (((cc & 7) ^ (R & 7)) << 4));
+        w[4 * c] = v.x;
+        w[4 * c + 1] = v.y;
+        w[4 * c + 2] = v.z;
+        w[4 * c + 3] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        if constexpr (sizeof(Tin) == 2) {
+            // word k holds elements 2k (low half) and 2k+1 (high half)
+            const uint32_t lo = w[j >> 1], hi = w[(j + kPairs) >> 1];
+            a = __uint_as_float((j & 1) ? (lo & 0xFFFF0000u) : (lo << 16));
+            b = __uint_as_float((j & 1) ? (hi & 0xFFFF0000u) : (hi << 16));
+        } else {
+            a = __uint_as_float(w[j]);
+            b = __uint_as_float(w[j + kPairs]);
+        }
+        P[j] = pk(a, b);
+    }
+}
+
+// Stages h = 1, 2, ..., kPairs/2 (packed, both halves at once) then
+// h = kPairs (inside each pair).  Butterfly (u, w) -> (u + w, u - w), u the
+// lower index.
+__device__ __forceinline__ void fwht_in_registers(uint64_t (&P)[kPairs]) {
+#pragma unroll
+    for (int h = 1; h < kPairs; h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < kPairs; ++j) {
+            if ((j & h) == 0) {
+                const uint64_t u = P[j], w = P[j + h];
+                P[j] = add2(u, w);
+                P[j + h] = sub2(u, w);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float u, w;
+        upk(P[j], u, w);
+        P[j] = pk(__fadd_rn(u, w), __fsub_rn(u, w));
+    }
+}
+
+// Stage across lanes: the partner (lane ^ sh) holds the elements
+// sh*kPerThread positions away.  sign = +1 on the lower side (self + partner), -1 on the
+// upper side (partner - self); fma(sign, self, partner) rounds once, exactly
+// like that add or subtract.
+__device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[kPairs], int sh, bool upper) {
+    const float sg = upper ? -1.0f : 1.0f;
+    const uint64_t S = pk(sg, sg);
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        upk(P[j], a, b);
+        const float pa = __shfl_xor_sync(0xFFFFFFFFu, a, sh);
+        const float pb = __shfl_xor_sync(0xFFFFFFFFu, b, sh);
+        P[j] = fma2(S, P[j], pk(pa, pb));
+    }
+}
+
+// Round and store this thread's codes: v = z * inv rounded to f32 (packed
+// multiply), then round-half-to-even to int32 (|v| <= 127*(1+2^-24) < 127.5,
+// so no clamp can bind); byte permutes pack four codes per word; two 32-byte
+// stores write the thread's 64 codes at `dst` (32-byte aligned).
+// The product must be rounded on its own before the integer rounding: the
+// usual "add 1.5*2^23" trick was contracted with the packed multiply into one
+// FMA, which rounds the exact product instead.
+__device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], float inv, int8_t* dst) {
+    const uint64_t inv2 = pk(inv, inv);
+    uint32_t c[kPerThread];  // codes in element order, one per 32-bit word
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        upk(mul2(P[j], inv2), a, b);
+        c[j] = static_cast<uint32_t>(__float2int_rn(a));
+        c[j + kPairs] = static_cast<uint32_t>(__float2int_rn(b));
+    }
+    uint32_t word[kPerThread / 4];
+#pragma unroll
+    for (int i = 0; i < kPerThread / 4; ++i)
+        word[i] =
+            prmt(prmt(c[4 * i], c[4 * i + 1], 0x0040u), prmt(c[4 * i + 2], c[4 * i + 3], 0x0040u), 0x5410u);
+#pragma unroll
+    for (int i = 0; i < kPerThread / 32; ++i)
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 32 * i),
+                     "r"(word[8 * i]), "r"(word[8 * i + 1]), "r"(word[8 * i + 2]), "r"(word[8 * i + 3]),
+                     "r"(word[8 * i + 4]), "r"(word[8 * i + 5]), "r"(word[8 * i + 6]), "r"(word[8 * i + 7])
+                     : "memory");
+}
+
+// The whole 128-point transform of this thread's piece; t is the thread's
+// index within its row (lanes t and t^1 share a block).
+__device__ __forceinline__ void fwht128(uint64_t (&P)[kPairs], int t) {
+    fwht_in_registers(P);
+#pragma unroll
+    for (int sh = 1; sh < kLanesPerBlock; sh <<= 1)  // h = kPerThread * sh
+        fwht_across_lanes(P, sh, (t & sh) != 0);
+}
+
+// Largest |z| over this thread's piece.
+__device__ __forceinline__ float piece_absmax(const uint64_t (&P)[kPairs]) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        upk(P[j], a, b);
+        amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+    }
+    return amax;
+}
+
+}  // namespace qcore
+}  // namespace convrot
