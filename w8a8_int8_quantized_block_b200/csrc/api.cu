@@ -9,7 +9,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/convrot.h"
+#include "convrot.h"
 #include "kernels.h"
 
 namespace convrot {
@@ -196,11 +196,7 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
     if (!d) return CONVROT_ECUDA;
     if (!d->supported) return CONVROT_EUNSUPPORTED;
     const int64_t K = desc->K, N = desc->N;
-    CUtensorMap xmap, amap, bmap, ymap;
-    if (!encode_3d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 64, static_cast<uint64_t>(K / 64),
-                   static_cast<uint64_t>(M), 128, static_cast<uint64_t>(ldx) * 2, 64,
-                   static_cast<uint32_t>(fused_box1(K)), 1, CU_TENSOR_MAP_SWIZZLE_128B))
-        return CONVROT_ECUDA;
+    CUtensorMap amap, bmap, ymap;
     if (!encode_3d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, static_cast<uint64_t>(K), static_cast<uint64_t>(M), 1,
                    static_cast<uint64_t>(K), static_cast<uint64_t>(M * K), kGemmBK, kGemmBM, 1,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -226,8 +222,8 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
     a.alpha = alpha_for_block(desc->block);
     a.limit_ns = g_limit_ns.load();
     a.err = d->err;
-    return cuda_status(launch_linear_fused(xmap, amap, bmap, ymap, a, qx, sx, ready, desc->block > 1 ? 128 : 0, epi,
-                                           d->num_sms, true, stream));
+    return cuda_status(launch_linear_fused(x, ldx, amap, bmap, ymap, a, qx, sx, ready, desc->block > 1 ? 128 : 0,
+                                           epi, d->num_sms, true, stream));
 }
 
 }  // namespace

@@ -77,15 +77,11 @@ constexpr int kEpiRows = 32;     // rows per epilogue store (one warp)
 // Largest K the one-kernel linear handles (one 96-thread group per row).
 constexpr int kFusedMaxK = 6144;
 
-// 128-byte rows in one input-row box of the fused kernel's quantiser.
-int fused_box1(int64_t K);
-
 // Rotate + quantise + GEMM + epilogue in one persistent CTA-pair kernel.
-// xmap: bf16 rows (3D: 64 elements, K/64, M; box {64, fused_box1(K), 1},
-// 128-byte swizzle); amap/bmap/ymap as for launch_igemm with batch 1, amap
-// over q.  q, s: the codes and scales it writes; ready: ceil(M/256) zeroed
-// counters.  block: 128 or 0.
-cudaError_t launch_linear_fused(const CUtensorMap& xmap, const CUtensorMap& amap, const CUtensorMap& bmap,
+// x: bf16 rows [M][ldx] (16-byte aligned rows); amap/bmap/ymap as for
+// launch_igemm with batch 1, amap over q.  q, s: the codes and scales it
+// writes; ready: ceil(M/256) zeroed counters.  block: 128 or 0.
+cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMap& amap, const CUtensorMap& bmap,
                                 const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
                                 unsigned int* ready, int block, int epilogue, int num_sms, bool pdl,
                                 cudaStream_t stream);

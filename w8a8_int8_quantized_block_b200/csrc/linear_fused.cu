@@ -13,19 +13,20 @@
 // Why one kernel: the GEMM is tensor-bound and leaves most of the SM's issue
 // slots and HBM bandwidth idle, while the quantiser is memory- and
 // latency-bound.  Here each CTA of the CTA-pair GEMM (cta_group::2, 256 x 256
-// tiles, see igemm_tcgen05.cu) also runs three quantiser groups of three warps.
-// Rows are dealt round-robin to the groups of all CTAs; each group keeps a
-// two-slot TMA ring of input rows, quantises a row, writes its codes and scale
-// to global memory and adds the row to its 256-row panel's ready count
-// (release).  The GEMM producer of a tile acquires its panel's count before it
+// tiles, see igemm_tcgen05.cu) also runs two quantiser groups of three warps.
+// Rows are dealt round-robin to the groups of all CTAs; each group reads its
+// next row straight from global memory into registers while it quantises the
+// current one (no shared memory: the GEMM keeps its full 6-stage ring), writes
+// the codes and scale to global memory and adds the row to its 256-row panel's
+// ready count (release).  The GEMM producer of a tile acquires its panel's count before it
 // loads A by TMA; the epilogue does the same before it reads the panel's
 // scales.  Panels become ready in order, the tiles walk the panels in order,
 // and every CTA is resident (the grid is sized to what fits), so every wait
 // ends; each wait is bounded all the same.
 //
-// Shared memory per CTA: a 4-stage GEMM ring (128 KB), epilogue staging and
-// column scales (24 KB) and 3 groups x 2 slots of one input row each
-// (<= 72 KB for K <= 6144).
+// Shared memory per CTA: the 6-stage GEMM ring (192 KB) and epilogue staging
+// and column scales (24 KB), as in the GEMM alone.  (A 4-stage ring, which
+// left room to stage input rows by TMA, ran the GEMM part 10% slower.)
 #include <cuda_bf16.h>
 
 #include "gemm_core.cuh"
@@ -41,32 +42,30 @@ using namespace gcore;
 using qcore::kPairs;
 using qcore::kPerThread;
 
-constexpr int kQGroups = 3;                    // quantiser groups per CTA
+constexpr int kQGroups = 2;                    // quantiser groups per CTA
 constexpr int kQWarps = 3;                     // warps per group: one row of K <= 6144
 constexpr int kQThreads = kQWarps * 32;
-constexpr int kQSlots = 2;                     // input rows in flight per group
 constexpr int kFirstQWarp = 2 + kEpiWarps;
 constexpr int kThreadsF = (kFirstQWarp + kQGroups * kQWarps) * 32;
 constexpr int kPanelRows = 2 * kGemmBM;        // 256: the pair's tile height
-constexpr int kStagesF = 4;
+constexpr int kStagesF = 6;
 constexpr int kAStageF = kGemmBM * BK;
 constexpr int kBStageF = (BN / 2) * BK;
 constexpr int kSmemRingF = kStagesF * (kAStageF + kBStageF);
-constexpr int kMaxRow128 = kFusedMaxK * 2 / 128;  // 128-byte rows of one bf16 input row
-constexpr int kSmemQ = kQGroups * kQSlots * kMaxRow128 * 128;
-constexpr int kSmemBarsF = 8 * (2 * kStagesF + 2 * kAccBufs + kQGroups * kQSlots) + 16;
+constexpr int kSmemBarsF = 8 * (2 * kStagesF + 2 * kAccBufs) + 16;
 constexpr int kSmemRedF = kQGroups * 2 * kQWarps * 4;
-constexpr int kSmemTotalF = kSmemRingF + kSmemEpi + kSmemCols + kSmemQ + kSmemBarsF + kSmemRedF + 1024;
+constexpr int kSmemTotalF = kSmemRingF + kSmemEpi + kSmemCols + kSmemBarsF + kSmemRedF + 1024;
 static_assert(kSmemTotalF <= 227 * 1024, "shared memory budget");
 static_assert(kQThreads * kPerThread >= kFusedMaxK, "a group must cover a row");
 
 struct FusedArgs {
     GemmArgs g;             // the GEMM and its epilogue (s_a = the scales below)
+    const uint16_t* x;      // [M][ldx] bf16 activations
+    int64_t ldx;
     int8_t* q;              // [M][K] codes (workspace)
     float* s;               // [M] scales (workspace)
     unsigned int* ready;    // [ceil(M/256)] rows of each panel already quantised (zeroed)
     int tpr;                // K / 64: threads of a group holding data
-    int box1;               // 128-byte rows per input-row box (multiple of 8)
     int block;              // 128 = rotate, 0 = no rotation
 };
 
@@ -77,25 +76,21 @@ __device__ __forceinline__ uint32_t panel_rows(int panel, int M) {
 
 template <int EPI>
 __global__ void __launch_bounds__(kThreadsF, 1)
-    linear_fused_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap amap,
-                        const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap ymap,
-                        const FusedArgs f) {
+    linear_fused_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                        const __grid_constant__ CUtensorMap ymap, const FusedArgs f) {
     const GemmArgs& p = f.g;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStagesF * kAStageF;
-    uint8_t* sQ = smem + kSmemRingF;  // [group][slot][input row]
-    uint8_t* sEpi = sQ + kSmemQ;
+    uint8_t* sEpi = smem + kSmemRingF;
     float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);
     uint64_t* empty_bar = full_bar + kStagesF;
     uint64_t* accf_bar = empty_bar + kStagesF;
     uint64_t* acce_bar = accf_bar + kAccBufs;
-    uint64_t* qfull = acce_bar + kAccBufs;  // [group][slot]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + kQGroups * kQSlots);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + kAccBufs);
     float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [group][2][warp]
-    __shared__ int abort_q[kQGroups];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -106,10 +101,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     const int tiles_n = (p.N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int k_blocks = (p.K + BK - 1) / BK;
-    const uint32_t qslot_bytes = static_cast<uint32_t>(f.box1) * 128u;
 
     if (threadIdx.x == 0) {
-        tma_prefetch_desc(&xmap);
         tma_prefetch_desc(&amap);
         tma_prefetch_desc(&bmap);
         tma_prefetch_desc(&ymap);
@@ -121,8 +114,6 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             mbar_init(&accf_bar[a], 1);
             mbar_init(&acce_bar[a], 2 * kEpiWarps);
         }
-        for (int i = 0; i < kQGroups * kQSlots; ++i) mbar_init(&qfull[i], 1);
-        for (int g = 0; g < kQGroups; ++g) abort_q[g] = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -140,31 +131,20 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         // ================================================================ quantiser groups
         const int qg = (warp - kFirstQWarp) / kQWarps;
         const int qw = (warp - kFirstQWarp) % kQWarps;
-        const int t = (warp - kFirstQWarp - qg * kQWarps) * 32 + lane;  // 0..95 within the group
+        const int t = qw * 32 + lane;  // 0..95 within the group
+        const bool holds = t < f.tpr;
         const int64_t stride = static_cast<int64_t>(gridDim.x) * kQGroups;
         const int64_t first = blockIdx.x + static_cast<int64_t>(gridDim.x) * qg;
-        uint8_t* ring = sQ + static_cast<size_t>(qg) * kQSlots * kMaxRow128 * 128;
-        uint64_t* bars = qfull + qg * kQSlots;
         float* gred = red + qg * 2 * kQWarps;
-        auto issue = [&](int64_t row, int slot) {
-            mbar_arrive_expect_tx(&bars[slot], qslot_bytes);
-            tma_load_3d(ring + static_cast<size_t>(slot) * kMaxRow128 * 128, &xmap, &bars[slot], 0, 0,
-                        static_cast<int>(row));
-        };
-        if (t == 0) {
-            for (int i = 0; i < kQSlots; ++i) {
-                const int64_t r = first + i * stride;
-                if (r < p.M) issue(r, i);
-            }
-        }
+        uint32_t w[qcore::kRawWords];  // the next row's elements, loaded ahead
+        if (holds && first < p.M) qcore::load_bf16_global(f.x + first * f.ldx, t, w);
         int it = 0;
         for (int64_t row = first; row < p.M; row += stride, ++it) {
-            const int slot = it & (kQSlots - 1);
-            const uint32_t parity = static_cast<uint32_t>(it / kQSlots) & 1u;
-            if (!mbar_wait_bounded(&bars[slot], parity, p.limit_ns, kErrTimeoutLoad, p.err)) abort_q[qg] = 1;
             uint64_t P[kPairs];
-            if (t < f.tpr) {
-                qcore::load_pairs<__nv_bfloat16>(ring + static_cast<size_t>(slot) * kMaxRow128 * 128, 0, t, P);
+            if (holds) {
+                qcore::unpack_bf16_pairs(w, P);
+                const int64_t rn = row + stride;
+                if (rn < p.M) qcore::load_bf16_global(f.x + rn * f.ldx, t, w);  // prefetch
             } else {
 #pragma unroll
                 for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
@@ -174,18 +154,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             if (lane == 0) gred[(it & 1) * kQWarps + qw] = amax;
-            named_bar_sync(1 + qg, kQThreads);  // slot read, warp maxima published
-            if (abort_q[qg]) break;
-            if (t == 0) {
-                const int64_t rn = row + kQSlots * stride;
-                if (rn < p.M) {
-                    fence_proxy_async_smem();
-                    issue(rn, slot);
-                }
-            }
+            named_bar_sync(1 + qg, kQThreads);  // warp maxima published
             amax = gred[(it & 1) * kQWarps];
             for (int i = 1; i < kQWarps; ++i) amax = fmaxf(amax, gred[(it & 1) * kQWarps + i]);
-            if (t < f.tpr) {
+            if (holds) {
                 const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
                 qcore::quantize_store(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
                 if (t == 0) f.s[row] = __fdiv_rn(amax, 127.0f);
@@ -323,9 +295,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 }
 
 template <int EPI>
-cudaError_t launch_fused_epi(const CUtensorMap& xmap, const CUtensorMap& amap, const CUtensorMap& bmap,
-                             const CUtensorMap& ymap, const FusedArgs& f, int num_sms, bool pdl,
-                             cudaStream_t stream) {
+cudaError_t launch_fused_epi(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
+                             const FusedArgs& f, int num_sms, bool pdl, cudaStream_t stream) {
     auto kern = linear_fused_kernel<EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalF);
     if (e != cudaSuccess) return e;
@@ -352,33 +323,32 @@ cudaError_t launch_fused_epi(const CUtensorMap& xmap, const CUtensorMap& amap, c
     const int64_t tiles = static_cast<int64_t>((f.g.M + kPanelRows - 1) / kPanelRows) * ((f.g.N + BN - 1) / BN);
     const int64_t pairs = tiles < max_clusters ? tiles : max_clusters;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    e = cudaLaunchKernelEx(&cfg, kern, xmap, amap, bmap, ymap, f);
+    e = cudaLaunchKernelEx(&cfg, kern, amap, bmap, ymap, f);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int fused_box1(int64_t K) { return static_cast<int>(((K * 2 / 128) + 7) / 8 * 8); }
-
-cudaError_t launch_linear_fused(const CUtensorMap& xmap, const CUtensorMap& amap, const CUtensorMap& bmap,
+cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMap& amap, const CUtensorMap& bmap,
                                 const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
                                 unsigned int* ready, int block, int epilogue, int num_sms, bool pdl,
                                 cudaStream_t stream) {
     FusedArgs f;
     f.g = g;
+    f.x = x;
+    f.ldx = ldx;
     f.q = q;
     f.s = s;
     f.ready = ready;
     f.tpr = g.K / kPerThread;
-    f.box1 = fused_box1(g.K);
     f.block = block;
-    if (f.box1 > kMaxRow128 || f.tpr > kQThreads) return cudaErrorInvalidValue;
+    if (f.tpr > kQThreads || g.K % kPerThread != 0) return cudaErrorInvalidValue;
     switch (epilogue) {
         case kEpiBf16:
-            return launch_fused_epi<kEpiBf16>(xmap, amap, bmap, ymap, f, num_sms, pdl, stream);
+            return launch_fused_epi<kEpiBf16>(amap, bmap, ymap, f, num_sms, pdl, stream);
         case kEpiBf16Gelu:
-            return launch_fused_epi<kEpiBf16Gelu>(xmap, amap, bmap, ymap, f, num_sms, pdl, stream);
+            return launch_fused_epi<kEpiBf16Gelu>(amap, bmap, ymap, f, num_sms, pdl, stream);
         default:
             return cudaErrorInvalidValue;
     }

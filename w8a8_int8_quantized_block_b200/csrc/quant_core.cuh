@@ -63,6 +63,39 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // into pairs P[j] = (element j, element j + kPairs).  `R0` is the 128-byte
 // shared row holding element 0 of the thread's input row.  A 16-byte chunk c
 // of 128-byte row R sits at chunk position c ^ (R & 7) (128-byte swizzle).
+constexpr int kRawWords = kPerThread / 2;  // 32-bit words of one thread's bf16 elements
+
+// bf16 words (word k holds elements 2k in its low half and 2k+1 in its high
+// half; widening to f32 is exact) into pairs P[j] = (element j, element j + kPairs).
+__device__ __forceinline__ void unpack_bf16_pairs(const uint32_t (&w)[kRawWords], uint64_t (&P)[kPairs]) {
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        const uint32_t lo = w[j >> 1], hi = w[(j + kPairs) >> 1];
+        const float a = __uint_as_float((j & 1) ? (lo & 0xFFFF0000u) : (lo << 16));
+        const float b = __uint_as_float((j & 1) ? (hi & 0xFFFF0000u) : (hi << 16));
+        P[j] = pk(a, b);
+    }
+}
+
+// This thread's kPerThread bf16 elements of a row, straight from global
+// memory (read-only path): 16-byte loads at `row + t*kPerThread` (16-byte
+// aligned).
+__device__ __forceinline__ void load_bf16_global(const uint16_t* row, int t, uint32_t (&w)[kRawWords]) {
+    const uint4* src = reinterpret_cast<const uint4*>(row + static_cast<int64_t>(t) * kPerThread);
+#pragma unroll
+    for (int c = 0; c < kRawWords / 4; ++c) {
+        const uint4 v = __ldg(src + c);
+        w[4 * c] = v.x;
+        w[4 * c + 1] = v.y;
+        w[4 * c + 2] = v.z;
+        w[4 * c + 3] = v.w;
+    }
+}
+
+// Load this thread's kPerThread consecutive elements from a swizzled
+// shared-memory slot into pairs.  `R0` is the 128-byte shared row holding
+// element 0 of the thread's input row.  A 16-byte chunk c of 128-byte row R
+// sits at chunk position c ^ (R & 7) (128-byte swizzle).
 template <typename Tin>
 __device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, uint64_t (&P)[kPairs]) {
     constexpr int kBytes = kPerThread * static_cast<int>(sizeof(Tin));
@@ -79,19 +112,11 @@ __device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, u
         w[4 * c + 2] = v.z;
         w[4 * c + 3] = v.w;
     }
+    if constexpr (sizeof(Tin) == 2) {
+        unpack_bf16_pairs(w, P);
+    } else {
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-        float a, b;
-        if constexpr (sizeof(Tin) == 2) {
-            // word k holds elements 2k (low half) and 2k+1 (high half)
-            const uint32_t lo = w[j >> 1], hi = w[(j + kPairs) >> 1];
-            a = __uint_as_float((j & 1) ? (lo & 0xFFFF0000u) : (lo << 16));
-            b = __uint_as_float((j & 1) ? (hi & 0xFFFF0000u) : (hi << 16));
-        } else {
-            a = __uint_as_float(w[j]);
-            b = __uint_as_float(w[j + kPairs]);
-        }
-        P[j] = pk(a, b);
+        for (int j = 0; j < kPairs; ++j) P[j] = pk(__uint_as_float(w[j]), __uint_as_float(w[j + kPairs]));
     }
 }
 
@@ -144,19 +169,23 @@ __device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[kPairs], int sh,
 // FMA, which rounds the exact product instead.
 __device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], float inv, int8_t* dst) {
     const uint64_t inv2 = pk(inv, inv);
-    uint32_t c[kPerThread];  // codes in element order, one per 32-bit word
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-        float a, b;
-        upk(mul2(P[j], inv2), a, b);
-        c[j] = static_cast<uint32_t>(__float2int_rn(a));
-        c[j + kPairs] = static_cast<uint32_t>(__float2int_rn(b));
-    }
+    // Pairs 4i..4i+3 hold elements 4i..4i+3 (low halves) and kPairs+4i..+3
+    // (high halves): each group of four pairs completes word i and word
+    // kPairs/4 + i, so the codes are packed as soon as they exist.
     uint32_t word[kPerThread / 4];
 #pragma unroll
-    for (int i = 0; i < kPerThread / 4; ++i)
-        word[i] =
-            prmt(prmt(c[4 * i], c[4 * i + 1], 0x0040u), prmt(c[4 * i + 2], c[4 * i + 3], 0x0040u), 0x5410u);
+    for (int i = 0; i < kPairs / 4; ++i) {
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float a, b;
+            upk(mul2(P[4 * i + k], inv2), a, b);
+            lo[k] = static_cast<uint32_t>(__float2int_rn(a));
+            hi[k] = static_cast<uint32_t>(__float2int_rn(b));
+        }
+        word[i] = prmt(prmt(lo[0], lo[1], 0x0040u), prmt(lo[2], lo[3], 0x0040u), 0x5410u);
+        word[kPairs / 4 + i] = prmt(prmt(hi[0], hi[1], 0x0040u), prmt(hi[2], hi[3], 0x0040u), 0x5410u);
+    }
 #pragma unroll
     for (int i = 0; i < kPerThread / 32; ++i)
         asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 32 * i),
