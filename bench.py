@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=60.0,
+                    help="CPU time budget of the whole --impl reference run (warm-up + timed steps)")
     ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm"], default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
                          "(for profiler captures; prints no result line)")
@@ -80,6 +82,24 @@ def profiled_traffic():
         return float(kv["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         return None
+
+
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """Largest value over all ranks (every rank must call it, in the same order)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(ops_per_step: float, steps: int, world: int, slowest_rank_s: float) -> float:
+    """Whole-job throughput under weak scaling: every rank runs the full
+    per-rank workload, so the job does world * ops_per_step * steps in the
+    slowest rank's time."""
+    return world * ops_per_step * steps / slowest_rank_s / 1e12
 
 
 class ClockSampler:
@@ -196,7 +216,7 @@ def run_reference(args, rank: int):
     xb = O.bf16_bits(x)
     qw, sw = O.pack_weight(w.numpy(), spec.block)
     b = bias.numpy().astype(np.float32)
-    per_step_target = max(0.05, 60.0 / max(1, args.steps + args.warmup))
+    per_step_target = max(0.02, args.reference_seconds / max(1, args.steps + args.warmup))
     t = oracle_sample(xb, qw, sw, b, 8, spec.block)
     rows = int(min(spec.M, max(1, round(8 * per_step_target / max(t, 1e-4)))))
     for _ in range(args.warmup):
@@ -260,13 +280,6 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     def step():
         C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream)
 
@@ -298,11 +311,11 @@ def main():
             step()
         e1.record(stream)
         barrier()
-    elapsed_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    elapsed_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
     st, code = C.last_device_status()
     if st != C.OK:
         raise RuntimeError(f"device status {st} (code {code}) after the timed region")
-    value = world * spec.ops * args.steps / elapsed_s / 1e12
+    value = job_tops(spec.ops, args.steps, world, elapsed_s)
 
     # Per-kernel durations, same stream, CUDA events around each launch: the
     # one-kernel step (its ready-counter memset included), then the two
@@ -335,8 +348,8 @@ def main():
         C.linear_fused_host(x_host, pw, bias, False, x_dev, ws, y, y_host, stream=stream)
     e1.record(stream)
     barrier()
-    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-    e2e_value = world * spec.ops * args.e2e_steps / e2e_s / 1e12
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    e2e_value = job_tops(spec.ops, args.e2e_steps, world, e2e_s)
     st, code = C.last_device_status()
     if st != C.OK:
         raise RuntimeError(f"device status {st} (code {code}) after the end-to-end leg")

@@ -32,8 +32,10 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "convrot_oracle.c")
-_LIB_PATH = os.path.join(_HERE, "liboracle.so")
-_CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+# CONVROT_ORACLE_LIB points the wrapper at another build of the oracle; the
+# mutation tests use it to check that the pins catch planted mistakes.
+_LIB_PATH = os.environ.get("CONVROT_ORACLE_LIB") or os.path.join(_HERE, "liboracle.so")
+CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 __all__ = [
     "build", "lib", "num_threads", "hadamard", "hadamard_sylvester", "fwht",
@@ -46,8 +48,10 @@ __all__ = [
 
 def build(force: bool = False) -> str:
     """Compile the C oracle into ``oracle/liboracle.so`` (gcc, no fast-math)."""
+    if os.environ.get("CONVROT_ORACLE_LIB"):
+        return _LIB_PATH  # an explicitly chosen build is used as it is
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        subprocess.check_call(["gcc", *_CFLAGS, "-o", _LIB_PATH, _SRC, "-lm"])
+        subprocess.check_call(["gcc", *CFLAGS, "-o", _LIB_PATH, _SRC, "-lm"])
     return _LIB_PATH
 
 
