@@ -146,6 +146,24 @@ def test_linear_ragged_shapes(M, K, N):
     assert_close_bf16(f32_of_bf16(y), yr, f"linear {M}x{K}x{N}")
 
 
+@pytest.mark.parametrize("pad", [8, 16])
+def test_linear_fused_strided_rows(pad):
+    # Row stride K + 8 (16-byte aligned rows) takes the two-kernel path, K + 16
+    # (32-byte aligned) the one-kernel path; both must match the oracle.
+    M, K, N = 300, 5376, 512
+    spec, (x, w, bias) = W.custom_linear(M, K, N, seed=pad, n_out=20, token_scale=True)
+    xp = torch.zeros(M, K + pad, dtype=torch.bfloat16)
+    xp[:, :K] = x
+    pw = C.pack_weight(w.to(DEV), 128)
+    y = C.linear_fused(xp.to(DEV)[:, :K], pw, bias.to(DEV))
+    torch.cuda.synchronize()
+    assert C.last_device_status() == (C.OK, 0)
+    yr, *_ = O.linear(bits(x), w.numpy(), bias.numpy(), 128)
+    assert_close_bf16(f32_of_bf16(y), yr, f"strided linear pad {pad}")
+    y2 = C.linear_fused(x.to(DEV), pw, bias.to(DEV))
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
 def test_linear_gelu_epilogue():
     spec, (x, w, bias) = W.custom_linear(300, 1024, 768, seed=5, n_out=10)
     y, pw = _run_linear((x, w, bias), fused=True, gelu=True)

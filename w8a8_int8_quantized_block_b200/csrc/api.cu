@@ -210,7 +210,7 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
                    CU_TENSOR_MAP_SWIZZLE_64B))
         return CONVROT_ECUDA;
     const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
-    if (cudaMemsetAsync(ready, 0, panels * 4, stream) != cudaSuccess) return CONVROT_ECUDA;
+    if (cudaMemsetAsync(ready, 0, (panels + 1) * 4, stream) != cudaSuccess) return CONVROT_ECUDA;
     GemmArgs a;
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(N);
@@ -284,7 +284,7 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
     const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
     return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) + round256(static_cast<size_t>(M) * 4) +
-           round256(panels * 4);
+           round256((panels + 1) * 4);
 }
 
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
@@ -301,11 +301,11 @@ convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, c
                                                           round256(static_cast<size_t>(M) * 4));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int epi = epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16;
-    if (fused_eligible(desc->K, desc->block)) {
-        // One kernel: the quantiser warps run ahead of the tensor cores.
-        if (!aligned16(x) || ldx < desc->K || ldx % 8 != 0) return CONVROT_EINVAL;
+    if (!x || !aligned16(x) || ldx < desc->K || ldx % 8 != 0) return CONVROT_EINVAL;
+    // One kernel (the quantiser warps run ahead of the tensor cores) when the
+    // rows suit its 32-byte loads; otherwise the two-kernel path below.
+    if (fused_eligible(desc->K, desc->block) && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && ldx % 16 == 0)
         return linear_one_kernel(x, M, ldx, qw, s_w, desc, bias, epi, qx, sx, ready, y, ldy, s);
-    }
     st = rotate_quant(x, 2, M, desc->K, ldx, desc->block, qx, sx, s);
     if (st != CONVROT_OK) return st;
     return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block), epi, 1, M, desc->N, desc->K, y, ldy, true, s);

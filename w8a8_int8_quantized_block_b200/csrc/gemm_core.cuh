@@ -65,11 +65,14 @@ __device__ __forceinline__ void load_tile_columns(const GemmArgs& p, const TileC
 
 // Drain one 32-row x BN accumulator slice of TMEM (lane quadrant `quad`,
 // columns from `tmem_col`) into y rows [row0, row0 + 32), columns from n0.
+// The stores are marked first-to-evict in L2: y is written once and not read
+// back by this kernel, so it should not displace the operands.
 template <int EPI>
 __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensorMap* ymap, uint32_t tmem_base,
                                                int quad, uint32_t tmem_col, int row0, int n0, int b, float sa,
                                                const float* sColScale, const float* sColBias, uint8_t* ebuf,
                                                int lane) {
+    const uint64_t policy = l2_policy_evict_first();
     for (int cc = 0; cc < BN / 32; ++cc) {
         if (n0 + cc * 32 >= p.N) break;  // whole chunk past the last column
         uint32_t r[32];
@@ -89,7 +92,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_store_3d(ymap, ebuf, n0 + cc * 32, row0, b);
+                tma_store_3d_hint(ymap, ebuf, n0 + cc * 32, row0, b, policy);
                 bulk_commit_group();
             }
         } else {
@@ -121,7 +124,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_store_3d(ymap, buf, n0 + cc * 32, row0, b);
+                tma_store_3d_hint(ymap, buf, n0 + cc * 32, row0, b, policy);
                 bulk_commit_group();
             }
         }

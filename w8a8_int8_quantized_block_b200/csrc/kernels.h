@@ -80,7 +80,8 @@ constexpr int kFusedMaxK = 6144;
 // Rotate + quantise + GEMM + epilogue in one persistent CTA-pair kernel.
 // x: bf16 rows [M][ldx] (16-byte aligned rows); amap/bmap/ymap as for
 // launch_igemm with batch 1, amap over q.  q, s: the codes and scales it
-// writes; ready: ceil(M/256) zeroed counters.  block: 128 or 0.
+// writes; ready: ceil(M/256) + 1 zeroed counters (per-panel ready rows, then
+// the panels the GEMM has started).  block: 128 or 0.
 cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMap& amap, const CUtensorMap& bmap,
                                 const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
                                 unsigned int* ready, int block, int epilogue, int num_sms, bool pdl,

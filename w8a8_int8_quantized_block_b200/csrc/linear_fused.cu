@@ -48,6 +48,10 @@ constexpr int kQThreads = kQWarps * 32;
 constexpr int kFirstQWarp = 2 + kEpiWarps;
 constexpr int kThreadsF = (kFirstQWarp + kQGroups * kQWarps) * 32;
 constexpr int kPanelRows = 2 * kGemmBM;        // 256: the pair's tile height
+// Quantisers stay at most this many panels ahead of the first panel the GEMM
+// has not started, so the codes (1.4 MB per panel at K = 5376) are still in L2
+// when the tensor cores read them instead of making a round trip to HBM.
+constexpr int kPanelsAhead = 16;
 constexpr int kStagesF = 6;
 constexpr int kAStageF = kGemmBM * BK;
 constexpr int kBStageF = (BN / 2) * BK;
@@ -65,6 +69,7 @@ struct FusedArgs {
     int8_t* q;              // [M][K] codes (workspace)
     float* s;               // [M] scales (workspace)
     unsigned int* ready;    // [ceil(M/256)] rows of each panel already quantised (zeroed)
+    unsigned int* started;  // panels the GEMM has begun (a running max; zeroed)
     int tpr;                // K / 64: threads of a group holding data
     int block;              // 128 = rotate, 0 = no rotation
 };
@@ -140,6 +145,15 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         if (holds && first < p.M) qcore::load_bf16_global(f.x + first * f.ldx, t, w);
         int it = 0;
         for (int64_t row = first; row < p.M; row += stride, ++it) {
+            // Keep within kPanelsAhead panels of the GEMM (every thread of the
+            // group waits, so the group stays in step).  The GEMM starts panels
+            // in order and each group quantises its rows in order, so every
+            // panel inside the window gets finished and the window moves on.
+            const int panel = static_cast<int>(row / kPanelRows);
+            if (panel >= kPanelsAhead &&
+                !wait_count_bounded(f.started, static_cast<uint32_t>(panel - kPanelsAhead + 1), p.limit_ns,
+                                    kErrTimeoutPanel, p.err))
+                break;  // the error word is set; the GEMM side times out the same way
             uint64_t P[kPairs];
             if (holds) {
                 qcore::unpack_bf16_pairs(w, P);
@@ -187,6 +201,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     }
                     fence_proxy_async_global();  // the TMA reads below see the quantised panel
                     ready_panel = panel;
+                    atomicMax(f.started, static_cast<unsigned int>(panel + 1));  // lets the quantisers move on
                 }
                 const int a_row = c.m0 + static_cast<int>(rank) * kGemmBM;
                 const int b_row = c.n0 + static_cast<int>(rank) * (BN / 2);
@@ -341,6 +356,7 @@ cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMa
     f.q = q;
     f.s = s;
     f.ready = ready;
+    f.started = ready + (g.M + kPanelRows - 1) / kPanelRows;
     f.tpr = g.K / kPerThread;
     f.block = block;
     if (f.tpr > kQThreads || g.K % kPerThread != 0) return cudaErrorInvalidValue;

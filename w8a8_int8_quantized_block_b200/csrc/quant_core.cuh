@@ -78,17 +78,18 @@ __device__ __forceinline__ void unpack_bf16_pairs(const uint32_t (&w)[kRawWords]
 }
 
 // This thread's kPerThread bf16 elements of a row, straight from global
-// memory (read-only path): 16-byte loads at `row + t*kPerThread` (16-byte
-// aligned).
+// memory: 32-byte read-only loads at `row + t*kPerThread` (32-byte aligned),
+// marked first-to-evict in L2 (each input byte is read exactly once, so it
+// should not displace the codes and weights the tensor cores are about to use).
 __device__ __forceinline__ void load_bf16_global(const uint16_t* row, int t, uint32_t (&w)[kRawWords]) {
-    const uint4* src = reinterpret_cast<const uint4*>(row + static_cast<int64_t>(t) * kPerThread);
+    const uint16_t* src = row + static_cast<int64_t>(t) * kPerThread;
 #pragma unroll
-    for (int c = 0; c < kRawWords / 4; ++c) {
-        const uint4 v = __ldg(src + c);
-        w[4 * c] = v.x;
-        w[4 * c + 1] = v.y;
-        w[4 * c + 2] = v.z;
-        w[4 * c + 3] = v.w;
+    for (int c = 0; c < kRawWords / 8; ++c) {
+        asm volatile(
+            "ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+            : "=r"(w[8 * c]), "=r"(w[8 * c + 1]), "=r"(w[8 * c + 2]), "=r"(w[8 * c + 3]), "=r"(w[8 * c + 4]),
+              "=r"(w[8 * c + 5]), "=r"(w[8 * c + 6]), "=r"(w[8 * c + 7])
+            : "l"(src + 16 * c));
     }
 }
 

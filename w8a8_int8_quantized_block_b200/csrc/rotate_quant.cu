@@ -88,13 +88,14 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
     const int row_pitch = nbox * box1;  // 128-byte shared rows between consecutive input rows of a group
     (void)rows128;
 
+    const uint64_t policy = l2_policy_evict_first();  // every input byte is read once
     auto issue = [&](int64_t g, int slot) {
         // Full boxes are credited even where they run past the tensor (zero fill).
         mbar_arrive_expect_tx(&full[slot], slot_bytes);
         uint8_t* dst = ring + static_cast<size_t>(slot) * slot_bytes;
         for (int b = 0; b < nbox; ++b)
-            tma_load_3d(dst + static_cast<size_t>(b) * box1 * 128, &xmap, &full[slot], 0, b * box1,
-                        static_cast<int>(g * rows_per_cta));
+            tma_load_3d_hint(dst + static_cast<size_t>(b) * box1 * 128, &xmap, &full[slot], 0, b * box1,
+                             static_cast<int>(g * rows_per_cta), policy);
     };
 
     if (tid == 0) {
