@@ -146,8 +146,8 @@ convrot_status gemm(const int8_t* qa, const int8_t* qb, const float* sa, const f
         return CONVROT_ECUDA;
     if (!encode_3d(&ymap, s32 ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y,
                    static_cast<uint64_t>(N), static_cast<uint64_t>(M), static_cast<uint64_t>(batch),
-                   static_cast<uint64_t>(ldy) * ebytes, static_cast<uint64_t>(M * ldy) * ebytes, kEpiCols, kEpiRows,
-                   1, s32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+                   static_cast<uint64_t>(ldy) * ebytes, static_cast<uint64_t>(M * ldy) * ebytes,
+                   s32 ? kEpiColsS32 : kEpiColsBf16, kEpiRows, 1, CU_TENSOR_MAP_SWIZZLE_64B))
         return CONVROT_ECUDA;
     GemmArgs a;
     a.M = static_cast<int>(M);
@@ -206,7 +206,7 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
     if (!encode_3d(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, static_cast<uint64_t>(N), static_cast<uint64_t>(M), 1,
-                   static_cast<uint64_t>(ldy) * 2, static_cast<uint64_t>(M * ldy) * 2, kEpiCols, kEpiRows, 1,
+                   static_cast<uint64_t>(ldy) * 2, static_cast<uint64_t>(M * ldy) * 2, kEpiColsBf16, kEpiRows, 1,
                    CU_TENSOR_MAP_SWIZZLE_64B))
         return CONVROT_ECUDA;
     const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));

@@ -15,11 +15,15 @@ namespace gcore {
 
 constexpr int BN = kGemmBN, BK = kGemmBK;
 constexpr int kAccBufs = 2;
-constexpr int kEpiWarps = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kEpiBufBytes = 4096;                 // per epilogue warp
-constexpr int kSmemEpi = kEpiWarps * kEpiBufBytes;
-constexpr int kSmemCols = kEpiWarps * 2 * BN * 4;  // per-warp column scale and bias
+constexpr int kEpiRowBytes = 64;                  // one staged row: 32 bf16 or 16 int32
+constexpr int kEpiBufBytes = 32 * kEpiRowBytes;   // one 32-row staging buffer (64-byte swizzle)
+
+// Shared memory the epilogue of `ew` warps needs: staging buffers (two per
+// warp with four warps, one per warp with eight) and a private copy of the
+// tile's column scales and biases per warp.
+__host__ __device__ constexpr int epi_bufs(int ew) { return ew == 4 ? 2 : 1; }
+__host__ __device__ constexpr int epi_smem(int ew) { return ew * (epi_bufs(ew) * kEpiBufBytes + 2 * BN * 4); }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     const uint32_t a = smem_u32(p);
@@ -63,43 +67,56 @@ __device__ __forceinline__ void load_tile_columns(const GemmArgs& p, const TileC
     }
 }
 
-// Drain one 32-row x BN accumulator slice of TMEM (lane quadrant `quad`,
-// columns from `tmem_col`) into y rows [row0, row0 + 32), columns from n0.
-// The stores are marked first-to-evict in L2: y is written once and not read
-// back by this kernel, so it should not displace the operands.
-template <int EPI>
+// Drain a 32-row slice of the tile's accumulator (TMEM lane quadrant
+// `quad`, columns from `tmem_col`) into y rows [row0, row0 + 32).  With EW
+// epilogue warps, the EW/4 warps sharing a quadrant take every (EW/4)-th
+// 32-column chunk starting at `part`.  Values are staged in 64-byte rows
+// (64-byte swizzle, conflict-free 16-byte stores) and written by TMA; bf16
+// stores are marked first-to-evict in L2 (y is written once and not read
+// back here, so it should not displace the operands).  The raw int32 path
+// stores each chunk as two 16-column halves.
+template <int EPI, int EW>
 __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensorMap* ymap, uint32_t tmem_base,
                                                int quad, uint32_t tmem_col, int row0, int n0, int b, float sa,
                                                const float* sColScale, const float* sColBias, uint8_t* ebuf,
-                                               int lane) {
+                                               int lane, int part) {
+    constexpr int kStep = EW / 4;
+    constexpr int kBufs = epi_bufs(EW);
     const uint64_t policy = l2_policy_evict_first();
-    for (int cc = 0; cc < BN / 32; ++cc) {
+    const int sw = (lane >> 1) & 3;  // 64-byte swizzle: chunk j of row `lane` sits at j ^ sw
+    uint8_t* rowp_base = ebuf + lane * kEpiRowBytes;
+    int nbuf = 0;  // staging buffers used so far by this call
+    for (int cc = part; cc < BN / 32; cc += kStep) {
         if (n0 + cc * 32 >= p.N) break;  // whole chunk past the last column
         uint32_t r[32];
         tmem_ld_32x32b_x32(
             tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tmem_col + static_cast<uint32_t>(cc * 32), r);
         tmem_ld_wait();
         if constexpr (EPI == kEpiS32) {
-            // 32 int32 = 128 bytes per row, 128-byte swizzle, single buffer
-            if (lane == 0) bulk_wait_group_read<0>();
-            __syncwarp();
-            uint8_t* rowp = ebuf + lane * 128;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
-                    make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_3d_hint(ymap, ebuf, n0 + cc * 32, row0, b, policy);
-                bulk_commit_group();
+            for (int h = 0; h < 2; ++h) {
+                if (n0 + cc * 32 + h * 16 >= p.N) break;
+                uint8_t* buf = ebuf + (nbuf % kBufs) * kEpiBufBytes;
+                if (lane == 0) {
+                    if constexpr (kBufs == 1) bulk_wait_group_read<0>();
+                    else bulk_wait_group_read<1>();
+                }
+                __syncwarp();
+                uint8_t* rowp = buf + lane * kEpiRowBytes;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
+                        make_uint4(r[16 * h + 4 * j], r[16 * h + 4 * j + 1], r[16 * h + 4 * j + 2],
+                                   r[16 * h + 4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(ymap, buf, n0 + cc * 32 + h * 16, row0, b);
+                    bulk_commit_group();
+                }
+                ++nbuf;
             }
         } else {
-            // 32 bf16 = 64 bytes per row, 64-byte swizzle, two buffers
-            uint8_t* buf = ebuf + (cc & 1) * 2048;
-            if (lane == 0) bulk_wait_group_read<1>();
-            __syncwarp();
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -114,21 +131,28 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
                 }
                 w[j] = pack_bf16x2(y0, y1);
             }
-            uint8_t* rowp = buf + lane * 64;
-            const int sw = (lane >> 1) & 3;
+            // The values are ready; now wait until the buffer is free again.
+            uint8_t* buf = ebuf + (nbuf % kBufs) * kEpiBufBytes;
+            if (lane == 0) {
+                if constexpr (kBufs == 1) bulk_wait_group_read<0>();
+                else bulk_wait_group_read<1>();
+            }
+            __syncwarp();
+            uint8_t* rowp = buf + lane * kEpiRowBytes;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 4; ++j)
                 *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) =
                     make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 tma_store_3d_hint(ymap, buf, n0 + cc * 32, row0, b, policy);
                 bulk_commit_group();
             }
+            ++nbuf;
         }
     }
+    (void)rowp_base;
 }
 
 }  // namespace gcore

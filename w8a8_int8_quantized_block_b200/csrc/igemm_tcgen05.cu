@@ -18,7 +18,8 @@
 //   warp 1      MMA issuer: one thread issues tcgen05.mma kind::i8 (K = 32
 //               per instruction) into a TMEM accumulator; tcgen05.commit
 //               frees each stage and, per tile, signals the epilogue
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, scale + bias
+//   warps 2..    epilogue (4 warps, or 8 for CTA pairs: two per TMEM lane
+//               quadrant): tcgen05.ld 32 columns at a time, scale + bias
 //               (+ GELU), bf16, swizzled shared staging, TMA store
 // Two 256-column accumulators (all 512 TMEM columns) let the epilogue of one
 // tile overlap the main loop of the next.  Tiles run n-fastest so an A panel
@@ -49,7 +50,10 @@ namespace {
 
 using namespace gcore;
 
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kEpiWarps1 = 4;  // single-CTA tiles: one epilogue warp per TMEM lane quadrant
+constexpr int kEpiWarpsP = 8;  // CTA pairs: two per quadrant, alternate 32-column chunks
+constexpr int kThreads1 = (2 + kEpiWarps1) * 32;
+constexpr int kThreadsP = (2 + kEpiWarpsP) * 32;
 
 // single-CTA tiles
 constexpr int BM1 = kGemmBM;  // 128
@@ -58,7 +62,7 @@ constexpr int kAStage1 = BM1 * BK;  // 16 KB
 constexpr int kBStage1 = BN * BK;   // 32 KB
 constexpr int kSmemRing1 = kStages1 * (kAStage1 + kBStage1);
 constexpr int kSmemBars1 = 8 * (2 * kStages1 + 2 * kAccBufs) + 16;
-constexpr int kSmemTotal1 = kSmemRing1 + kSmemEpi + kSmemCols + kSmemBars1 + 1024;
+constexpr int kSmemTotal1 = kSmemRing1 + epi_smem(kEpiWarps1) + kSmemBars1 + 1024;
 static_assert(kSmemTotal1 <= 227 * 1024, "shared memory budget");
 
 // CTA-pair tiles
@@ -68,13 +72,13 @@ constexpr int kAStageP = kGemmBM * BK;   // 16 KB: this CTA's 128 rows of A
 constexpr int kBStageP = (BN / 2) * BK;  // 16 KB: this CTA's half of B
 constexpr int kSmemRingP = kStagesP * (kAStageP + kBStageP);
 constexpr int kSmemBarsP = 8 * (2 * kStagesP + 2 * kAccBufs) + 16;
-constexpr int kSmemTotalP = kSmemRingP + kSmemEpi + kSmemCols + kSmemBarsP + 1024;
+constexpr int kSmemTotalP = kSmemRingP + epi_smem(kEpiWarpsP) + kSmemBarsP + 1024;
 static_assert(kSmemTotalP <= 227 * 1024, "shared memory budget");
 
 // ============================================================================ single-CTA tiles
 
 template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads1, 1)
     igemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                  const __grid_constant__ CUtensorMap ymap, const GemmArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -82,8 +86,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages1 * kAStage1;
     uint8_t* sEpi = smem + kSmemRing1;
-    float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);  // [warp][scale | bias][BN]
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);
+    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarps1 * epi_bufs(kEpiWarps1) * kEpiBufBytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps1 * 2 * BN);
     uint64_t* empty_bar = full_bar + kStages1;
     uint64_t* accf_bar = empty_bar + kStages1;
     uint64_t* acce_bar = accf_bar + kAccBufs;
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < kAccBufs; ++a) {
             mbar_init(&accf_bar[a], 1);
-            mbar_init(&acce_bar[a], kEpiWarps * 32);
+            mbar_init(&acce_bar[a], kEpiWarps1 * 32);
         }
         fence_mbar_init();
     }
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // -------------------------------------------------------------- epilogue
         const int ew = warp - 2;    // 0..3
         const int quad = warp & 3;  // TMEM lane quadrant this warp may read
-        uint8_t* ebuf = sEpi + ew * kEpiBufBytes;
+        uint8_t* ebuf = sEpi + ew * epi_bufs(kEpiWarps1) * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         int acc = 0;
@@ -207,8 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (row0 + lane < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + row0 + lane];
             }
             if (ok && row0 < p.M)
-                epilogue_slice<EPI>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0, c.b, sa,
-                                    sColScale, sColBias, ebuf, lane);
+                epilogue_slice<EPI, kEpiWarps1>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0,
+                                                c.b, sa, sColScale, sColBias, ebuf, lane, 0);
             tc_fence_before_sync();
             mbar_arrive(&acce_bar[acc]);
             if (!ok) break;
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================ CTA-pair tiles
 
 template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsP, 1)
     igemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                       const __grid_constant__ CUtensorMap ymap, const GemmArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -239,8 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStagesP * kAStageP;
     uint8_t* sEpi = smem + kSmemRingP;
-    float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);  // used in the leader
+    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarpsP * epi_bufs(kEpiWarpsP) * kEpiBufBytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarpsP * 2 * BN);  // used in the leader
     uint64_t* empty_bar = full_bar + kStagesP;                                       // in both CTAs
     uint64_t* accf_bar = empty_bar + kStagesP;                                       // in both CTAs
     uint64_t* acce_bar = accf_bar + kAccBufs;                                        // used in the leader
@@ -266,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < kAccBufs; ++a) {
             mbar_init(&accf_bar[a], 1);              // the leader's commit arrives (multicast)
-            mbar_init(&acce_bar[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs
+            mbar_init(&acce_bar[a], 2 * kEpiWarpsP);  // every epilogue warp of both CTAs
         }
         fence_mbar_init();
     }
@@ -352,9 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue (both CTAs)
-        const int ew = warp - 2;
-        const int quad = warp & 3;
-        uint8_t* ebuf = sEpi + ew * kEpiBufBytes;
+        const int ew = warp - 2;     // 0..7
+        const int quad = warp & 3;   // TMEM lane quadrant this warp may read
+        const int part = ew >> 2;    // which alternate 32-column chunks it drains
+        uint8_t* ebuf = sEpi + ew * epi_bufs(kEpiWarpsP) * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         const uint32_t leader_acce0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
@@ -371,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (row0 + lane < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + row0 + lane];
             }
             if (ok && row0 < p.M)
-                epilogue_slice<EPI>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0, c.b, sa,
-                                    sColScale, sColBias, ebuf, lane);
+                epilogue_slice<EPI, kEpiWarpsP>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0,
+                                                c.b, sa, sColScale, sColBias, ebuf, lane, part);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acce0 + static_cast<uint32_t>(acc * 8));
@@ -403,7 +408,7 @@ cudaError_t launch_single(const CUtensorMap& amap, const CUtensorMap& bmap, cons
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kThreads1);
     cfg.dynamicSmemBytes = kSmemTotal1;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -424,7 +429,7 @@ cudaError_t launch_pair(const CUtensorMap& amap, const CUtensorMap& bmap, const 
     if (e != cudaSuccess) return e;
     const int64_t tiles = static_cast<int64_t>((a.M + BMP - 1) / BMP) * ((a.N + BN - 1) / BN) * a.batch;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kThreadsP);
     cfg.dynamicSmemBytes = kSmemTotalP;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];

@@ -69,8 +69,9 @@ int gemm_b_box_rows();
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;     // bytes of K per stage (= int8 elements)
-constexpr int kEpiCols = 32;     // output columns per epilogue store
-constexpr int kEpiRows = 32;     // rows per epilogue store (one warp)
+constexpr int kEpiColsBf16 = 32;  // output columns per epilogue store (bf16: 64-byte rows)
+constexpr int kEpiColsS32 = 16;   // output columns per epilogue store (int32: 64-byte rows)
+constexpr int kEpiRows = 32;      // rows per epilogue store (one warp)
 
 // ---------------------------------------------------------------- fused linear (one kernel)
 

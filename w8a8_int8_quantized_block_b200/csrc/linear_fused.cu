@@ -45,7 +45,8 @@ using qcore::kPerThread;
 constexpr int kQGroups = 2;                    // quantiser groups per CTA
 constexpr int kQWarps = 3;                     // warps per group: one row of K <= 6144
 constexpr int kQThreads = kQWarps * 32;
-constexpr int kFirstQWarp = 2 + kEpiWarps;
+constexpr int kEpiWarpsF = 4;  // one epilogue warp per TMEM lane quadrant
+constexpr int kFirstQWarp = 2 + kEpiWarpsF;
 constexpr int kThreadsF = (kFirstQWarp + kQGroups * kQWarps) * 32;
 constexpr int kPanelRows = 2 * kGemmBM;        // 256: the pair's tile height
 // Quantisers stay at most this many panels ahead of the first panel the GEMM
@@ -58,7 +59,7 @@ constexpr int kBStageF = (BN / 2) * BK;
 constexpr int kSmemRingF = kStagesF * (kAStageF + kBStageF);
 constexpr int kSmemBarsF = 8 * (2 * kStagesF + 2 * kAccBufs) + 16;
 constexpr int kSmemRedF = kQGroups * 2 * kQWarps * 4;
-constexpr int kSmemTotalF = kSmemRingF + kSmemEpi + kSmemCols + kSmemBarsF + kSmemRedF + 1024;
+constexpr int kSmemTotalF = kSmemRingF + epi_smem(kEpiWarpsF) + kSmemBarsF + kSmemRedF + 1024;
 static_assert(kSmemTotalF <= 227 * 1024, "shared memory budget");
 static_assert(kQThreads * kPerThread >= kFusedMaxK, "a group must cover a row");
 
@@ -89,8 +90,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStagesF * kAStageF;
     uint8_t* sEpi = smem + kSmemRingF;
-    float* sCols = reinterpret_cast<float*>(sEpi + kSmemEpi);
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps * 2 * BN);
+    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarpsF * epi_bufs(kEpiWarpsF) * kEpiBufBytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarpsF * 2 * BN);
     uint64_t* empty_bar = full_bar + kStagesF;
     uint64_t* accf_bar = empty_bar + kStagesF;
     uint64_t* acce_bar = accf_bar + kAccBufs;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         }
         for (int a = 0; a < kAccBufs; ++a) {
             mbar_init(&accf_bar[a], 1);
-            mbar_init(&acce_bar[a], 2 * kEpiWarps);
+            mbar_init(&acce_bar[a], 2 * kEpiWarpsF);
         }
         fence_mbar_init();
     }
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         // -------------------------------------------------------------- epilogue (both CTAs)
         const int ew = warp - 2;
         const int quad = warp & 3;
-        uint8_t* ebuf = sEpi + ew * kEpiBufBytes;
+        uint8_t* ebuf = sEpi + ew * epi_bufs(kEpiWarpsF) * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         const uint32_t leader_acce0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
@@ -289,8 +290,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             float sa = 0.0f;
             if (ok && row0 + lane < p.M) sa = f.s[row0 + lane];
             if (ok && row0 < p.M)
-                epilogue_slice<EPI>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0, 0, sa,
-                                    sColScale, sColBias, ebuf, lane);
+                epilogue_slice<EPI, kEpiWarpsF>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0,
+                                                0, sa, sColScale, sColBias, ebuf, lane, 0);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acce0 + static_cast<uint32_t>(acc * 8));
