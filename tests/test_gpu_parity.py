@@ -93,6 +93,37 @@ def test_igemm_s32_bitexact(B, M, N, K):
         assert (acc[b].cpu().numpy().astype(np.int64) == ref).all()
 
 
+@pytest.mark.parametrize("B,M,N,K", [(8, 2048, 336, 128), (4, 1536, 80, 256), (2, 2048, 592, 384)])
+def test_igemm_s32_many_ragged_tiles(B, M, N, K):
+    # More tiles than CTA pairs, each ending in a part-filled column tile (an
+    # odd number of 32-column chunks), so every epilogue warp cycles its
+    # staging buffers across tiles of uneven length, and prefetches the next
+    # tile's scales while it drains one that ends short.
+    qa = _codes((B, M, K), 11 + N)
+    qb = _codes((B, N, K), 12 + N)
+    acc = C.igemm_s32(qa.to(DEV), qb.to(DEV)).cpu().numpy().astype(np.int64)
+    assert C.last_device_status() == (C.OK, 0)
+    for b in range(B):
+        assert (acc[b] == O.igemm(qa[b].numpy(), qb[b].numpy())).all(), f"batch {b}"
+
+
+def test_bmm_many_ragged_tiles_matches_oracle():
+    B, M, N, K = 8, 2048, 336, 128
+    q, k = W.bmm_inputs(W.QK_BMM, M=M, N=N)
+    q, k = q[:B], k[:B]
+    qa, sa = C.quantize_act(q.to(DEV).reshape(B * M, K), 0)
+    qb, sb = C.quantize_act(k.to(DEV).reshape(B * N, K), 0)
+    y = C.w8a8_bmm(qa.view(B, M, K), sa, qb.view(B, N, K), sb)
+    torch.cuda.synchronize()
+    assert C.last_device_status() == (C.OK, 0)
+    qar, sar = O.quantize_act(bits(q.reshape(B * M, K)), 0)
+    qbr, sbr = O.quantize_act(bits(k.reshape(B * N, K)), 0)
+    for b in range(B):
+        acc = O.igemm(qar[b * M:(b + 1) * M], qbr[b * N:(b + 1) * N])
+        yr = O.dequant(acc, sar[b * M:(b + 1) * M], sbr[b * N:(b + 1) * N], None, 0)
+        assert_close_bf16(f32_of_bf16(y[b]), yr, f"bmm head {b}")
+
+
 def test_igemm_s32_extreme_accumulators():
     K = 21504
     qa = torch.full((1, 130, K), -127, dtype=torch.int8)
@@ -144,6 +175,18 @@ def test_linear_ragged_shapes(M, K, N):
     y, pw = _run_linear((x, w, bias), fused=True)
     yr, *_ = O.linear(bits(x), w.numpy(), bias.numpy(), 128)
     assert_close_bf16(f32_of_bf16(y), yr, f"linear {M}x{K}x{N}")
+
+
+def test_linear_fused_many_ragged_tiles():
+    # 32 row panels x 3 column tiles (256, 256, 80 columns): more tiles than
+    # CTA pairs, and every third tile drains an odd number of 32-column chunks
+    # through the epilogue's two staging buffers.
+    M, K, N = 8192, 512, 592
+    spec, (x, w, bias) = W.custom_linear(M, K, N, seed=17, n_out=5, token_scale=True)
+    y, pw = _run_linear((x, w, bias), fused=True)
+    assert C.last_device_status() == (C.OK, 0)
+    yr, *_ = O.linear(bits(x), w.numpy(), bias.numpy(), 128)
+    assert_close_bf16(f32_of_bf16(y), yr, "linear 8192x512x592")
 
 
 @pytest.mark.parametrize("pad", [8, 16])

@@ -19,11 +19,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kEpiRowBytes = 64;                  // one staged row: 32 bf16 or 16 int32
 constexpr int kEpiBufBytes = 32 * kEpiRowBytes;   // one 32-row staging buffer (64-byte swizzle)
 
-// Shared memory the epilogue of `ew` warps needs: staging buffers (two per
-// warp with four warps, one per warp with eight) and a private copy of the
-// tile's column scales and biases per warp.
-__host__ __device__ constexpr int epi_bufs(int ew) { return ew == 4 ? 2 : 1; }
-__host__ __device__ constexpr int epi_smem(int ew) { return ew * (epi_bufs(ew) * kEpiBufBytes + 2 * BN * 4); }
+// Shared memory the epilogue of `ew` warps with `bufs` staging buffers each
+// needs: the buffers and a private copy of the tile's column scales and
+// biases per warp.
+__host__ __device__ constexpr int epi_smem(int ew, int bufs) { return ew * (bufs * kEpiBufBytes + 2 * BN * 4); }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     const uint32_t a = smem_u32(p);
@@ -67,6 +66,45 @@ __device__ __forceinline__ void load_tile_columns(const GemmArgs& p, const TileC
     }
 }
 
+// A tile's column scales and biases (raw s_b, not yet times alpha) and this
+// lane's row scale, fetched into registers one tile ahead so that the global
+// loads' latency overlaps the previous tile's drain instead of preceding it.
+struct TileScales {
+    float col_scale[BN / 32];
+    float col_bias[BN / 32];
+    float row_scale;
+};
+
+template <int EPI>
+__device__ __forceinline__ void fetch_tile_scales(const GemmArgs& p, const TileCoord& c, int row, int lane,
+                                                  TileScales& ts) {
+    if constexpr (EPI != kEpiS32) {
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) {
+            const int n = c.n0 + lane + 32 * j;
+            const bool in = n < p.N;
+            ts.col_scale[j] = in ? p.s_b[static_cast<int64_t>(c.b) * p.N + n] : 0.0f;
+            ts.col_bias[j] = (in && p.bias != nullptr) ? p.bias[n] : 0.0f;
+        }
+        ts.row_scale = row < p.M ? p.s_a[static_cast<int64_t>(c.b) * p.M + row] : 0.0f;
+    }
+}
+
+// The prefetched column values into this warp's private shared-memory copy.
+template <int EPI>
+__device__ __forceinline__ void store_tile_columns(const TileScales& ts, float alpha, float* sColScale,
+                                                   float* sColBias, int lane) {
+    if constexpr (EPI != kEpiS32) {
+        __syncwarp();  // every lane is done with the previous tile's columns
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) {
+            sColScale[lane + 32 * j] = ts.col_scale[j] * alpha;
+            sColBias[lane + 32 * j] = ts.col_bias[j];
+        }
+        __syncwarp();
+    }
+}
+
 // Drain a 32-row slice of the tile's accumulator (TMEM lane quadrant
 // `quad`, columns from `tmem_col`) into y rows [row0, row0 + 32).  With EW
 // epilogue warps, the EW/4 warps sharing a quadrant take every (EW/4)-th
@@ -74,18 +112,19 @@ __device__ __forceinline__ void load_tile_columns(const GemmArgs& p, const TileC
 // (64-byte swizzle, conflict-free 16-byte stores) and written by TMA; bf16
 // stores are marked first-to-evict in L2 (y is written once and not read
 // back here, so it should not displace the operands).  The raw int32 path
-// stores each chunk as two 16-column halves.
-template <int EPI, int EW>
+// stores each chunk as two 16-column halves.  The warp's NBUF staging
+// buffers rotate through `nbuf`, which the caller keeps across tiles: a
+// buffer is rewritten only after the store that last read it (NBUF stores
+// ago) has finished reading, however many chunks a ragged tile had.
+template <int EPI, int EW, int NBUF>
 __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensorMap* ymap, uint32_t tmem_base,
                                                int quad, uint32_t tmem_col, int row0, int n0, int b, float sa,
                                                const float* sColScale, const float* sColBias, uint8_t* ebuf,
-                                               int lane, int part) {
+                                               int lane, int part, int& nbuf) {
     constexpr int kStep = EW / 4;
-    constexpr int kBufs = epi_bufs(EW);
+    static_assert(NBUF >= 1, "at least one staging buffer");
     const uint64_t policy = l2_policy_evict_first();
     const int sw = (lane >> 1) & 3;  // 64-byte swizzle: chunk j of row `lane` sits at j ^ sw
-    uint8_t* rowp_base = ebuf + lane * kEpiRowBytes;
-    int nbuf = 0;  // staging buffers used so far by this call
     for (int cc = part; cc < BN / 32; cc += kStep) {
         if (n0 + cc * 32 >= p.N) break;  // whole chunk past the last column
         uint32_t r[32];
@@ -96,11 +135,8 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 if (n0 + cc * 32 + h * 16 >= p.N) break;
-                uint8_t* buf = ebuf + (nbuf % kBufs) * kEpiBufBytes;
-                if (lane == 0) {
-                    if constexpr (kBufs == 1) bulk_wait_group_read<0>();
-                    else bulk_wait_group_read<1>();
-                }
+                uint8_t* buf = ebuf + nbuf * kEpiBufBytes;
+                if (lane == 0) bulk_wait_group_read<NBUF - 1>();
                 __syncwarp();
                 uint8_t* rowp = buf + lane * kEpiRowBytes;
 #pragma unroll
@@ -114,7 +150,7 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
                     tma_store_3d(ymap, buf, n0 + cc * 32 + h * 16, row0, b);
                     bulk_commit_group();
                 }
-                ++nbuf;
+                if (++nbuf == NBUF) nbuf = 0;
             }
         } else {
             uint32_t w[16];
@@ -132,11 +168,8 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
                 w[j] = pack_bf16x2(y0, y1);
             }
             // The values are ready; now wait until the buffer is free again.
-            uint8_t* buf = ebuf + (nbuf % kBufs) * kEpiBufBytes;
-            if (lane == 0) {
-                if constexpr (kBufs == 1) bulk_wait_group_read<0>();
-                else bulk_wait_group_read<1>();
-            }
+            uint8_t* buf = ebuf + nbuf * kEpiBufBytes;
+            if (lane == 0) bulk_wait_group_read<NBUF - 1>();
             __syncwarp();
             uint8_t* rowp = buf + lane * kEpiRowBytes;
 #pragma unroll
@@ -149,10 +182,9 @@ __device__ __forceinline__ void epilogue_slice(const GemmArgs& p, const CUtensor
                 tma_store_3d_hint(ymap, buf, n0 + cc * 32, row0, b, policy);
                 bulk_commit_group();
             }
-            ++nbuf;
+            if (++nbuf == NBUF) nbuf = 0;
         }
     }
-    (void)rowp_base;
 }
 
 }  // namespace gcore

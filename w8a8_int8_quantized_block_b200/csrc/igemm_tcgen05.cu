@@ -58,21 +58,23 @@ constexpr int kThreadsP = (2 + kEpiWarpsP) * 32;
 // single-CTA tiles
 constexpr int BM1 = kGemmBM;  // 128
 constexpr int kStages1 = 4;
+constexpr int kEpiBufs1 = 2;
 constexpr int kAStage1 = BM1 * BK;  // 16 KB
 constexpr int kBStage1 = BN * BK;   // 32 KB
 constexpr int kSmemRing1 = kStages1 * (kAStage1 + kBStage1);
 constexpr int kSmemBars1 = 8 * (2 * kStages1 + 2 * kAccBufs) + 16;
-constexpr int kSmemTotal1 = kSmemRing1 + epi_smem(kEpiWarps1) + kSmemBars1 + 1024;
+constexpr int kSmemTotal1 = kSmemRing1 + epi_smem(kEpiWarps1, kEpiBufs1) + kSmemBars1 + 1024;
 static_assert(kSmemTotal1 <= 227 * 1024, "shared memory budget");
 
 // CTA-pair tiles
 constexpr int BMP = 2 * kGemmBM;         // 256 rows per pair, 128 per CTA
-constexpr int kStagesP = 6;
 constexpr int kAStageP = kGemmBM * BK;   // 16 KB: this CTA's 128 rows of A
 constexpr int kBStageP = (BN / 2) * BK;  // 16 KB: this CTA's half of B
+constexpr int kStagesP = 6;
+constexpr int kEpiBufsP = 1;  // with eight epilogue warps one staging buffer each fits beside 6 stages
 constexpr int kSmemRingP = kStagesP * (kAStageP + kBStageP);
 constexpr int kSmemBarsP = 8 * (2 * kStagesP + 2 * kAccBufs) + 16;
-constexpr int kSmemTotalP = kSmemRingP + epi_smem(kEpiWarpsP) + kSmemBarsP + 1024;
+constexpr int kSmemTotalP = kSmemRingP + epi_smem(kEpiWarpsP, kEpiBufsP) + kSmemBarsP + 1024;
 static_assert(kSmemTotalP <= 227 * 1024, "shared memory budget");
 
 // ============================================================================ single-CTA tiles
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages1 * kAStage1;
     uint8_t* sEpi = smem + kSmemRing1;
-    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarps1 * epi_bufs(kEpiWarps1) * kEpiBufBytes);
+    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarps1 * kEpiBufs1 * kEpiBufBytes);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarps1 * 2 * BN);
     uint64_t* empty_bar = full_bar + kStages1;
     uint64_t* accf_bar = empty_bar + kStages1;
@@ -195,24 +197,31 @@ __global__ void __launch_bounds__(kThreads1, 1)
         // -------------------------------------------------------------- epilogue
         const int ew = warp - 2;    // 0..3
         const int quad = warp & 3;  // TMEM lane quadrant this warp may read
-        uint8_t* ebuf = sEpi + ew * epi_bufs(kEpiWarps1) * kEpiBufBytes;
+        uint8_t* ebuf = sEpi + ew * kEpiBufs1 * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         int acc = 0;
         uint32_t acc_phase = 0;
+        int nbuf = 0;
+        TileScales next{};
+        if (blockIdx.x < num_tiles) {
+            const TileCoord c = tile_coord(blockIdx.x, tiles_m, tiles_n, BM1);
+            fetch_tile_scales<EPI>(p, c, c.m0 + quad * 32 + lane, lane, next);
+        }
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1);
-            load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
+            store_tile_columns<EPI>(next, p.alpha, sColScale, sColBias, lane);
+            const float sa = next.row_scale;
+            if (t + static_cast<int>(gridDim.x) < num_tiles) {
+                const TileCoord cn = tile_coord(t + gridDim.x, tiles_m, tiles_n, BM1);
+                fetch_tile_scales<EPI>(p, cn, cn.m0 + quad * 32 + lane, lane, next);
+            }
             const bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
             tc_fence_after_sync();
             const int row0 = c.m0 + quad * 32;
-            float sa = 0.0f;
-            if constexpr (EPI != kEpiS32) {
-                if (row0 + lane < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + row0 + lane];
-            }
             if (ok && row0 < p.M)
-                epilogue_slice<EPI, kEpiWarps1>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0,
-                                                c.b, sa, sColScale, sColBias, ebuf, lane, 0);
+                epilogue_slice<EPI, kEpiWarps1, kEpiBufs1>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN),
+                                                           row0, c.n0, c.b, sa, sColScale, sColBias, ebuf, lane, 0, nbuf);
             tc_fence_before_sync();
             mbar_arrive(&acce_bar[acc]);
             if (!ok) break;
@@ -243,7 +252,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStagesP * kAStageP;
     uint8_t* sEpi = smem + kSmemRingP;
-    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarpsP * epi_bufs(kEpiWarpsP) * kEpiBufBytes);
+    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarpsP * kEpiBufsP * kEpiBufBytes);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarpsP * 2 * BN);  // used in the leader
     uint64_t* empty_bar = full_bar + kStagesP;                                       // in both CTAs
     uint64_t* accf_bar = empty_bar + kStagesP;                                       // in both CTAs
@@ -359,25 +368,34 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         const int ew = warp - 2;     // 0..7
         const int quad = warp & 3;   // TMEM lane quadrant this warp may read
         const int part = ew >> 2;    // which alternate 32-column chunks it drains
-        uint8_t* ebuf = sEpi + ew * epi_bufs(kEpiWarpsP) * kEpiBufBytes;
+        uint8_t* ebuf = sEpi + ew * kEpiBufsP * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         const uint32_t leader_acce0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
+        int nbuf = 0;
+        const int row_off = static_cast<int>(rank) * kGemmBM + quad * 32;  // this warp's rows within the tile
+        TileScales next{};
+        if (pair < num_tiles) {
+            const TileCoord c = tile_coord(pair, tiles_m, tiles_n, BMP);
+            fetch_tile_scales<EPI>(p, c, c.m0 + row_off + lane, lane, next);
+        }
         for (int t = pair; t < num_tiles; t += num_pairs) {
             const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP);
-            load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
+            store_tile_columns<EPI>(next, p.alpha, sColScale, sColBias, lane);
+            const float sa = next.row_scale;
+            if (t + num_pairs < num_tiles) {
+                const TileCoord cn = tile_coord(t + num_pairs, tiles_m, tiles_n, BMP);
+                fetch_tile_scales<EPI>(p, cn, cn.m0 + row_off + lane, lane, next);
+            }
             const bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
             tc_fence_after_sync();
-            const int row0 = c.m0 + static_cast<int>(rank) * kGemmBM + quad * 32;
-            float sa = 0.0f;
-            if constexpr (EPI != kEpiS32) {
-                if (row0 + lane < p.M) sa = p.s_a[static_cast<int64_t>(c.b) * p.M + row0 + lane];
-            }
+            const int row0 = c.m0 + row_off;
             if (ok && row0 < p.M)
-                epilogue_slice<EPI, kEpiWarpsP>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0,
-                                                c.b, sa, sColScale, sColBias, ebuf, lane, part);
+                epilogue_slice<EPI, kEpiWarpsP, kEpiBufsP>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN),
+                                                          row0, c.n0, c.b, sa, sColScale, sColBias, ebuf, lane, part,
+                                                          nbuf);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acce0 + static_cast<uint32_t>(acc * 8));

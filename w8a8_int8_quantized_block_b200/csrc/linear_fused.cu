@@ -46,6 +46,7 @@ constexpr int kQGroups = 2;                    // quantiser groups per CTA
 constexpr int kQWarps = 3;                     // warps per group: one row of K <= 6144
 constexpr int kQThreads = kQWarps * 32;
 constexpr int kEpiWarpsF = 4;  // one epilogue warp per TMEM lane quadrant
+constexpr int kEpiBufsF = 2;   // staging buffers per epilogue warp
 constexpr int kFirstQWarp = 2 + kEpiWarpsF;
 constexpr int kThreadsF = (kFirstQWarp + kQGroups * kQWarps) * 32;
 constexpr int kPanelRows = 2 * kGemmBM;        // 256: the pair's tile height
@@ -59,7 +60,7 @@ constexpr int kBStageF = (BN / 2) * BK;
 constexpr int kSmemRingF = kStagesF * (kAStageF + kBStageF);
 constexpr int kSmemBarsF = 8 * (2 * kStagesF + 2 * kAccBufs) + 16;
 constexpr int kSmemRedF = kQGroups * 2 * kQWarps * 4;
-constexpr int kSmemTotalF = kSmemRingF + epi_smem(kEpiWarpsF) + kSmemBarsF + kSmemRedF + 1024;
+constexpr int kSmemTotalF = kSmemRingF + epi_smem(kEpiWarpsF, kEpiBufsF) + kSmemBarsF + kSmemRedF + 1024;
 static_assert(kSmemTotalF <= 227 * 1024, "shared memory budget");
 static_assert(kQThreads * kPerThread >= kFusedMaxK, "a group must cover a row");
 
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStagesF * kAStageF;
     uint8_t* sEpi = smem + kSmemRingF;
-    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarpsF * epi_bufs(kEpiWarpsF) * kEpiBufBytes);
+    float* sCols = reinterpret_cast<float*>(sEpi + kEpiWarpsF * kEpiBufsF * kEpiBufBytes);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sCols + kEpiWarpsF * 2 * BN);
     uint64_t* empty_bar = full_bar + kStagesF;
     uint64_t* accf_bar = empty_bar + kStagesF;
@@ -268,12 +269,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         // -------------------------------------------------------------- epilogue (both CTAs)
         const int ew = warp - 2;
         const int quad = warp & 3;
-        uint8_t* ebuf = sEpi + ew * epi_bufs(kEpiWarpsF) * kEpiBufBytes;
+        uint8_t* ebuf = sEpi + ew * kEpiBufsF * kEpiBufBytes;
         float* sColScale = sCols + ew * 2 * BN;
         float* sColBias = sColScale + BN;
         const uint32_t leader_acce0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
+        int nbuf = 0;
         for (int t = pair; t < num_tiles; t += num_pairs) {
             const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows);
             load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
@@ -290,8 +292,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             float sa = 0.0f;
             if (ok && row0 + lane < p.M) sa = f.s[row0 + lane];
             if (ok && row0 < p.M)
-                epilogue_slice<EPI, kEpiWarpsF>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN), row0, c.n0,
-                                                0, sa, sColScale, sColBias, ebuf, lane, 0);
+                epilogue_slice<EPI, kEpiWarpsF, kEpiBufsF>(p, &ymap, tmem_base, quad, static_cast<uint32_t>(acc * BN),
+                                                           row0, c.n0, 0, sa, sColScale, sColBias, ebuf, lane, 0, nbuf);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acce0 + static_cast<uint32_t>(acc * 8));
