@@ -19,6 +19,7 @@ MUTANTS = {
     "butterfly_sign": ("v[j + h] = u - w;", "v[j + h] = w - u;"),
     "missing_last_stage": ("for (int h = 1; h < b; h <<= 1) {", "for (int h = 1; h < b / 2; h <<= 1) {"),
     "round_half_away": ("float r = rintf(v);", "float r = roundf(v);"),
+    "product_rounded_once": ("float r = rintf(v); /*", "float r = (float)rint((double)z[k] * (double)inv); /*"),
     "scale_over_128": ("*s = amax / 127.0f;", "*s = amax / 128.0f;"),
     "inverse_scale_128": ("float inv = 127.0f / amax;", "float inv = 128.0f / amax;"),
     "zero_row_scale_one": ("        *s = 0.0f;\n        memset(q, 0, (size_t)K);", "        *s = 1.0f;\n        memset(q, 0, (size_t)K);"),

@@ -285,3 +285,19 @@ def test_rotated_linear_equals_unrotated_math_on_exact_inputs():
     zx = np.stack([O.fwht(r, b) for r in xz]).astype(np.int64)
     zw = np.stack([O.fwht(r, b) for r in wz]).astype(np.int64)
     assert ((zx @ zw.T) == b * (xz.astype(np.int64) @ wz.astype(np.int64).T)).all()
+
+
+@pytest.mark.parametrize("block", [128, 0])
+def test_quantiser_rounds_the_f32_product_before_the_integer(block):
+    # Rows where f32(z * inv) is exactly 63.5 but z * inv is a little below:
+    # rounding twice gives 64 (ties to even), rounding the exact product once
+    # would give 63.  Every such element must come out as +-64.
+    from near_ties import plain_rows, rotated_rows
+    x = rotated_rows() if block == 128 else plain_rows()
+    q, s = O.quantize_act(_bf16(x), block)
+    half = np.abs(x) > 0
+    assert (np.abs(q) == 64).sum() >= x.shape[0]
+    assert not (np.abs(q) == 63).any()
+    if block == 0:
+        # the a/2 entries are exactly the near-tie elements
+        assert ((np.abs(q) == 64) == (half & (np.abs(x) < x.max(axis=1, keepdims=True)))).all()

@@ -13,7 +13,7 @@ namespace convrot {
 // Launch geometry of the rotate+quantise kernel for one row length.
 struct RqGeometry {
     int tpr;           // threads holding data in one row (K / 32)
-    int tpr_pad;       // threads per row including idle ones
+    int tpr_pad;       // threads per row including idle ones (long rows: = tpr, packed back to back)
     int rows_per_cta;  // rows one CTA handles
     int threads;       // CTA size
     int rows128;       // 128-byte shared-memory rows per input row

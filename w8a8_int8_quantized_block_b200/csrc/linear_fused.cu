@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             for (int i = 1; i < kQWarps; ++i) amax = fmaxf(amax, gred[(it & 1) * kQWarps + i]);
             if (holds) {
                 const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-                qcore::quantize_store(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
+                qcore::quantize_store<false>(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
                 if (t == 0) f.s[row] = __fdiv_rn(amax, 127.0f);
             }
             __threadfence();                    // this thread's codes are visible device-wide

@@ -162,14 +162,28 @@ __device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[kPairs], int sh,
 }
 
 // Round and store this thread's codes: v = z * inv rounded to f32 (packed
-// multiply), then round-half-to-even to int32 (|v| <= 127*(1+2^-24) < 127.5,
-// so no clamp can bind); byte permutes pack four codes per word; two 32-byte
-// stores write the thread's 64 codes at `dst` (32-byte aligned).
-// The product must be rounded on its own before the integer rounding: the
-// usual "add 1.5*2^23" trick was contracted with the packed multiply into one
-// FMA, which rounds the exact product instead.
+// multiply), then rounded half-to-even to an integer (|v| <= 127*(1+2^-24) <
+// 127.5, so no clamp can bind); byte permutes pack four codes per word; two
+// 32-byte stores write the thread's 64 codes at `dst` (32-byte aligned).
+//
+// Two ways to round v to an integer:
+//   kMagicAdd = false: cvt.rni to int32, one conversion per element.
+//   kMagicAdd = true:  a packed fma(v, 1, 1.5 * 2^23), half an instruction
+//     per element and no conversion unit.  Near 1.5 * 2^23 the f32 spacing is
+//     exactly 1, so the fma (v * 1 is exact, so it is the plain add) rounds v
+//     half-to-even to an integer, and the low byte of the sum's bits is the
+//     code in two's complement.  The multiply and this add must stay two
+//     separate roundings: fused into one FMA they would round the exact
+//     product instead, which moves values that sit within half an ulp of a
+//     tie.  Written as a plain packed add (add.rn.f32x2), ptxas fused it with
+//     the packed multiply even with -fmad=false; as fma(v, 1, c) there is no
+//     multiply-add pair to fuse.  Crafted rows whose f32 product is exactly
+//     k + 1/2 while the exact product is not check this on the GPU.
+template <bool kMagicAdd>
 __device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], float inv, int8_t* dst) {
     const uint64_t inv2 = pk(inv, inv);
+    const uint64_t one2 = pk(1.0f, 1.0f);
+    const uint64_t magic2 = pk(12582912.0f, 12582912.0f);  // 1.5 * 2^23
     // Pairs 4i..4i+3 hold elements 4i..4i+3 (low halves) and kPairs+4i..+3
     // (high halves): each group of four pairs completes word i and word
     // kPairs/4 + i, so the codes are packed as soon as they exist.
@@ -180,9 +194,15 @@ __device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], floa
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             float a, b;
-            upk(mul2(P[4 * i + k], inv2), a, b);
-            lo[k] = static_cast<uint32_t>(__float2int_rn(a));
-            hi[k] = static_cast<uint32_t>(__float2int_rn(b));
+            if constexpr (kMagicAdd) {
+                upk(fma2(mul2(P[4 * i + k], inv2), one2, magic2), a, b);
+                lo[k] = __float_as_uint(a);
+                hi[k] = __float_as_uint(b);
+            } else {
+                upk(mul2(P[4 * i + k], inv2), a, b);
+                lo[k] = static_cast<uint32_t>(__float2int_rn(a));
+                hi[k] = static_cast<uint32_t>(__float2int_rn(b));
+            }
         }
         word[i] = prmt(prmt(lo[0], lo[1], 0x0040u), prmt(lo[2], lo[3], 0x0040u), 0x5410u);
         word[kPairs / 4 + i] = prmt(prmt(hi[0], hi[1], 0x0040u), prmt(hi[2], hi[3], 0x0040u), 0x5410u);

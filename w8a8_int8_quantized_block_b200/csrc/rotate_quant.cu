@@ -23,15 +23,18 @@
 //     values and one packed FMA with a +-1 sign computes self + partner on
 //     the lower side and partner - self on the upper side, each rounded once
 //     exactly like the add or subtract it replaces;
-//   - the row absmax is reduced with shuffles (and shared memory when a row
-//     spans several warps);
-//   - codes: v = z * (127/amax) (packed multiply, rounded), then a
-//     round-to-nearest-even conversion to int32 (|v| <= 127*(1+2^-24) < 127.5,
-//     so no clamp can bind); byte permutes pack four codes per word and two
-//     32-byte stores write the thread's 64 codes.  (The product must be rounded
-//     on its own before the integer rounding: adding 1.5*2^23 to round was
-//     contracted with the packed multiply into one FMA, which rounds the exact
-//     product instead and moves values that sit within half an ulp of a tie.)
+//   - the row absmax is reduced with shuffles when a row fits in a warp;
+//     longer rows are packed back to back (no padding threads between them,
+//     so a 5376-element row takes 84 threads and three rows fill eight
+//     warps): a max-reduction over each warp's segment of a row, then one
+//     64-bit shared-memory atomicMax per segment, tagged with the group's
+//     iteration so that no reset between groups is needed;
+//   - codes: v = z * (127/amax) (packed multiply, rounded), then a packed
+//     fma(v, 1, 1.5*2^23) rounds v half-to-even to an integer whose low byte
+//     is the code (|v| <= 127*(1+2^-24) < 127.5, so no clamp can bind); byte
+//     permutes pack four codes per word and two 32-byte stores write the
+//     thread's 64 codes.  The product is rounded on its own before the
+//     integer rounding, as the definition has it (see quantize_store).
 // The arithmetic is therefore the same sequence of IEEE single-precision
 // operations as the plain definition, in the same order.
 #include <cuda_bf16.h>
@@ -56,10 +59,11 @@ constexpr int kMaxThreads = kPerThread == 32 ? 1024 : 512;
 #ifndef CONVROT_RQ_STAGES
 #define CONVROT_RQ_STAGES 2  // ring slots (row groups in flight) per CTA
 #endif
-#ifndef CONVROT_RQ_LONG_ROWS
-#define CONVROT_RQ_LONG_ROWS 1  // rows per group when a row spans more than one warp
+#ifndef CONVROT_RQ_MAX_IDLE_PCT
+#define CONVROT_RQ_MAX_IDLE_PCT 2  // pack long rows until at most this share of threads is idle
 #endif
 constexpr int kMaxStages = 3;
+constexpr int kMaxLongRows = 8;  // rows per group when rows span several warps
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     const uint32_t a = smem_u32(p);
@@ -75,7 +79,8 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
                                                             unsigned int* err) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full[kMaxStages];
-    __shared__ float red[2][32];  // warp maxima, double-buffered across iterations
+    // Row maxima of long rows: (iteration << 32) | bits of the max, double-buffered.
+    __shared__ unsigned long long rowmax[2][kMaxLongRows];
     __shared__ int abort_flag;
     uint8_t* ring = align1024(smem_raw);
 
@@ -84,6 +89,17 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
     const int warp = tid >> 5;
     const int rloc = tid / tpr_pad;
     const int t = tid - rloc * tpr_pad;
+    const bool active = rloc < rows_per_cta && t < tpr;  // long rows: threads past the last row idle
+    // Long rows: the row this lane reduces into (idle lanes join the last
+    // row) and the first lane of the warp's second row segment (32: none).
+    const bool long_rows = tpr_pad > 32;
+    const int rr = rloc < rows_per_cta ? rloc : rows_per_cta - 1;
+    int split = 32;
+    if (long_rows) {
+        const int r0 = min((warp * 32) / tpr, rows_per_cta - 1);
+        if (r0 < rows_per_cta - 1) split = min((r0 + 1) * tpr - warp * 32, 32);
+    }
+    const uint32_t lo_mask = split >= 32 ? 0xFFFFFFFFu : ((1u << split) - 1u);
     const uint32_t slot_bytes = static_cast<uint32_t>(nbox) * box1 * 128u * rows_per_cta;
     const int row_pitch = nbox * box1;  // 128-byte shared rows between consecutive input rows of a group
     (void)rows128;
@@ -98,6 +114,7 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
                              static_cast<int>(g * rows_per_cta), policy);
     };
 
+    if (tid < 2 * kMaxLongRows) rowmax[tid / kMaxLongRows][tid % kMaxLongRows] = 0ull;
     if (tid == 0) {
         abort_flag = 0;
         for (int i = 0; i < nstage; ++i) mbar_init(&full[i], 1);
@@ -118,7 +135,7 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
         if (!mbar_wait_bounded(&full[slot], parity, limit_ns, kErrTimeoutLoad, err)) abort_flag = 1;
 
         uint64_t P[kPairs];
-        if (t < tpr) {
+        if (active) {
             load_pairs<Tin>(ring + static_cast<size_t>(slot) * slot_bytes, rloc * row_pitch, t, P);
         } else {
 #pragma unroll
@@ -127,17 +144,20 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
 
         if constexpr (BLOCK == 128) fwht128(P, t);
         float amax = piece_absmax(P);
-        float* rbuf = red[it & 1];
-        if (tpr_pad <= 32) {
+        if (!long_rows) {
             for (int o = tpr_pad >> 1; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         } else {
-            // rows span whole warps: warp maxima through shared memory
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-            if (lane == 0) rbuf[warp] = amax;
+            // amax is a non-negative, non-NaN float (fmaxf from +0 drops NaNs),
+            // so its bits order like the values.
+            const uint32_t bits = __float_as_uint(amax);
+            uint32_t m;
+            if (lane < split) m = __reduce_max_sync(lo_mask, bits);
+            else m = __reduce_max_sync(~lo_mask, bits);
+            if (lane == 0 || lane == split)
+                atomicMax(&rowmax[it & 1][rr], (static_cast<unsigned long long>(it) << 32) | m);
         }
         // The one CTA barrier per group: every thread has read the slot (so it
-        // can be refilled) and has published its warp maximum.
+        // can be refilled) and has published its share of the row maximum.
         __syncthreads();
         if (abort_flag) break;  // uniform across the CTA
         if (tid == 0) {
@@ -147,16 +167,14 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
                 issue(gn, slot);
             }
         }
-        if (tpr_pad > 32) {
-            const int nw = tpr_pad >> 5;  // warps per row
-            amax = rbuf[rloc * nw];
-            for (int i = 1; i < nw; ++i) amax = fmaxf(amax, rbuf[rloc * nw + i]);
-        }
+        // Every row's first segment wrote with this iteration's tag, which
+        // beats whatever an earlier group left in this buffer.
+        if (long_rows) amax = __uint_as_float(static_cast<uint32_t>(rowmax[it & 1][rr]));
 
         const int64_t row = g * rows_per_cta + rloc;
-        if (row < M && t < tpr) {
+        if (row < M && active) {
             const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-            quantize_store(P, inv, q + row * ldq + static_cast<int64_t>(t) * kPerThread);
+            quantize_store<true>(P, inv, q + row * ldq + static_cast<int64_t>(t) * kPerThread);
             if (t == 0) s[row] = __fdiv_rn(amax, 127.0f);
         }
     }
@@ -201,19 +219,39 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
         g->rows_per_cta = 256 / g->tpr_pad;
         g->nbox = 1;
         g->box1 = g->rows128;  // <= 32; the slot size is a multiple of 1024 bytes
+        g->threads = g->tpr_pad * g->rows_per_cta;
     } else {
-        // Long rows: whole warps per row; boxes padded to 8 rows of 128 bytes
-        // so every box and slot starts on a 1024-byte boundary.
-        g->tpr_pad = (g->tpr + 31) / 32 * 32;
+        // Long rows: packed back to back, tpr threads each (tpr is even, so
+        // the lane pairs of the last butterfly stage never straddle rows);
+        // boxes padded to 8 rows of 128 bytes so every box and slot starts on
+        // a 1024-byte boundary.
+        g->tpr_pad = g->tpr;
         g->nbox = (g->rows128 + 255) / 256;
         const int per = (g->rows128 + g->nbox - 1) / g->nbox;
         g->box1 = (per + 7) / 8 * 8;
         if (g->box1 > 256) return false;
-        // Several rows per group share the CTA's barriers (at most 1024 threads).
-        g->rows_per_cta = g->nbox == 1 ? CONVROT_RQ_LONG_ROWS : 1;
-        while (g->rows_per_cta > 1 && g->tpr_pad * g->rows_per_cta > kMaxThreads) --g->rows_per_cta;
+        // Rows per group: one when a row needs several boxes (the slot holds
+        // one row's boxes back to back), else the fewest rows that leave at
+        // most CONVROT_RQ_MAX_IDLE_PCT of the CTA's threads idle (or, failing
+        // that, the fewest idle threads).
+        auto round32 = [](int v) { return (v + 31) / 32 * 32; };
+        g->rows_per_cta = 1;
+        if (g->nbox == 1) {
+            int best = 1;
+            for (int r = 1; r <= kMaxLongRows && round32(r * g->tpr) <= kMaxThreads; ++r) {
+                const int thr = round32(r * g->tpr);
+                const int idle = thr - r * g->tpr;
+                if (idle * 100 <= CONVROT_RQ_MAX_IDLE_PCT * thr) {
+                    best = r;
+                    break;
+                }
+                const int bthr = round32(best * g->tpr);
+                if (idle * bthr < (bthr - best * g->tpr) * thr) best = r;
+            }
+            g->rows_per_cta = best;
+        }
+        g->threads = round32(g->rows_per_cta * g->tpr);
     }
-    g->threads = g->tpr_pad * g->rows_per_cta;
     const size_t slot = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
     if (slot % 1024 != 0) return false;  // slots must stay 1024-byte aligned for the swizzle
     const size_t budget = 200 * 1024;
