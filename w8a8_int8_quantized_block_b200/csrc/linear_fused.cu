@@ -166,16 +166,16 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                 for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
             }
             if (f.block == 128) qcore::fwht128(P, t);
-            float amax = qcore::piece_absmax(P);
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            // amax is a non-negative, non-NaN float (fmaxf from +0 drops NaNs),
+            // so its bits order like the values.
+            float amax = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(qcore::piece_absmax(P))));
             if (lane == 0) gred[(it & 1) * kQWarps + qw] = amax;
             named_bar_sync(1 + qg, kQThreads);  // warp maxima published
             amax = gred[(it & 1) * kQWarps];
             for (int i = 1; i < kQWarps; ++i) amax = fmaxf(amax, gred[(it & 1) * kQWarps + i]);
             if (holds) {
                 const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-                qcore::quantize_store<false>(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
+                qcore::quantize_store<true>(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
                 if (t == 0) f.s[row] = __fdiv_rn(amax, 127.0f);
             }
             __threadfence();                    // this thread's codes are visible device-wide
