@@ -22,6 +22,20 @@
  *              in fp32, stages h = 1, 2, 4, ..., b/2 in that order, each
  *              butterfly (u, v) -> (u + v, u - v) rounded to nearest-even.
  *              The pages fix no order; this one is the reading both sides use.
+ *  regular     the "DC-balanced regular orthogonal Hadamard matrix
+ *              H_256 = H_4^(x)4" of "MiniMax-H3-Rung-Omega" README, section
+ *              "Technical Architecture Overview", item 1 (there for another
+ *              weight format; here an alternative rotation of orders 16, 64,
+ *              256).  H_4 is read as J - 2I: every row sums to +2, so the
+ *              Kronecker power of order b = 4^k has every row sum sqrt(b) and
+ *              maps a constant block to a constant block.  Entry (i, j) is the
+ *              product over the k base-4 digits of -1 where the digits agree
+ *              and +1 where they differ.  Computed in fp32 as k radix-4
+ *              stages, digit strides 1, 4, 16, 64 in that order; each group
+ *              (x0, x1, x2, x3) of a stage becomes t - 2 x_i with
+ *              t = (x0 + x1) + (x2 + x3), every operation rounded to
+ *              nearest-even (2 x_i is exact, so each output rounds once more).
+ *              Again the order is this reading's, shared by both sides.
  *  act quant   rowwise symmetric int8 ("SwiGLU + ConvRot64 + Rowwise INT8
  *              Quantize" -- MiniMax-H3-Rung-Omega README, "Technical
  *              Architecture Overview", item 2, Floor 1):
@@ -39,11 +53,14 @@
  *              alpha = 1/b for a rotated pair (b = 0 or 1: alpha = 1);
  *              optional exact-erf GELU.
  *
- * Pins (tests/test_oracle_pins.py): H*H^T = b*I in exact integers; the FWHT
- * equals the explicit matrix product on integer inputs and is an involution up
- * to b; constant and spike blocks give closed-form codes; rounding ties match
- * an exact rational arbiter; sign and power-of-two scale invariances; the
- * int64 GEMM equals a pure-Python brute force.
+ * Pins (tests/test_oracle_pins.py): H*H^T = b*I in exact integers for both
+ * kinds; the Sylvester entries equal the doubling recursion and the regular
+ * ones numpy's Kronecker powers of J - 2I, with every row sum sqrt(b); both
+ * transforms equal the explicit matrix product on integer inputs and are
+ * involutions up to b; constant and spike blocks give closed-form codes;
+ * rounding ties match an exact rational arbiter; the product is rounded to
+ * f32 before the integer; sign and power-of-two scale invariances; the int64
+ * GEMM equals a pure-Python brute force.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fPIC -shared (no fast-math).
  */
@@ -88,6 +105,42 @@ void oracle_fwht_f32(float *v, int64_t n, int b) {
     for (int64_t o = 0; o < n; o += b) fwht_block_f32(v + o, b);
 }
 
+/* Regular H_4^(x)k, b = 4^k: entry from its definition, digit by digit. */
+int oracle_regular_entry(int64_t i, int64_t j, int b) {
+    int sign = 1;
+    for (int st = 1; st < b; st *= 4) {
+        if ((i / st) % 4 == (j / st) % 4) sign = -sign; /* H_4 = J - 2I: -1 on the diagonal */
+    }
+    return sign;
+}
+
+/* In-place regular transform of one block of b = 4^k floats: stages with
+ * digit strides 1, 4, ..., b/4; each group (x0, x1, x2, x3) -> t - 2 x_i,
+ * t = (x0 + x1) + (x2 + x3). */
+static void rfwht_block_f32(float *v, int b) {
+    for (int st = 1; st < b; st *= 4) {
+        for (int i = 0; i < b; i += 4 * st) {
+            for (int j = i; j < i + st; ++j) {
+                float x0 = v[j], x1 = v[j + st], x2 = v[j + 2 * st], x3 = v[j + 3 * st];
+                float t = (x0 + x1) + (x2 + x3);
+                v[j] = t - 2.0f * x0;
+                v[j + st] = t - 2.0f * x1;
+                v[j + 2 * st] = t - 2.0f * x2;
+                v[j + 3 * st] = t - 2.0f * x3;
+            }
+        }
+    }
+}
+
+/* The rotation of a vector of n floats: Sylvester blocks, or regular ones. */
+void oracle_rotate_f32(float *v, int64_t n, int b, int regular) {
+    if (b <= 1) return;
+    for (int64_t o = 0; o < n; o += b) {
+        if (regular) rfwht_block_f32(v + o, b);
+        else fwht_block_f32(v + o, b);
+    }
+}
+
 /* Rowwise symmetric quantisation of one row of K rotated values. */
 static void quantize_row(const float *z, int64_t K, int8_t *q, float *s) {
     float amax = 0.0f;
@@ -127,14 +180,14 @@ static float bf16_bits_to_f32(uint16_t h) {
 
 /* Activations: bf16 rows (raw bits) -> rotate per block of b -> int8 + scale. */
 void oracle_quantize_act_bf16(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
-                              int b, int8_t *q, int64_t ldq, float *s) {
+                              int b, int regular, int8_t *q, int64_t ldq, float *s) {
 #pragma omp parallel
     {
         float *row = (float *)malloc((size_t)K * sizeof(float));
 #pragma omp for schedule(static)
         for (int64_t m = 0; m < M; ++m) {
             for (int64_t k = 0; k < K; ++k) row[k] = bf16_bits_to_f32(x[m * ldx + k]);
-            oracle_fwht_f32(row, K, b);
+            oracle_rotate_f32(row, K, b, regular);
             quantize_row(row, K, q + m * ldq, s + m);
         }
         free(row);
@@ -142,7 +195,7 @@ void oracle_quantize_act_bf16(const uint16_t *x, int64_t M, int64_t K, int64_t l
 }
 
 /* Weights: f32 [N, K] rows -> same rotation along K -> int8 + per-row scale. */
-void oracle_pack_weight_f32(const float *w, int64_t N, int64_t K, int b,
+void oracle_pack_weight_f32(const float *w, int64_t N, int64_t K, int b, int regular,
                             int8_t *q, float *s) {
 #pragma omp parallel
     {
@@ -150,7 +203,7 @@ void oracle_pack_weight_f32(const float *w, int64_t N, int64_t K, int b,
 #pragma omp for schedule(static)
         for (int64_t n = 0; n < N; ++n) {
             memcpy(row, w + n * K, (size_t)K * sizeof(float));
-            oracle_fwht_f32(row, K, b);
+            oracle_rotate_f32(row, K, b, regular);
             quantize_row(row, K, q + n * K, s + n);
         }
         free(row);
@@ -216,12 +269,12 @@ void oracle_dequant_pairs_f64(const int64_t *acc, const int64_t *mi, const int64
 }
 
 /*
- * Exact-arithmetic companion of the rotation: z = blockdiag(H_b) x by the
- * explicit matrix, accumulated in fp64 (exact for bf16 inputs whose block
- * spans fewer than ~45 binades).  Used only to measure how far a quantiser
- * input sits from a rounding boundary.
+ * Exact-arithmetic companion of the rotation: z = blockdiag(H_b) x (Sylvester
+ * or regular H_b) by the explicit matrix, accumulated in fp64 (exact for bf16
+ * inputs whose block spans fewer than ~45 binades).  Used only to measure how
+ * far a quantiser input sits from a rounding boundary.
  */
-void oracle_rotate_explicit_f64(const float *x, int64_t M, int64_t K, int b, double *z) {
+void oracle_rotate_explicit_f64(const float *x, int64_t M, int64_t K, int b, int regular, double *z) {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
         const float *xr = x + m * K;
@@ -233,7 +286,10 @@ void oracle_rotate_explicit_f64(const float *x, int64_t M, int64_t K, int b, dou
         for (int64_t o = 0; o < K; o += b) {
             for (int i = 0; i < b; ++i) {
                 double acc = 0.0;
-                for (int j = 0; j < b; ++j) acc += (double)oracle_hadamard_entry(i, j) * (double)xr[o + j];
+                for (int j = 0; j < b; ++j) {
+                    int e = regular ? oracle_regular_entry(i, j, b) : oracle_hadamard_entry(i, j);
+                    acc += (double)e * (double)xr[o + j];
+                }
                 zr[o + i] = acc;
             }
         }

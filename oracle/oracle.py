@@ -14,12 +14,17 @@ Every function cites the passage it follows (page title and section):
 * per-output-channel F32 weight scales, [output, input] storage -- "MiniMax H3 -
   pruned INT8 ConvRot - input-major", section "Input-major checkpoint";
 * exact undo of the rotation -- "HyperFlow H3 Flash MLX", section "How to run";
-* W8A8 INT8 -- HyperFlow H3 Flash card, "Choose a Weight Format".
+* W8A8 INT8 -- HyperFlow H3 Flash card, "Choose a Weight Format";
+* the regular rotation H_4^(x)k ("DC-balanced regular orthogonal Hadamard
+  matrix H_256 = H_4^(x)4") -- MiniMax-H3-Rung-Omega README, "Technical
+  Architecture Overview", item 1.
 
 Readings where the pages are silent (all listed in the design doc): Sylvester
 order H[i][j] = (-1)^popcount(i & j); unnormalised transform with the 1/b
 folded into the dequantisation; fp32 butterflies in ascending stage order;
-s = amax/127 and q = rne(z * (127/amax)) in f32; a zero row has s = 0.
+s = amax/127 and q = rne(z * (127/amax)) in f32; a zero row has s = 0;
+regular H_4 = J - 2I, its fp32 stages in ascending digit stride, each group
+t = (x0 + x1) + (x2 + x3), x_i -> t - 2 x_i.
 """
 from __future__ import annotations
 
@@ -38,7 +43,7 @@ _LIB_PATH = os.environ.get("CONVROT_ORACLE_LIB") or os.path.join(_HERE, "liborac
 CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 __all__ = [
-    "build", "lib", "num_threads", "hadamard", "hadamard_sylvester", "fwht",
+    "build", "lib", "num_threads", "hadamard", "hadamard_sylvester", "hadamard_regular_kron", "fwht",
     "quantize_rows", "quantize_act", "pack_weight", "igemm", "igemm_pairs",
     "dequant", "dequant_pairs", "linear", "rotate_explicit_f64",
     "bf16_bits", "bf16_bits_to_f32", "py_fwht_exact", "py_quantize_row_exact",
@@ -69,15 +74,18 @@ def lib() -> ctypes.CDLL:
         L.oracle_hadamard_entry.argtypes = [I64, I64]
         L.oracle_hadamard_entry.restype = I32
         L.oracle_num_threads.restype = I32
+        L.oracle_regular_entry.argtypes = [I64, I64, I32]
+        L.oracle_regular_entry.restype = I32
         L.oracle_fwht_f32.argtypes = [P, I64, I32]
+        L.oracle_rotate_f32.argtypes = [P, I64, I32, I32]
         L.oracle_quantize_rows_f32.argtypes = [P, I64, I64, I64, P, I64, P]
-        L.oracle_quantize_act_bf16.argtypes = [P, I64, I64, I64, I32, P, I64, P]
-        L.oracle_pack_weight_f32.argtypes = [P, I64, I64, I32, P, P]
+        L.oracle_quantize_act_bf16.argtypes = [P, I64, I64, I64, I32, I32, P, I64, P]
+        L.oracle_pack_weight_f32.argtypes = [P, I64, I64, I32, I32, P, P]
         L.oracle_igemm_s64.argtypes = [P, I64, P, I64, I64, I64, I64, P, I64]
         L.oracle_igemm_s64_pairs.argtypes = [P, I64, P, I64, I64, P, P, I64, P]
         L.oracle_dequant_f64.argtypes = [P, I64, I64, P, P, P, ctypes.c_double, I32, P]
         L.oracle_dequant_pairs_f64.argtypes = [P, P, P, I64, P, P, P, ctypes.c_double, I32, P]
-        L.oracle_rotate_explicit_f64.argtypes = [P, I64, I64, I32, P]
+        L.oracle_rotate_explicit_f64.argtypes = [P, I64, I64, I32, I32, P]
         _lib = L
     return _lib
 
@@ -94,9 +102,12 @@ def num_threads() -> int:
 # ---------------------------------------------------------------- Hadamard
 
 
-def hadamard(b: int) -> np.ndarray:
-    """H_b from its entry definition (-1)^popcount(i & j), via the C oracle."""
+def hadamard(b: int, regular: bool = False) -> np.ndarray:
+    """H_b from its entry definition, via the C oracle: Sylvester
+    (-1)^popcount(i & j), or the regular H_4^(x)k digit by digit."""
     L = lib()
+    if regular:
+        return np.array([[L.oracle_regular_entry(i, j, b) for j in range(b)] for i in range(b)], dtype=np.int64)
     return np.array([[L.oracle_hadamard_entry(i, j) for j in range(b)] for i in range(b)], dtype=np.int64)
 
 
@@ -110,19 +121,34 @@ def hadamard_sylvester(b: int) -> list[list[int]]:
     return H
 
 
-def fwht(x: np.ndarray, b: int) -> np.ndarray:
-    """Block-diagonal FWHT of the last axis of a float32 array (canonical order)."""
+def hadamard_regular_kron(b: int) -> np.ndarray:
+    """Independent construction of the regular matrix: Kronecker powers of
+    H_4 = J - 2I (numpy), b = 4^k."""
+    H4 = np.ones((4, 4), dtype=np.int64) - 2 * np.eye(4, dtype=np.int64)
+    H = np.ones((1, 1), dtype=np.int64)
+    while H.shape[0] < b:
+        H = np.kron(H, H4)
+    if H.shape[0] != b:
+        raise ValueError("b must be a power of four")
+    return H
+
+
+def fwht(x: np.ndarray, b: int, regular: bool = False) -> np.ndarray:
+    """Block-diagonal rotation of the last axis of a float32 array (canonical order)."""
     v = np.ascontiguousarray(x, dtype=np.float32).copy()
-    lib().oracle_fwht_f32(_p(v), v.size, b)
+    if regular:
+        lib().oracle_rotate_f32(_p(v), v.size, b, 1)
+    else:
+        lib().oracle_fwht_f32(_p(v), v.size, b)
     return v
 
 
-def rotate_explicit_f64(x: np.ndarray, b: int) -> np.ndarray:
+def rotate_explicit_f64(x: np.ndarray, b: int, regular: bool = False) -> np.ndarray:
     """z = blockdiag(H_b) x by the explicit matrix, fp64 accumulation."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     M, K = x.shape
     z = np.empty((M, K), dtype=np.float64)
-    lib().oracle_rotate_explicit_f64(_p(x), M, K, b, _p(z))
+    lib().oracle_rotate_explicit_f64(_p(x), M, K, b, int(regular), _p(z))
     return z
 
 
@@ -152,23 +178,23 @@ def quantize_rows(z: np.ndarray):
     return q, s
 
 
-def quantize_act(x_bits: np.ndarray, b: int):
+def quantize_act(x_bits: np.ndarray, b: int, regular: bool = False):
     """bf16 activations (uint16 bits [M, K]) -> rotate (block b) -> (q, s_x)."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     M, K = x_bits.shape
     q = np.empty((M, K), dtype=np.int8)
     s = np.empty((M,), dtype=np.float32)
-    lib().oracle_quantize_act_bf16(_p(x_bits), M, K, K, b, _p(q), K, _p(s))
+    lib().oracle_quantize_act_bf16(_p(x_bits), M, K, K, b, int(regular), _p(q), K, _p(s))
     return q, s
 
 
-def pack_weight(w: np.ndarray, b: int):
+def pack_weight(w: np.ndarray, b: int, regular: bool = False):
     """f32 weights [N, K] -> rotate along K -> per-output-channel (q_w, s_w)."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     N, K = w.shape
     q = np.empty((N, K), dtype=np.int8)
     s = np.empty((N,), dtype=np.float32)
-    lib().oracle_pack_weight_f32(_p(w), N, K, b, _p(q), _p(s))
+    lib().oracle_pack_weight_f32(_p(w), N, K, b, int(regular), _p(q), _p(s))
     return q, s
 
 
@@ -229,10 +255,12 @@ def dequant_pairs(acc, mi, ni, s_a, s_b, bias, b: int, gelu: bool = False) -> np
     return y
 
 
-def linear(x_bits: np.ndarray, w: np.ndarray, bias: np.ndarray | None, b: int, gelu: bool = False):
-    """Whole path on the CPU: returns (y fp64, q_x, s_x, q_w, s_w, acc)."""
-    qx, sx = quantize_act(x_bits, b)
-    qw, sw = pack_weight(w, b)
+def linear(x_bits: np.ndarray, w: np.ndarray, bias: np.ndarray | None, b: int, gelu: bool = False,
+           regular: bool = False):
+    """Whole path on the CPU: returns (y fp64, q_x, s_x, q_w, s_w, acc).  Both
+    H_b H_b^T = b I kinds share alpha = 1/b."""
+    qx, sx = quantize_act(x_bits, b, regular)
+    qw, sw = pack_weight(w, b, regular)
     acc = igemm(qx, qw)
     y = dequant(acc, sx, sw, bias, b, gelu)
     return y, qx, sx, qw, sw, acc
@@ -241,9 +269,12 @@ def linear(x_bits: np.ndarray, w: np.ndarray, bias: np.ndarray | None, b: int, g
 # ---------------------------------------------------------------- pure-Python references (tiny inputs)
 
 
-def py_fwht_exact(x: list, b: int) -> list:
+def py_fwht_exact(x: list, b: int, regular: bool = False) -> list:
     """Explicit H_b x per block with exact rational arithmetic (no rounding)."""
-    H = hadamard_sylvester(b) if b > 1 else [[1]]
+    if regular:
+        H = hadamard_regular_kron(b).tolist()
+    else:
+        H = hadamard_sylvester(b) if b > 1 else [[1]]
     bb = max(b, 1)
     out = []
     for o in range(0, len(x), bb):

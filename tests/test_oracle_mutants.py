@@ -30,6 +30,10 @@ MUTANTS = {
     "dequant_drops_bias": ("            if (bias) v += (double)bias[n];\n            if (gelu) v = gelu_f64(v);\n            y[m * N + n] = v;",
                            "            if (gelu) v = gelu_f64(v);\n            y[m * N + n] = v;"),
     "gelu_half_missing": ("return 0.5 * y * (1.0 + erf(y / sqrt(2.0)));", "return y * (1.0 + erf(y / sqrt(2.0)));"),
+    "regular_output_drops_factor_2": ("v[j] = t - 2.0f * x0;", "v[j] = t - x0;"),
+    "regular_missing_last_stage": ("for (int st = 1; st < b; st *= 4) {\n        for (int i = 0; i < b; i += 4 * st) {",
+                                   "for (int st = 1; st < b / 4; st *= 4) {\n        for (int i = 0; i < b; i += 4 * st) {"),
+    "regular_h4_sign": ("if ((i / st) % 4 == (j / st) % 4) sign = -sign;", "if ((i / st) % 4 != (j / st) % 4) sign = -sign;"),
     "amax_skips_first": ("for (int64_t k = 0; k < K; ++k) {\n        float a = fabsf(z[k]);", "for (int64_t k = 1; k < K; ++k) {\n        float a = fabsf(z[k]);"),
 }
 

@@ -41,6 +41,25 @@ def test_hadamard_definition_matches_sylvester_and_is_orthogonal(b):
     assert (H @ H.T == b * np.eye(b, dtype=np.int64)).all()
 
 
+@pytest.mark.parametrize("b", [4, 16, 64, 256])
+def test_regular_hadamard_definition_matches_kronecker_power_and_is_regular(b):
+    # The pages' regular matrix: H_256 = H_4 (x) H_4 (x) H_4 (x) H_4, orthogonal
+    # and "DC-balanced": every row has the same sum, so a constant block stays
+    # constant.  Read with H_4 = J - 2I (row sum +2).
+    H = O.hadamard(b, regular=True)
+    K = O.hadamard_regular_kron(b)
+    assert (H == K).all()
+    assert (H == H.T).all()
+    assert (H @ H.T == b * np.eye(b, dtype=np.int64)).all()
+    r = int(round(b ** 0.5))
+    assert (H.sum(axis=1) == r).all() and (H.sum(axis=0) == r).all()
+    # a regular Hadamard matrix is not a Sylvester one: H_b 1 is constant,
+    # while Sylvester sends 1 to (b, 0, ..., 0)
+    S = np.array(O.hadamard_sylvester(b), dtype=np.int64)
+    assert (S @ np.ones(b, dtype=np.int64) == np.eye(b, dtype=np.int64)[0] * b).all()
+    assert (H @ np.ones(b, dtype=np.int64) == r).all()
+
+
 # ------------------------------------------------------------ rotation
 
 
@@ -301,3 +320,85 @@ def test_quantiser_rounds_the_f32_product_before_the_integer(block):
     if block == 0:
         # the a/2 entries are exactly the near-tie elements
         assert ((np.abs(q) == 64) == (half & (np.abs(x) < x.max(axis=1, keepdims=True)))).all()
+
+
+
+# ------------------------------------------------------------ regular rotation H_4^(x)k
+
+
+@pytest.mark.parametrize("b", [16, 64, 256])
+def test_regular_rotation_equals_explicit_matrix_on_integers(b):
+    rng = np.random.default_rng(b + 1)
+    x = rng.integers(-1000, 1000, size=3 * b).astype(np.float32)  # every fp32 op exact
+    z = O.fwht(x, b, regular=True)
+    exact = O.py_fwht_exact([int(v) for v in x], b, regular=True)
+    assert [Fraction(float(v)) for v in z] == exact
+
+
+@pytest.mark.parametrize("b", [16, 64, 256])
+def test_regular_rotation_is_involution_up_to_b(b):
+    rng = np.random.default_rng(b + 2)
+    x = rng.integers(-500, 500, size=2 * b).astype(np.float32)
+    assert (O.fwht(O.fwht(x, b, regular=True), b, regular=True) == b * x).all()
+
+
+@pytest.mark.parametrize("b", [16, 64, 256])
+def test_regular_rotation_f32_within_error_bound(b):
+    # k = log4(b) radix-4 stages; each output of a stage is t - 2x with
+    # t = (x0 + x1) + (x2 + x3): three roundings per stage, each bounded by
+    # 2^-24 times the sum of the magnitudes feeding it, so the error stays
+    # within 3k * 2^-24 * sum|x| of the block (first order).
+    # f32 inputs (the weight path), so that the sums do round.
+    k = {16: 2, 64: 3, 256: 4}[b]
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 2 * b)).astype(np.float32)
+    x[:, 3] *= 30
+    z = np.stack([O.fwht(r, b, regular=True) for r in x])
+    exact = O.rotate_explicit_f64(x, b, regular=True)
+    absx = np.abs(x).reshape(6, 2, b).sum(-1)
+    bound = 3 * k * 2.0 ** -24 * np.repeat(absx, b, axis=1) * 1.0001
+    assert (np.abs(z - exact) <= bound).all()
+    assert np.abs(z - exact).max() > 0
+
+
+@pytest.mark.parametrize("b", [16, 64, 256])
+def test_regular_rotation_of_constant_block_stays_constant(b):
+    # DC-balanced: x = c 1 gives z = sqrt(b) c 1, so every code is 127
+    c = 0.75
+    x = np.full((1, 2 * b), c, dtype=np.float32)
+    q, s = O.quantize_act(_bf16(x), b, regular=True)
+    assert (q[0] == 127).all()
+    assert s[0] == np.float32(b ** 0.5 * c) / np.float32(127)
+    qw, sw = O.pack_weight(x, b, regular=True)
+    assert (qw[0] == 127).all() and sw[0] == s[0]
+
+
+@pytest.mark.parametrize("b,i", [(16, 0), (16, 11), (64, 37), (256, 200)])
+def test_regular_rotation_of_spike_gives_column_signs(b, i):
+    c = -3.0
+    x = np.zeros((1, b), dtype=np.float32)
+    x[0, i] = c
+    q, s = O.quantize_act(_bf16(x), b, regular=True)
+    H = O.hadamard_regular_kron(b)
+    assert (q[0] == (-127 * H[:, i])).all()
+    assert s[0] == np.float32(3.0) / np.float32(127)
+
+
+@pytest.mark.parametrize("b,regular", [(64, False), (256, False), (16, True), (64, True), (256, True)])
+def test_linear_with_other_blocks_matches_unquantised_product(b, regular):
+    # H_b H_b^T = b I for both kinds, so the rotated codes dequantised with
+    # alpha = 1/b approximate x W^T + bias; quantisation error bounds the gap
+    rng = np.random.default_rng(b + regular)
+    M, K, N = 24, 512, 40
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, 9] *= 25
+    xb = _bf16(x)
+    w = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    bias = (rng.standard_normal(N) * 0.01).astype(np.float32)
+    y, *_ = O.linear(xb, w, bias, b, regular=regular)
+    ref = O.bf16_bits_to_f32(xb).astype(np.float64) @ w.T.astype(np.float64) + bias
+    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert rel < 0.02
+    # rotating spreads the outlier channel: the error is well below no rotation
+    y0, *_ = O.linear(xb, w, bias, 0)
+    assert rel < np.linalg.norm(y0 - ref) / np.linalg.norm(ref)
