@@ -37,6 +37,27 @@ INT8_PER_BF16 = 2.0  # nominal dense ratio of 8-bit to bf16 tensor throughput (4
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 
+REGULAR = 0x10000  # the C ABI's CONVROT_HADAMARD_REGULAR flag on a block value
+BLOCK_CHOICES = {"64": 64, "128": 128, "256": 256,
+                 "reg16": REGULAR | 16, "reg64": REGULAR | 64, "reg256": REGULAR | 256}
+
+
+def workload(args):
+    """The 768p projection with the chosen rotation (the inputs do not change)."""
+    import dataclasses
+    from w8a8_int8_quantized_block_b200 import workloads as W
+    spec = W.PROJ_768P
+    if args.block == "128":
+        return spec
+    return dataclasses.replace(spec, block=BLOCK_CHOICES[args.block], name=f"{spec.name}_block{args.block}")
+
+
+def oracle_block(block: int):
+    """(b, regular) of a block value, as the oracle takes them."""
+    n = block & ~REGULAR
+    return (n if n > 1 else 1), bool(block & REGULAR)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -47,6 +68,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-seconds", type=float, default=60.0,
                     help="CPU time budget of the whole --impl reference run (warm-up + timed steps)")
+    ap.add_argument("--block", choices=sorted(BLOCK_CHOICES), default="128",
+                    help="rotation of the step: Sylvester H_b (64, 128, 256) or the regular H_4^(x)k "
+                         "(reg16, reg64, reg256); the headline is 128")
     ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm"], default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
                          "(for profiler captures; prints no result line)")
@@ -177,11 +201,18 @@ def oracle_sample(x_bits, qw, sw, bias, rows: int, block: int):
     """The oracle's whole path (quantise, int64 GEMM, fp64 dequant) on `rows`
     token rows; returns seconds."""
     from oracle import oracle as O
+    b, reg = oracle_block(block)
     t0 = time.perf_counter()
-    qx, sx = O.quantize_act(x_bits[:rows], block)
+    qx, sx = O.quantize_act(x_bits[:rows], b, reg)
     acc = O.igemm(qx, qw)
-    O.dequant(acc, sx, sw, bias, block)
+    O.dequant(acc, sx, sw, bias, b)
     return time.perf_counter() - t0
+
+
+def oracle_pack(w, block: int):
+    from oracle import oracle as O
+    b, reg = oracle_block(block)
+    return O.pack_weight(w, b, reg)
 
 
 def cpu_baseline(spec, target_s: float = 12.0):
@@ -191,7 +222,7 @@ def cpu_baseline(spec, target_s: float = 12.0):
     from w8a8_int8_quantized_block_b200 import workloads as W
     x, w, bias = W.linear_inputs(spec)
     xb = O.bf16_bits(x)
-    qw, sw = O.pack_weight(w.numpy(), spec.block)  # offline on both sides: not timed
+    qw, sw = oracle_pack(w.numpy(), spec.block)  # offline on both sides: not timed
     b = bias.numpy().astype(np.float32)
     rows = 16
     t = oracle_sample(xb, qw, sw, b, rows, spec.block)
@@ -211,10 +242,10 @@ def run_reference(args, rank: int):
     import numpy as np
     if rank != 0:
         return
-    spec = W.PROJ_768P
+    spec = workload(args)
     x, w, bias = W.linear_inputs(spec)
     xb = O.bf16_bits(x)
-    qw, sw = O.pack_weight(w.numpy(), spec.block)
+    qw, sw = oracle_pack(w.numpy(), spec.block)
     b = bias.numpy().astype(np.float32)
     per_step_target = max(0.02, args.reference_seconds / max(1, args.steps + args.warmup))
     t = oracle_sample(xb, qw, sw, b, 8, spec.block)
@@ -265,7 +296,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    spec = W.PROJ_768P
+    spec = workload(args)
     x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
     x = x_cpu.cuda()
     bias = b_cpu.cuda()
@@ -368,7 +399,7 @@ def main():
             "roofline": {"bound": "tensor",
                          "kernel": "linear_fused_kernel (rotate + quantise + int8 GEMM + dequant epilogue, one launch)",
                          "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
-                         "traffic": profiled_traffic(),
+                         "traffic": profiled_traffic() if args.block == "128" else None,
                          "peak_source": f"{kind} bf16 burst {bf16} TFLOP/s x {INT8_PER_BF16} (nominal int8:bf16)",
                          "algorithmic_ops_per_launch": spec.ops},
             "kernels": {

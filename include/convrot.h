@@ -4,7 +4,8 @@
  *
  * The operation (the pages' "int8_convrot" linear):
  *   1. rotate: z = blockdiag(H_b) x for every token, H_b the Sylvester Hadamard
- *      matrix H[i][j] = (-1)^popcount(i & j), b = 128 ("180 linear layers
+ *      matrix H[i][j] = (-1)^popcount(i & j), b = 128 (other blocks and the
+ *      regular H_4^(x)k: see "Block values" below) ("180 linear layers
  *      quantized to INT8 behind a block-diagonal Hadamard rotation" -- lehuy.net,
  *      "Nen mo hinh video khuech tan 31B xuong 14B chi voi 6 buoc", section
  *      "Cach nen hoat dong");
@@ -21,6 +22,24 @@
  *      Flash MLX", section "How to run").
  * The 1/b folds the 1/sqrt(b) of both orthonormal rotations into one exact
  * power-of-two factor.
+ *
+ * Block values (the `block` argument and convrot_wdesc.block):
+ *   0 or 1                      no rotation (b = 1);
+ *   64, 128, 256                Sylvester H_b, fp32 butterflies in stage order
+ *                               h = 1, 2, ..., b/2 (128 is the pages' ConvRot
+ *                               block; 64 is their "ConvRot64", MiniMax-H3-
+ *                               Rung-Omega README, "Technical Architecture
+ *                               Overview", item 2);
+ *   CONVROT_HADAMARD_REGULAR | b, b = 16, 64, 256
+ *                               the regular H_4^(x)k with H_4 = J - 2I, every
+ *                               row summing to sqrt(b) (the "DC-balanced
+ *                               regular orthogonal Hadamard matrix
+ *                               H_256 = H_4^(x)4", same README, item 1); fp32
+ *                               radix-4 stages in digit strides 1, 4, 16, 64,
+ *                               each group (x0..x3) -> t - 2 x_i with
+ *                               t = (x0 + x1) + (x2 + x3).
+ * Both kinds satisfy H_b H_b^T = b I, so the dequantisation divides by b.
+ * Any other value is CONVROT_EUNSUPPORTED; K must be a multiple of b.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, except
@@ -70,10 +89,13 @@ typedef struct convrot_wdesc {
     uint32_t magic;    /* CONVROT_WDESC_MAGIC */
     uint32_t version;  /* CONVROT_WDESC_VERSION */
     uint32_t layout;   /* CONVROT_LAYOUT_OUTPUT_MAJOR */
-    int32_t block;     /* Hadamard block used when packing: 128, or 0 = none */
+    int32_t block;     /* block value used when packing (see above); 0 = none */
     int64_t N;         /* output channels */
     int64_t K;         /* input channels */
 } convrot_wdesc;
+
+/* Flag on a block value selecting the regular H_4^(x)k rotation. */
+#define CONVROT_HADAMARD_REGULAR 0x10000
 
 /* Epilogue selector of the linear entry points. */
 #define CONVROT_EPI_NONE 0  /* y = acc*s_x*s_w/b + bias */
@@ -86,16 +108,16 @@ const char* convrot_status_string(int status);
 int convrot_abi_version(void);
 
 /* Offline weight packing (step 3's weights).
- * w: f32 [N][K] row-major.  block: 128 (rotate) or 0 (no rotation).
+ * w: f32 [N][K] row-major.  block: a block value (see above).
  * Writes q: int8 [N][K] (K contiguous, "output-major") and s_w: f32 [N], and
  * fills *desc (HOST pointer) synchronously.  Requires K % 64 == 0,
- * K % block == 0, K <= 32768, N <= 2^31-1, 16-byte aligned pointers. */
+ * K % b == 0, K <= 32768, N <= 2^31-1, 16-byte aligned pointers. */
 convrot_status convrot_pack_weight(const float* w, int64_t N, int64_t K, int32_t block, int8_t* q,
                                    float* s_w, convrot_wdesc* desc, void* stream);
 
 /* Steps 1-2: x: bf16 [M][K] with row stride ldx (elements) ->
- * q: int8 [M][K] (contiguous) and s_x: f32 [M].  block: 128 or 0.
- * Requires K % 64 == 0, K % block == 0, K <= 32768, ldx >= K, ldx % 8 == 0,
+ * q: int8 [M][K] (contiguous) and s_x: f32 [M].  block: a block value.
+ * Requires K % 64 == 0, K % b == 0, K <= 32768, ldx >= K, ldx % 8 == 0,
  * 0 < M <= 2^31-1.  A row of zeros gives s_x = 0 and zero codes. */
 convrot_status convrot_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int32_t block,
                                     int8_t* q, float* s_x, void* stream);

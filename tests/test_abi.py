@@ -56,11 +56,42 @@ FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: validation fails first
     (4, 512, 500, 128, C.EINVAL),      # ldx < K
     (4, 512, 516, 128, C.EINVAL),      # ldx % 8
     (4, 65536, 65536, 128, C.EINVAL),  # K too large
-    (4, 512, 512, 64, C.EUNSUPPORTED),
+    (4, 512, 512, 32, C.EUNSUPPORTED),                # no 32-point rotation
+    (4, 512, 512, 512, C.EUNSUPPORTED),
+    (4, 512, 512, C.REGULAR | 128, C.EUNSUPPORTED),   # no regular Hadamard of order 128
+    (4, 512, 512, C.REGULAR, C.EUNSUPPORTED),
+    (4, 384, 384, 256, C.EINVAL),                     # K % 256
+    (4, 384, 384, C.REGULAR | 256, C.EINVAL),
 ])
 def test_quantize_act_rejects_bad_arguments(M, K, ldx, block, expect):
     st = C.load().convrot_quantize_act(FAKE, M, K, ldx, block, FAKE, FAKE, None)
     assert st == expect
+
+
+def _skip_if_gpu():
+    # With a GPU these calls would pass validation and launch on fake pointers.
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present")
+    except ImportError:
+        pass
+
+
+@pytest.mark.parametrize("block", C.BLOCKS)
+def test_every_block_value_passes_validation(block):
+    # a valid block gets past the argument checks to the device query, which
+    # fails without a GPU: ECUDA, never EUNSUPPORTED or EINVAL
+    _skip_if_gpu()
+    st = C.load().convrot_quantize_act(FAKE, 4, 512, 512, block, FAKE, FAKE, None)
+    assert st == C.ECUDA
+
+
+def test_regular_flag_matches_the_header():
+    hdr = open(os.path.join(ROOT, "include", "convrot.h")).read()
+    m = re.search(r"#define CONVROT_HADAMARD_REGULAR (0x[0-9a-fA-F]+)", hdr)
+    assert m and int(m.group(1), 16) == C.REGULAR
+    assert [C.block_length(b) for b in C.BLOCKS] == [1, 64, 128, 256, 16, 64, 256]
 
 
 def test_null_pointers_rejected():
@@ -85,8 +116,8 @@ def _desc(**kw):
     return d
 
 
-@pytest.mark.parametrize("field,value", [("magic", 0x12345678), ("version", 2), ("layout", 0), ("block", 64),
-                                         ("N", 0), ("K", 100)])
+@pytest.mark.parametrize("field,value", [("magic", 0x12345678), ("version", 2), ("layout", 0), ("block", 32),
+                                         ("block", C.REGULAR | 128), ("N", 0), ("K", 100), ("K", 320)])
 def test_bad_weight_descriptor_is_a_layout_error(field, value):
     d = _desc(**{field: value})
     st = C.load().convrot_w8a8_linear(FAKE, FAKE, FAKE, FAKE, ctypes.byref(d), None, 0, 16, FAKE, 512, None)
@@ -112,11 +143,6 @@ def test_bmm_and_igemm_shape_rules():
 
 
 def test_valid_call_without_a_gpu_reports_cuda_error():
-    try:
-        import torch
-        if torch.cuda.is_available():
-            pytest.skip("a GPU is present")
-    except ImportError:
-        pass
+    _skip_if_gpu()
     st = C.load().convrot_quantize_act(FAKE, 4, 512, 512, 128, FAKE, FAKE, None)
     assert st == C.ECUDA

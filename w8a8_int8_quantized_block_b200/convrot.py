@@ -21,6 +21,16 @@ EPI_NONE, EPI_GELU = 0, 1
 WDESC_MAGIC = 0x52564E43
 WDESC_VERSION = 1
 LAYOUT_OUTPUT_MAJOR = 1
+# Block values: 0 = no rotation, 64/128/256 = Sylvester H_b, REGULAR | 16/64/256
+# = the regular H_4^(x)k (H_4 = J - 2I).
+REGULAR = 0x10000
+BLOCKS = (0, 64, 128, 256, REGULAR | 16, REGULAR | 64, REGULAR | 256)
+
+
+def block_length(block: int) -> int:
+    """b of a block value (1 for no rotation)."""
+    n = block & ~REGULAR
+    return n if n > 1 else 1
 
 # Every symbol include/convrot.h declares.
 EXPORTS = (

@@ -89,13 +89,37 @@ constexpr int64_t kMaxI32 = 2147483647;
 
 convrot_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CONVROT_OK : CONVROT_ECUDA; }
 
+// The ABI's block value: 0 or 1 = no rotation; 64, 128, 256 = Sylvester H_b;
+// CONVROT_HADAMARD_REGULAR | 16, 64, 256 = the regular H_4^(x)k.  Sets the
+// block length b (1 when there is no rotation) and the kernels' RotKind.
+bool decode_block(int32_t block, int* b, int* kind) {
+    const bool regular = (block & CONVROT_HADAMARD_REGULAR) != 0;
+    const int32_t n = block & ~CONVROT_HADAMARD_REGULAR;
+    int k = -1;
+    if (!regular) {
+        if (n == 0 || n == 1) k = kRotNone;
+        else if (n == 64) k = kRotSyl64;
+        else if (n == 128) k = kRotSyl128;
+        else if (n == 256) k = kRotSyl256;
+    } else {
+        if (n == 16) k = kRotReg16;
+        else if (n == 64) k = kRotReg64;
+        else if (n == 256) k = kRotReg256;
+    }
+    if (k < 0) return false;
+    *b = n > 1 ? n : 1;
+    *kind = k;
+    return true;
+}
+
 // Shared by activations (bf16) and weights (f32).
 convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t K, int64_t ldx, int32_t block,
                             int8_t* q, float* s, cudaStream_t stream) {
     if (!x || !q || !s) return CONVROT_EINVAL;
     if (M <= 0 || M > kMaxI32 || K <= 0) return CONVROT_EINVAL;
-    if (block != 0 && block != 1 && block != 128) return CONVROT_EUNSUPPORTED;
-    if (K % 64 != 0 || K > 32768 || (block > 1 && K % block != 0)) return CONVROT_EINVAL;
+    int b = 1, kind = kRotNone;
+    if (!decode_block(block, &b, &kind)) return CONVROT_EUNSUPPORTED;
+    if (K % 64 != 0 || K > 32768 || K % b != 0) return CONVROT_EINVAL;
     if (ldx < K || (ldx * in_elem_bytes) % 16 != 0) return CONVROT_EINVAL;
     if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u) != 0) return CONVROT_EINVAL;
     const DeviceInfo* d = device_info();
@@ -111,7 +135,7 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
                    static_cast<uint64_t>(ldx) * in_elem_bytes, inner, static_cast<uint32_t>(g.box1),
                    static_cast<uint32_t>(g.rows_per_cta), CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
-    return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, block, M, K, g, q, K, s, g_limit_ns.load(),
+    return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, kind, M, K, g, q, K, s, g_limit_ns.load(),
                                            d->err, d->num_sms, stream));
 }
 
@@ -122,7 +146,8 @@ convrot_status check_desc(const convrot_wdesc* desc) {
         return CONVROT_ELAYOUT;
     if (desc->N <= 0 || desc->N > kMaxI32 || desc->K <= 0 || desc->K % 16 != 0 || desc->K > kMaxI32)
         return CONVROT_ELAYOUT;
-    if (desc->block != 0 && desc->block != 1 && desc->block != 128) return CONVROT_ELAYOUT;
+    int b = 1, kind = kRotNone;
+    if (!decode_block(desc->block, &b, &kind) || desc->K % b != 0) return CONVROT_ELAYOUT;
     return CONVROT_OK;
 }
 
@@ -163,7 +188,18 @@ convrot_status gemm(const int8_t* qa, const int8_t* qb, const float* sa, const f
     return cuda_status(launch_igemm(amap, bmap, ymap, a, epi, d->num_sms, pdl, stream));
 }
 
-float alpha_for_block(int32_t block) { return block > 1 ? 1.0f / static_cast<float>(block) : 1.0f; }
+// H_b H_b^T = b I for both kinds, so a rotated pair of operands carries a
+// factor b that the epilogue removes (1/b is a power of two: exact).
+float alpha_for_block(int32_t block) {
+    int b = 1, kind = kRotNone;
+    if (!decode_block(block, &b, &kind)) return 1.0f;
+    return 1.0f / static_cast<float>(b);
+}
+
+int kind_for_block(int32_t block) {
+    int b = 1, kind = kRotNone;
+    return decode_block(block, &b, &kind) ? kind : kRotNone;
+}
 
 bool tiles_fit_int(int64_t batch, int64_t M, int64_t N) {
     const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + kGemmBN - 1) / kGemmBN) * batch;
@@ -183,10 +219,12 @@ convrot_status linear_checks(const int8_t* qw, const float* s_w, const convrot_w
     return CONVROT_OK;
 }
 
-// The one-kernel linear covers rotated (block 128) or unrotated rows whose
-// length fits one quantiser group.
+// The one-kernel linear covers every rotation kind for rows whose length
+// fits one quantiser group (the descriptor check has already tied the block
+// to K).
 bool fused_eligible(int64_t K, int32_t block) {
-    return (block == 128 || block == 0) && K % 128 == 0 && K >= 128 && K <= kFusedMaxK;
+    int b = 1, kind = kRotNone;
+    return decode_block(block, &b, &kind) && K % 128 == 0 && K >= 128 && K <= kFusedMaxK;
 }
 
 convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
@@ -222,7 +260,7 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
     a.alpha = alpha_for_block(desc->block);
     a.limit_ns = g_limit_ns.load();
     a.err = d->err;
-    return cuda_status(launch_linear_fused(x, ldx, amap, bmap, ymap, a, qx, sx, ready, desc->block > 1 ? 128 : 0,
+    return cuda_status(launch_linear_fused(x, ldx, amap, bmap, ymap, a, qx, sx, ready, kind_for_block(desc->block),
                                            epi, d->num_sms, true, stream));
 }
 

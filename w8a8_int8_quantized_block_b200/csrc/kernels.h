@@ -26,9 +26,21 @@ struct RqGeometry {
 // in_elem_bytes: 2 for bf16 activations, 4 for f32 weights.
 bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g);
 
+// The rotations a row can get: none, Sylvester H_b (b = 64, 128, 256) or the
+// regular H_4^(x)k (b = 16, 64, 256).
+enum RotKind : int {
+    kRotNone = 0,
+    kRotSyl64 = 1,
+    kRotSyl128 = 2,
+    kRotSyl256 = 3,
+    kRotReg16 = 4,
+    kRotReg64 = 5,
+    kRotReg256 = 6,
+};
+
 // x: bf16 (bits) or f32 rows, described by `xmap` (3D: 128-byte inner rows,
-// rows128, M) with 128-byte swizzling.  block: 0/1 (no rotation) or 128.
-cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int block, int64_t M, int64_t K,
+// rows128, M) with 128-byte swizzling.  kind: a RotKind.
+cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
                                 unsigned int* err, int num_sms, cudaStream_t stream);
 
@@ -82,10 +94,10 @@ constexpr int kFusedMaxK = 6144;
 // x: bf16 rows [M][ldx] (16-byte aligned rows); amap/bmap/ymap as for
 // launch_igemm with batch 1, amap over q.  q, s: the codes and scales it
 // writes; ready: ceil(M/256) + 1 zeroed counters (per-panel ready rows, then
-// the panels the GEMM has started).  block: 128 or 0.
+// the panels the GEMM has started).  kind: a RotKind.
 cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMap& amap, const CUtensorMap& bmap,
                                 const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
-                                unsigned int* ready, int block, int epilogue, int num_sms, bool pdl,
+                                unsigned int* ready, int kind, int epilogue, int num_sms, bool pdl,
                                 cudaStream_t stream);
 
 }  // namespace convrot

@@ -73,7 +73,7 @@ struct FusedArgs {
     unsigned int* ready;    // [ceil(M/256)] rows of each panel already quantised (zeroed)
     unsigned int* started;  // panels the GEMM has begun (a running max; zeroed)
     int tpr;                // K / 64: threads of a group holding data
-    int block;              // 128 = rotate, 0 = no rotation
+    int kind;               // the rotation (a RotKind; the kernel is instantiated for it)
 };
 
 __device__ __forceinline__ uint32_t panel_rows(int panel, int M) {
@@ -81,7 +81,7 @@ __device__ __forceinline__ uint32_t panel_rows(int panel, int M) {
     return static_cast<uint32_t>(r < kPanelRows ? r : kPanelRows);
 }
 
-template <int EPI>
+template <int EPI, int KIND>
 __global__ void __launch_bounds__(kThreadsF, 1)
     linear_fused_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                         const __grid_constant__ CUtensorMap ymap, const FusedArgs f) {
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 #pragma unroll
                 for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
             }
-            if (f.block == 128) qcore::fwht128(P, t);
+            qcore::rotate_piece<KIND>(P, t);
             // amax is a non-negative, non-NaN float (fmaxf from +0 drops NaNs),
             // so its bits order like the values.
             float amax = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(qcore::piece_absmax(P))));
@@ -312,10 +312,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-template <int EPI>
+template <int EPI, int KIND>
 cudaError_t launch_fused_epi(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
                              const FusedArgs& f, int num_sms, bool pdl, cudaStream_t stream) {
-    auto kern = linear_fused_kernel<EPI>;
+    auto kern = linear_fused_kernel<EPI, KIND>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalF);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -346,11 +346,26 @@ cudaError_t launch_fused_epi(const CUtensorMap& amap, const CUtensorMap& bmap, c
     return cudaGetLastError();
 }
 
+template <int EPI>
+cudaError_t launch_fused_kind(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
+                              const FusedArgs& f, int num_sms, bool pdl, cudaStream_t stream) {
+    switch (f.kind) {
+        case kRotNone: return launch_fused_epi<EPI, kRotNone>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kRotSyl64: return launch_fused_epi<EPI, kRotSyl64>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kRotSyl128: return launch_fused_epi<EPI, kRotSyl128>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kRotSyl256: return launch_fused_epi<EPI, kRotSyl256>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kRotReg16: return launch_fused_epi<EPI, kRotReg16>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kRotReg64: return launch_fused_epi<EPI, kRotReg64>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        case kRotReg256: return launch_fused_epi<EPI, kRotReg256>(amap, bmap, ymap, f, num_sms, pdl, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMap& amap, const CUtensorMap& bmap,
                                 const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
-                                unsigned int* ready, int block, int epilogue, int num_sms, bool pdl,
+                                unsigned int* ready, int kind, int epilogue, int num_sms, bool pdl,
                                 cudaStream_t stream) {
     FusedArgs f;
     f.g = g;
@@ -361,13 +376,13 @@ cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMa
     f.ready = ready;
     f.started = ready + (g.M + kPanelRows - 1) / kPanelRows;
     f.tpr = g.K / kPerThread;
-    f.block = block;
+    f.kind = kind;
     if (f.tpr > kQThreads || g.K % kPerThread != 0) return cudaErrorInvalidValue;
     switch (epilogue) {
         case kEpiBf16:
-            return launch_fused_epi<kEpiBf16>(amap, bmap, ymap, f, num_sms, pdl, stream);
+            return launch_fused_kind<kEpiBf16>(amap, bmap, ymap, f, num_sms, pdl, stream);
         case kEpiBf16Gelu:
-            return launch_fused_epi<kEpiBf16Gelu>(amap, bmap, ymap, f, num_sms, pdl, stream);
+            return launch_fused_kind<kEpiBf16Gelu>(amap, bmap, ymap, f, num_sms, pdl, stream);
         default:
             return cudaErrorInvalidValue;
     }

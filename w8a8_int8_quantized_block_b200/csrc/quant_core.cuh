@@ -1,27 +1,29 @@
 // quant_core.cuh -- the per-thread pieces of the rotate + quantise pipeline,
 // shared by the standalone quantiser and the fused quantise-ahead linear.
 //
-// A thread owns kPerThread consecutive elements of a row (half a 128-point
-// Hadamard block), held as packed f32x2 register pairs P[j] = (element j,
-// element j + kPairs).  All arithmetic is IEEE single precision with
-// round-to-nearest-even, in the order of the textbook in-place fast
-// Walsh-Hadamard transform (stages h = 1, 2, ..., 64).
+// A thread owns kPerThread = 64 consecutive elements of a row, held as
+// packed f32x2 register pairs P[j] = (element j, element j + 32).  All
+// arithmetic is IEEE single precision with round-to-nearest-even, in the
+// canonical order of each rotation:
+//   Sylvester H_b (b = 64, 128, 256): the textbook in-place fast
+//     Walsh-Hadamard transform, stages h = 1, 2, ..., b/2, butterfly
+//     (u, w) -> (u + w, u - w); blocks wider than 64 span 2 or 4 lanes.
+//   regular H_4^(x)k (b = 16, 64, 256), H_4 = J - 2I: radix-4 stages with
+//     digit strides 1, 4, 16, 64; a group (x0, x1, x2, x3) becomes t - 2 x_i
+//     with t = (x0 + x1) + (x2 + x3) (2 x_i is exact, so t - 2 x_i is one
+//     rounding, done as fma(-2, x_i, t)); the order-256 block spans 4 lanes.
 #pragma once
 
 #include <cstdint>
 
+#include "kernels.h"
 #include "ptx.cuh"
 
 namespace convrot {
 namespace qcore {
 
-#ifndef CONVROT_RQ_EPT
-#define CONVROT_RQ_EPT 64  // elements each thread owns (32 or 64)
-#endif
-constexpr int kPerThread = CONVROT_RQ_EPT;
-static_assert(kPerThread == 32 || kPerThread == 64, "32 or 64 elements per thread");
-constexpr int kPairs = kPerThread / 2;          // P[j] = (element j, element j + kPairs)
-constexpr int kLanesPerBlock = 128 / kPerThread;  // lanes sharing one Hadamard block
+constexpr int kPerThread = 64;            // elements each thread owns
+constexpr int kPairs = kPerThread / 2;    // P[j] = (element j, element j + kPairs)
 
 // ---- packed single-precision pairs (one 64-bit register pair)
 
@@ -215,13 +217,80 @@ __device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], floa
                      : "memory");
 }
 
-// The whole 128-point transform of this thread's piece; t is the thread's
-// index within its row (lanes t and t^1 share a block).
-__device__ __forceinline__ void fwht128(uint64_t (&P)[kPairs], int t) {
-    fwht_in_registers(P);
+// ---- regular H_4^(x)k stages
+
+// One radix-4 group of packed pairs: (X0, X1, X2, X3) -> T - 2 X_i with
+// T = (X0 + X1) + (X2 + X3), both halves of every pair at once.
+__device__ __forceinline__ void reg_group(uint64_t& X0, uint64_t& X1, uint64_t& X2, uint64_t& X3) {
+    const uint64_t m2 = pk(-2.0f, -2.0f);
+    const uint64_t T = add2(add2(X0, X1), add2(X2, X3));
+    X0 = fma2(m2, X0, T);
+    X1 = fma2(m2, X1, T);
+    X2 = fma2(m2, X2, T);
+    X3 = fma2(m2, X3, T);
+}
+
+// Digit stride ST (1 or 4) inside each half: the group (e, e+ST, e+2ST,
+// e+3ST) of elements is the same group of pair indices, in both halves.
+template <int ST>
+__device__ __forceinline__ void reg_stage_pairs(uint64_t (&P)[kPairs]) {
 #pragma unroll
-    for (int sh = 1; sh < kLanesPerBlock; sh <<= 1)  // h = kPerThread * sh
-        fwht_across_lanes(P, sh, (t & sh) != 0);
+    for (int j = 0; j < kPairs; ++j) {
+        if ((j / ST) % 4 == 0) reg_group(P[j], P[j + ST], P[j + 2 * ST], P[j + 3 * ST]);
+    }
+}
+
+// Digit stride 16: the group (e, e+16, e+32, e+48) is
+// (P[e].lo, P[e+16].lo, P[e].hi, P[e+16].hi); t = (x0 + x1) + (x2 + x3) is
+// the packed sum of the two pairs followed by the sum of its halves.
+__device__ __forceinline__ void reg_stage16(uint64_t (&P)[kPairs]) {
+    const uint64_t m2 = pk(-2.0f, -2.0f);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float s01, s23;
+        upk(add2(P[e], P[e + 16]), s01, s23);
+        const float t = __fadd_rn(s01, s23);
+        const uint64_t T = pk(t, t);
+        P[e] = fma2(m2, P[e], T);
+        P[e + 16] = fma2(m2, P[e + 16], T);
+    }
+}
+
+// Digit stride 64: the four 64-element pieces of an order-256 block sit in
+// lanes t, t^1, t^2, t^3 (t & 3 = piece).  First u = own + partner(^1), i.e.
+// x0 + x1 or x2 + x3 (addition commutes, so both partners round alike), then
+// t = u + partner(^2)'s u = (x0 + x1) + (x2 + x3) in every lane.
+__device__ __forceinline__ void reg_stage_lanes(uint64_t (&P)[kPairs]) {
+    const uint64_t m2 = pk(-2.0f, -2.0f);
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        upk(P[j], a, b);
+        const uint64_t U = add2(P[j], pk(__shfl_xor_sync(0xFFFFFFFFu, a, 1), __shfl_xor_sync(0xFFFFFFFFu, b, 1)));
+        float u0, u1;
+        upk(U, u0, u1);
+        const uint64_t T = add2(U, pk(__shfl_xor_sync(0xFFFFFFFFu, u0, 2), __shfl_xor_sync(0xFFFFFFFFu, u1, 2)));
+        P[j] = fma2(m2, P[j], T);
+    }
+}
+
+// ---- the rotation kinds
+
+// The whole block transform of this thread's piece; t is the thread's index
+// within its row (lanes sharing a block are t ^ 1 and, for 256, t ^ 2, t ^ 3).
+template <int KIND>
+__device__ __forceinline__ void rotate_piece(uint64_t (&P)[kPairs], int t) {
+    if constexpr (KIND == kRotSyl64 || KIND == kRotSyl128 || KIND == kRotSyl256) {
+        fwht_in_registers(P);  // h = 1 .. 32
+        if constexpr (KIND != kRotSyl64) fwht_across_lanes(P, 1, (t & 1) != 0);  // h = 64
+        if constexpr (KIND == kRotSyl256) fwht_across_lanes(P, 2, (t & 2) != 0);  // h = 128
+    } else if constexpr (KIND == kRotReg16 || KIND == kRotReg64 || KIND == kRotReg256) {
+        reg_stage_pairs<1>(P);
+        reg_stage_pairs<4>(P);
+        if constexpr (KIND != kRotReg16) reg_stage16(P);
+        if constexpr (KIND == kRotReg256) reg_stage_lanes(P);
+    }
+    (void)t;
 }
 
 // Largest |z| over this thread's piece.

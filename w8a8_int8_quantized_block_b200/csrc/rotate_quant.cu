@@ -49,7 +49,7 @@ namespace {
 
 using namespace qcore;
 
-constexpr int kMaxThreads = kPerThread == 32 ? 1024 : 512;
+constexpr int kMaxThreads = 512;
 // 80 registers and two ring slots let eight 96-thread CTAs share an SM (the
 // kernel is latency-bound; more rows in flight beat more registers per thread).
 #ifndef CONVROT_RQ_MAXREG
@@ -70,7 +70,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-template <typename Tin, int BLOCK>
+template <typename Tin, int KIND>
 __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
                                                             int tpr, int tpr_pad, int rows_per_cta, int rows128,
                                                             int box1, int nbox, int nstage, int64_t num_groups,
@@ -142,7 +142,7 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
             for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
         }
 
-        if constexpr (BLOCK == 128) fwht128(P, t);
+        rotate_piece<KIND>(P, t);
         float amax = piece_absmax(P);
         if (!long_rows) {
             for (int o = tpr_pad >> 1; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -180,10 +180,10 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
     }
 }
 
-template <typename Tin, int BLOCK>
+template <typename Tin, int KIND>
 cudaError_t launch_typed(const CUtensorMap& xmap, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
                          float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
-    auto kern = rotate_quant_kernel<Tin, BLOCK>;
+    auto kern = rotate_quant_kernel<Tin, KIND>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(g.smem_bytes));
     if (e != cudaSuccess) return e;
@@ -262,16 +262,28 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
     return g->smem_bytes <= budget;
 }
 
-cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int block, int64_t M, int64_t K,
+template <typename Tin>
+cudaError_t launch_kind(const CUtensorMap& xmap, int kind, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
+                        float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
+    switch (kind) {
+        case kRotNone: return launch_typed<Tin, kRotNone>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotSyl64: return launch_typed<Tin, kRotSyl64>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotSyl128: return launch_typed<Tin, kRotSyl128>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotSyl256: return launch_typed<Tin, kRotSyl256>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotReg16: return launch_typed<Tin, kRotReg16>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotReg64: return launch_typed<Tin, kRotReg64>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotReg256: return launch_typed<Tin, kRotReg256>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
                                 unsigned int* err, int num_sms, cudaStream_t stream) {
     (void)K;
-    const bool rot = block == 128;
     if (in_elem_bytes == 2)
-        return rot ? launch_typed<__nv_bfloat16, 128>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream)
-                   : launch_typed<__nv_bfloat16, 0>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-    return rot ? launch_typed<float, 128>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream)
-               : launch_typed<float, 0>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        return launch_kind<__nv_bfloat16>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+    return launch_kind<float>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
 }
 
 namespace {
