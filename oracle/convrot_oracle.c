@@ -49,6 +49,14 @@
  *  GEMM        acc[m][n] = sum_k qx[m][k] * qw[n][k], exact in int64
  *              ("W8A8 INT8" -- HyperFlow H3 Flash card, "Choose a Weight
  *              Format").
+ *  activation  the down projection's input, "SwiGLU + ConvRot64 + Rowwise
+ *  prologue    INT8 Quantize" fused in MLP.fc2 (MiniMax-H3-Rung-Omega README,
+ *              "Technical Architecture Overview", item 2, Floor 1): from the
+ *              up projection's bf16 output h, x = silu(g) * u with
+ *              silu(g) = g / (1 + exp(-g)) and [g | u] the two halves of h's
+ *              row (gate first), or x = gelu(h) = h Phi(h) = 0.5 h erfc(-h/sqrt 2);
+ *              computed in fp64 and rounded once to f32, the precision the
+ *              rotation and the quantiser then work in.
  *  dequant     y = acc * s_x[m] * s_w[n] * alpha + bias[n] in fp64, where
  *              alpha = 1/b for a rotated pair (b = 0 or 1: alpha = 1);
  *              optional exact-erf GELU.
@@ -194,6 +202,47 @@ void oracle_quantize_act_bf16(const uint16_t *x, int64_t M, int64_t K, int64_t l
     }
 }
 
+/* gelu(y) = y * Phi(y), Phi the standard normal CDF, written as
+ * 0.5 * erfc(-y / sqrt 2): the same function as 0.5 * (1 + erf(y / sqrt 2))
+ * without the cancellation that form suffers for negative y. */
+static double gelu_f64(double y) { return 0.5 * y * erfc(-y / sqrt(2.0)); }
+static double silu_f64(double g) { return g / (1.0 + exp(-g)); }
+
+/* The activation of one row: act 0 = none (x = h), 1 = GELU (x = gelu(h),
+ * h has K columns), 2 = SwiGLU (x = silu(g) * u, g = h[0..K), u = h[K..2K)).
+ * Each x is the fp64 value rounded once to f32. */
+static void act_row_f32(const uint16_t *h, int64_t K, int act, float *x) {
+    for (int64_t k = 0; k < K; ++k) {
+        double v = (double)bf16_bits_to_f32(h[k]);
+        if (act == 1) v = gelu_f64(v);
+        else if (act == 2) v = silu_f64(v) * (double)bf16_bits_to_f32(h[K + k]);
+        x[k] = (float)v;
+    }
+}
+
+/* The activation alone, for the pins: x [M][K] f32. */
+void oracle_act_f32(const uint16_t *h, int64_t M, int64_t K, int64_t ldh, int act, float *x) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) act_row_f32(h + m * ldh, K, act, x + m * K);
+}
+
+/* Activation prologue + rotation + rowwise quantisation (the down
+ * projection's input): h bf16 rows of K (GELU) or 2K (SwiGLU) columns. */
+void oracle_act_quantize_bf16(const uint16_t *h, int64_t M, int64_t K, int64_t ldh, int act,
+                              int b, int regular, int8_t *q, int64_t ldq, float *s) {
+#pragma omp parallel
+    {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+        for (int64_t m = 0; m < M; ++m) {
+            act_row_f32(h + m * ldh, K, act, row);
+            oracle_rotate_f32(row, K, b, regular);
+            quantize_row(row, K, q + m * ldq, s + m);
+        }
+        free(row);
+    }
+}
+
 /* Weights: f32 [N, K] rows -> same rotation along K -> int8 + per-row scale. */
 void oracle_pack_weight_f32(const float *w, int64_t N, int64_t K, int b, int regular,
                             int8_t *q, float *s) {
@@ -239,7 +288,6 @@ void oracle_igemm_s64_pairs(const int8_t *A, int64_t lda, const int8_t *B, int64
     }
 }
 
-static double gelu_f64(double y) { return 0.5 * y * (1.0 + erf(y / sqrt(2.0))); }
 
 /* y = acc * s_a[m] * s_b[n] * alpha + bias[n] (bias may be NULL), in fp64. */
 void oracle_dequant_f64(const int64_t *acc, int64_t M, int64_t N,

@@ -15,6 +15,9 @@ Every function cites the passage it follows (page title and section):
   pruned INT8 ConvRot - input-major", section "Input-major checkpoint";
 * exact undo of the rotation -- "HyperFlow H3 Flash MLX", section "How to run";
 * W8A8 INT8 -- HyperFlow H3 Flash card, "Choose a Weight Format";
+* the activation prologue of the down projection ("SwiGLU + ConvRot64 +
+  Rowwise INT8 Quantize" in MLP.fc2) -- MiniMax-H3-Rung-Omega README,
+  "Technical Architecture Overview", item 2;
 * the regular rotation H_4^(x)k ("DC-balanced regular orthogonal Hadamard
   matrix H_256 = H_4^(x)4") -- MiniMax-H3-Rung-Omega README, "Technical
   Architecture Overview", item 1.
@@ -44,7 +47,8 @@ CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-s
 
 __all__ = [
     "build", "lib", "num_threads", "hadamard", "hadamard_sylvester", "hadamard_regular_kron", "fwht",
-    "quantize_rows", "quantize_act", "pack_weight", "igemm", "igemm_pairs",
+    "quantize_rows", "quantize_act", "act_f32", "act_quantize", "ACT_NONE", "ACT_GELU", "ACT_SWIGLU",
+    "pack_weight", "igemm", "igemm_pairs",
     "dequant", "dequant_pairs", "linear", "rotate_explicit_f64",
     "bf16_bits", "bf16_bits_to_f32", "py_fwht_exact", "py_quantize_row_exact",
     "py_igemm",
@@ -81,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_quantize_rows_f32.argtypes = [P, I64, I64, I64, P, I64, P]
         L.oracle_quantize_act_bf16.argtypes = [P, I64, I64, I64, I32, I32, P, I64, P]
         L.oracle_pack_weight_f32.argtypes = [P, I64, I64, I32, I32, P, P]
+        L.oracle_act_f32.argtypes = [P, I64, I64, I64, I32, P]
+        L.oracle_act_quantize_bf16.argtypes = [P, I64, I64, I64, I32, I32, I32, P, I64, P]
         L.oracle_igemm_s64.argtypes = [P, I64, P, I64, I64, I64, I64, P, I64]
         L.oracle_igemm_s64_pairs.argtypes = [P, I64, P, I64, I64, P, P, I64, P]
         L.oracle_dequant_f64.argtypes = [P, I64, I64, P, P, P, ctypes.c_double, I32, P]
@@ -185,6 +191,40 @@ def quantize_act(x_bits: np.ndarray, b: int, regular: bool = False):
     q = np.empty((M, K), dtype=np.int8)
     s = np.empty((M,), dtype=np.float32)
     lib().oracle_quantize_act_bf16(_p(x_bits), M, K, K, b, int(regular), _p(q), K, _p(s))
+    return q, s
+
+
+ACT_NONE, ACT_GELU, ACT_SWIGLU = 0, 1, 2
+
+
+def _act_width(h_bits: np.ndarray, act: int) -> int:
+    cols = h_bits.shape[1]
+    if act == ACT_SWIGLU:
+        assert cols % 2 == 0
+        return cols // 2
+    return cols
+
+
+def act_f32(h_bits: np.ndarray, act: int) -> np.ndarray:
+    """The activation alone: x = gelu(h) or silu(g) * u ([g | u] = h's halves),
+    each value computed in fp64 and rounded once to f32."""
+    h_bits = np.ascontiguousarray(h_bits, dtype=np.uint16)
+    M = h_bits.shape[0]
+    K = _act_width(h_bits, act)
+    x = np.empty((M, K), dtype=np.float32)
+    lib().oracle_act_f32(_p(h_bits), M, K, h_bits.shape[1], act, _p(x))
+    return x
+
+
+def act_quantize(h_bits: np.ndarray, act: int, b: int, regular: bool = False):
+    """Activation prologue + rotation + rowwise int8: the down projection's
+    (q, s_x) from the up projection's bf16 output h ([M, K] or [M, 2K])."""
+    h_bits = np.ascontiguousarray(h_bits, dtype=np.uint16)
+    M = h_bits.shape[0]
+    K = _act_width(h_bits, act)
+    q = np.empty((M, K), dtype=np.int8)
+    s = np.empty((M,), dtype=np.float32)
+    lib().oracle_act_quantize_bf16(_p(h_bits), M, K, h_bits.shape[1], act, b, int(regular), _p(q), K, _p(s))
     return q, s
 
 

@@ -29,7 +29,12 @@ MUTANTS = {
                                "double v = (double)acc[m * N + n] * (double)s_a[m] * (double)s_b[n];"),
     "dequant_drops_bias": ("            if (bias) v += (double)bias[n];\n            if (gelu) v = gelu_f64(v);\n            y[m * N + n] = v;",
                            "            if (gelu) v = gelu_f64(v);\n            y[m * N + n] = v;"),
-    "gelu_half_missing": ("return 0.5 * y * (1.0 + erf(y / sqrt(2.0)));", "return y * (1.0 + erf(y / sqrt(2.0)));"),
+    "gelu_half_missing": ("return 0.5 * y * erfc(-y / sqrt(2.0));", "return y * erfc(-y / sqrt(2.0));"),
+    "gelu_erfc_sign": ("return 0.5 * y * erfc(-y / sqrt(2.0));", "return 0.5 * y * erfc(y / sqrt(2.0));"),
+    "silu_sign": ("static double silu_f64(double g) { return g / (1.0 + exp(-g)); }",
+                  "static double silu_f64(double g) { return g / (1.0 + exp(g)); }"),
+    "swiglu_halves_swapped": ("else if (act == 2) v = silu_f64(v) * (double)bf16_bits_to_f32(h[K + k]);",
+                              "else if (act == 2) v = (double)bf16_bits_to_f32(h[K + k]) * 0 + silu_f64((double)bf16_bits_to_f32(h[K + k])) * v;"),
     "regular_output_drops_factor_2": ("v[j] = t - 2.0f * x0;", "v[j] = t - x0;"),
     "regular_missing_last_stage": ("for (int st = 1; st < b; st *= 4) {\n        for (int i = 0; i < b; i += 4 * st) {",
                                    "for (int st = 1; st < b / 4; st *= 4) {\n        for (int i = 0; i < b; i += 4 * st) {"),

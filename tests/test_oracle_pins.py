@@ -402,3 +402,84 @@ def test_linear_with_other_blocks_matches_unquantised_product(b, regular):
     # rotating spreads the outlier channel: the error is well below no rotation
     y0, *_ = O.linear(xb, w, bias, 0)
     assert rel < np.linalg.norm(y0 - ref) / np.linalg.norm(ref)
+
+
+# ------------------------------------------------------------ activation prologue (down projection)
+
+# Standard normal CDF from printed tables: Phi(0.5), Phi(1), Phi(2), Phi(3);
+# Phi(-x) = 1 - Phi(x); Phi(-10) = 7.619853024160527e-24.
+_PHI = {0.5: 0.6914624612740131, 1.0: 0.8413447460685429, 2.0: 0.9772498680518208, 3.0: 0.9986501019683699}
+
+
+def test_gelu_is_h_times_the_normal_cdf():
+    h, expect = [0.0], [0.0]
+    for x, p in _PHI.items():
+        h += [x, -x]
+        expect += [x * p, -x * (1.0 - p)]
+    h += [10.0, -10.0]
+    expect += [10.0, -10.0 * 7.619853024160527e-24]
+    a = O.act_f32(_bf16([h]), O.ACT_GELU)[0]
+    assert (a == np.array(expect, dtype=np.float32)).all(), (a, np.array(expect, dtype=np.float32))
+
+
+def test_gelu_odd_part_is_the_identity():
+    # gelu(x) - gelu(-x) = x Phi(x) + x Phi(-x) = x: each side is rounded
+    # once to f32, so the identity holds to one ulp of x
+    rng = np.random.default_rng(21)
+    x = O.bf16_bits_to_f32(_bf16(rng.standard_normal(4096) * 3))
+    a = O.act_f32(_bf16([x]), O.ACT_GELU)[0].astype(np.float64)
+    b = O.act_f32(_bf16([-x]), O.ACT_GELU)[0].astype(np.float64)
+    assert (np.abs(a - b - x) <= np.spacing(np.abs(x).astype(np.float32)).astype(np.float64) + 1e-45).all()
+
+
+def test_silu_and_swiglu_closed_forms_gate_first():
+    # silu(g) = g / (1 + e^-g): silu(2) = 2/(1 + e^-2), silu(-2), silu(1)
+    s2, sm2, s1 = 1.7615941559557646, -0.2384058440442351, 0.7310585786300049
+    g = [2.0, -2.0, 1.0, 0.0, 20.0]
+    u = [3.0, 0.5, -4.0, 7.0, 1.0]
+    a = O.act_f32(_bf16([g + u]), O.ACT_SWIGLU)[0]
+    expect = np.array([3 * s2, 0.5 * sm2, -4 * s1, 0.0, 20.0], dtype=np.float32)
+    assert (a == expect).all(), (a, expect)
+
+
+def test_silu_odd_part_is_the_identity():
+    # silu(x) - silu(-x) = x (sigmoid(x) + sigmoid(-x) = 1), with u = 1
+    rng = np.random.default_rng(22)
+    x = O.bf16_bits_to_f32(_bf16(rng.standard_normal(2048) * 4))
+    one = np.ones_like(x)
+    a = O.act_f32(_bf16([np.concatenate([x, one])]), O.ACT_SWIGLU)[0].astype(np.float64)
+    b = O.act_f32(_bf16([np.concatenate([-x, one])]), O.ACT_SWIGLU)[0].astype(np.float64)
+    assert (np.abs(a - b - x) <= np.spacing(np.abs(x).astype(np.float32)).astype(np.float64) + 1e-45).all()
+
+
+@pytest.mark.parametrize("b,regular", [(0, False), (64, False), (128, False), (64, True)])
+def test_act_none_prologue_is_the_plain_quantiser(b, regular):
+    rng = np.random.default_rng(23)
+    h = _bf16(rng.standard_normal((9, 256)) * 2)
+    q1, s1 = O.act_quantize(h, O.ACT_NONE, b, regular)
+    q2, s2 = O.quantize_act(h, b, regular)
+    assert (q1 == q2).all() and (s1.view(np.uint32) == s2.view(np.uint32)).all()
+
+
+@pytest.mark.parametrize("act", [1, 2])
+def test_down_projection_with_prologue_matches_unquantised_product(act):
+    # the prologue's codes times the packed down weights approximate
+    # act(h) W^T, with act from the library's erf / exp in fp64
+    import math
+    rng = np.random.default_rng(24 + act)
+    M, K, N = 20, 512, 48
+    h = rng.standard_normal((M, 2 * K if act == 2 else K)) * 1.5
+    hb = _bf16(h)
+    hf = O.bf16_bits_to_f32(hb).astype(np.float64)
+    if act == 1:
+        x = hf * 0.5 * np.vectorize(math.erfc)(-hf / math.sqrt(2.0))
+    else:
+        g, u = hf[:, :K], hf[:, K:]
+        x = g / (1.0 + np.exp(-g)) * u
+    w = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    for b in (64, 128):
+        qx, sx = O.act_quantize(hb, act, b)
+        qw, sw = O.pack_weight(w, b)
+        y = O.dequant(O.igemm(qx, qw), sx, sw, None, b)
+        ref = x @ w.T.astype(np.float64)
+        assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.02
