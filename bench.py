@@ -71,6 +71,12 @@ def parse():
     ap.add_argument("--block", choices=sorted(BLOCK_CHOICES), default="128",
                     help="rotation of the step: Sylvester H_b (64, 128, 256) or the regular H_4^(x)k "
                          "(reg16, reg64, reg256); the headline is 128")
+    ap.add_argument("--workload", choices=["proj", "mlp"], default="proj",
+                    help="proj: the 768p projection (the headline); mlp: the 768p MLP, up 5376 -> 21504 with "
+                         "GELU, then down, timed by both routes of the activation (see --mlp-route)")
+    ap.add_argument("--mlp-route", choices=["prologue", "epilogue"], default="prologue",
+                    help="the route the mlp line's value is for: GELU as the down projection's prologue "
+                         "(convrot_linear_act) or in the up projection's epilogue; both are timed")
     ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm"], default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
                          "(for profiler captures; prints no result line)")
@@ -278,6 +284,106 @@ def config_dict(spec, n):
 # ---------------------------------------------------------------------------- GPU path
 
 
+MLP_METRIC = "ConvRot W8A8 MLP TOPS at M=38656, K=5376, H=21504 (up + GELU + down)"
+
+
+def run_mlp(args, rank: int, world: int):
+    """The 768p MLP step by both routes of its GELU: in the up projection's
+    epilogue (then the plain quantiser on the down projection's input), or as
+    the down projection's prologue (convrot_linear_act on the plain up
+    projection's output).  The line's value is for --mlp-route."""
+    import torch
+    import torch.distributed as dist
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+
+    spec = W.MLP_768P
+    x_cpu, w1_cpu, w2_cpu = W.mlp_inputs(spec)
+    x = x_cpu.cuda()
+    p1 = C.pack_weight(w1_cpu.cuda(), spec.block)
+    p2 = C.pack_weight(w2_cpu.cuda(), spec.block)
+    del w1_cpu, w2_cpu
+    ws1 = C.alloc_workspace(spec.M, spec.K)
+    ws2 = C.alloc_workspace(spec.M, spec.H)
+    h = torch.empty(spec.M, spec.H, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(spec.M, spec.K, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def up(gelu):
+        C.linear_fused(x, p1, None, gelu=gelu, workspace=ws1, out=h, stream=stream)
+
+    def down(prologue):
+        if prologue:
+            C.linear_act(h, C.ACT_GELU, p2, None, workspace=ws2, out=y, stream=stream)
+        else:
+            C.linear_fused(h, p2, None, workspace=ws2, out=y, stream=stream)
+
+    routes = {"epilogue": (lambda: (up(True), down(False))), "prologue": (lambda: (up(False), down(True)))}
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for r in routes.values():
+        for _ in range(max(3, args.warmup)):
+            r()
+    barrier()
+    times, kern = {}, {}
+    clk_summary = None
+    for name in ("epilogue", "prologue"):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            barrier()
+            e0.record(stream)
+            for _ in range(args.steps):
+                routes[name]()
+            e1.record(stream)
+            barrier()
+        times[name] = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+        if name == args.mlp_route:
+            clk_summary = clk.summary()
+        # per launch: up projection, then the down projection's two kernels
+        nk = min(args.steps, 50)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nk)]
+        barrier()
+        for i in range(nk):
+            ev[i][0].record(stream)
+            up(name == "epilogue")
+            ev[i][1].record(stream)
+            down(name == "prologue")
+            ev[i][2].record(stream)
+        barrier()
+        kern[name] = {"up_us": sum(e[0].elapsed_time(e[1]) for e in ev) / nk * 1e3,
+                      "down_us": sum(e[1].elapsed_time(e[2]) for e in ev) / nk * 1e3}
+    st, code = C.last_device_status()
+    if st != C.OK:
+        raise RuntimeError(f"device status {st} (code {code})")
+    if rank == 0:
+        hbm, bf16, kind = peaks()
+        int8_peak = bf16 * INT8_PER_BF16
+        t = times[args.mlp_route]
+        value = job_tops(spec.ops, args.steps, world, t)
+        line = {
+            "metric": MLP_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "H": spec.H, "block": spec.block,
+                       "activation": "gelu", "route": args.mlp_route,
+                       "parallelism": f"dp{world} (independent token batches per GPU)",
+                       "l2": "inputs larger than L2: h is 1.66 GB per step"},
+            "pct_of_int8_peak": round(100.0 * value / world / int8_peak, 2),
+            "routes": {n: {"TOPS": job_tops(spec.ops, args.steps, world, times[n]),
+                           "ms_per_step": times[n] / args.steps * 1e3, **kern[n]} for n in times},
+            "clocks": clk_summary,
+            "gpu_launches": 3 * args.steps,  # up (one kernel), down (prologue quantiser + GEMM)
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -296,6 +402,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+    if args.workload == "mlp":
+        return run_mlp(args, rank, world)
     spec = workload(args)
     x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
     x = x_cpu.cuda()

@@ -134,14 +134,43 @@ convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int
  * (M*K, rounded up to 256) plus the scales (4*M, rounded up to 256). */
 size_t convrot_workspace_bytes(int64_t M, int64_t K);
 
-/* The whole linear, steps 1-4, in two kernels on `stream` (the GEMM starts
- * while the quantiser drains).  x: bf16 [M][K] (row stride ldx); the codes and
- * scales go to `workspace` (>= convrot_workspace_bytes(M, K) bytes, 256-byte
- * aligned, caller-owned, must not be shared by calls that overlap). */
+/* The whole linear, steps 1-4, on `stream`: one kernel (quantiser warps run
+ * ahead of the tensor cores in the same CTAs) when K % 128 == 0, 128 <= K <=
+ * 6144, x is 32-byte aligned and ldx % 16 == 0; otherwise two kernels (the
+ * GEMM starts while the quantiser drains).  x: bf16 [M][K] (row stride ldx);
+ * the codes and scales go to `workspace` (>= convrot_workspace_bytes(M, K)
+ * bytes, 256-byte aligned, caller-owned, must not be shared by calls that
+ * overlap). */
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw,
                                     const float* s_w, const convrot_wdesc* desc, const float* bias,
                                     int32_t epilogue, void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy,
                                     void* stream);
+
+/* Activation prologue of a down projection: the rotation and quantisation
+ * of act(h), where h is the up projection's bf16 output ("SwiGLU + ConvRot64
+ * + Rowwise INT8 Quantize" fused in MLP.fc2 -- MiniMax-H3-Rung-Omega README,
+ * "Technical Architecture Overview", item 2).  The pages print no formula;
+ * the reading here:
+ *   CONVROT_ACT_GELU    x = gelu(h) = h * Phi(h), h: bf16 [M][K];
+ *   CONVROT_ACT_SWIGLU  x = silu(g) * u, silu(g) = g / (1 + e^-g), where each
+ *                       row of h holds 2K bf16: g = h[m][0..K), u = h[m][K..2K).
+ * x is computed in f32 and goes straight into the rotation and quantiser of
+ * convrot_quantize_act (same block values, same q / s_x); it is never stored.
+ * Requires ldh >= K (GELU) or 2K (SwiGLU), ldh % 8 == 0, K % 64 == 0,
+ * K % b == 0, K <= 32768.  Any other act is CONVROT_EINVAL. */
+#define CONVROT_ACT_NONE 0
+#define CONVROT_ACT_GELU 1
+#define CONVROT_ACT_SWIGLU 2
+convrot_status convrot_act_quantize(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, int32_t act,
+                                    int32_t block, int8_t* q, float* s_x, void* stream);
+
+/* The down projection with the activation prologue: convrot_act_quantize of
+ * h into `workspace` (as convrot_linear_fused lays it out), then steps 3-4
+ * with the packed weights (K = desc->K).  Two kernels on `stream`; the GEMM
+ * starts while the prologue drains. */
+convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int32_t act, const int8_t* qw,
+                                  const float* s_w, const convrot_wdesc* desc, const float* bias, int32_t epilogue,
+                                  void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy, void* stream);
 
 /* End-to-end form of convrot_linear_fused for callers whose activations live
  * in host memory: copies x_host (bf16 [M][K], contiguous; pinned for overlap)

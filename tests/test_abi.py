@@ -94,6 +94,28 @@ def test_regular_flag_matches_the_header():
     assert [C.block_length(b) for b in C.BLOCKS] == [1, 64, 128, 256, 16, 64, 256]
 
 
+def test_activation_prologue_rejects_bad_arguments():
+    L = C.load()
+    # unknown activation, and "none" (that is convrot_quantize_act's job)
+    assert L.convrot_act_quantize(FAKE, 4, 512, 512, 7, 128, FAKE, FAKE, None) == C.EINVAL
+    assert L.convrot_act_quantize(FAKE, 4, 512, 512, C.ACT_NONE, 128, FAKE, FAKE, None) == C.EINVAL
+    # SwiGLU rows hold 2K elements: ldh must reach them
+    assert L.convrot_act_quantize(FAKE, 4, 512, 512, C.ACT_SWIGLU, 128, FAKE, FAKE, None) == C.EINVAL
+    assert L.convrot_act_quantize(FAKE, 4, 512, 512, C.ACT_GELU, 32, FAKE, FAKE, None) == C.EUNSUPPORTED
+    d = _desc()
+    assert L.convrot_linear_act(FAKE, 16, 512, 9, FAKE, FAKE, ctypes.byref(d), None, 0, FAKE, 1 << 20, FAKE, 512,
+                                None) == C.EINVAL
+    assert L.convrot_linear_act(FAKE, 16, 512, C.ACT_GELU, FAKE, FAKE, ctypes.byref(d), None, 0, FAKE, 16, FAKE,
+                                512, None) == C.EINVAL  # workspace too small
+
+
+def test_activation_prologue_valid_call_without_a_gpu_reports_cuda_error():
+    _skip_if_gpu()
+    L = C.load()
+    assert L.convrot_act_quantize(FAKE, 4, 512, 1024, C.ACT_SWIGLU, 64, FAKE, FAKE, None) == C.ECUDA
+    assert L.convrot_act_quantize(FAKE, 4, 512, 512, C.ACT_GELU, C.REGULAR | 256, FAKE, FAKE, None) == C.ECUDA
+
+
 def test_null_pointers_rejected():
     L = C.load()
     assert L.convrot_quantize_act(None, 4, 512, 512, 128, FAKE, FAKE, None) == C.EINVAL

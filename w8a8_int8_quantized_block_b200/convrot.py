@@ -25,6 +25,8 @@ LAYOUT_OUTPUT_MAJOR = 1
 # = the regular H_4^(x)k (H_4 = J - 2I).
 REGULAR = 0x10000
 BLOCKS = (0, 64, 128, 256, REGULAR | 16, REGULAR | 64, REGULAR | 256)
+# Activation prologues of a down projection (convrot_act_quantize).
+ACT_NONE, ACT_GELU, ACT_SWIGLU = 0, 1, 2
 
 
 def block_length(block: int) -> int:
@@ -37,7 +39,7 @@ EXPORTS = (
     "convrot_status_string", "convrot_abi_version", "convrot_pack_weight", "convrot_quantize_act",
     "convrot_w8a8_linear", "convrot_workspace_bytes", "convrot_linear_fused", "convrot_linear_fused_host",
     "convrot_w8a8_bmm", "convrot_igemm_s32", "convrot_last_device_status", "convrot_set_wait_limit_ns",
-    "convrot_selftest_wait_timeout", "convrot_linear_fused_noalloc",
+    "convrot_selftest_wait_timeout", "convrot_linear_fused_noalloc", "convrot_act_quantize", "convrot_linear_act",
 )
 
 
@@ -90,6 +92,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "convrot_selftest_wait_timeout": ([U64, P], ctypes.c_int),
         "convrot_linear_fused_noalloc": ([P, I64, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, I64, P],
                                          ctypes.c_int),
+        "convrot_act_quantize": ([P, I64, I64, I64, I32, I32, P, P, P], ctypes.c_int),
+        "convrot_linear_act": ([P, I64, I64, I32, P, P, ctypes.POINTER(WDesc), P, I32, P, ctypes.c_size_t, P, I64,
+                                P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -163,6 +168,46 @@ def quantize_act(x: torch.Tensor, block: int = 128, q: torch.Tensor | None = Non
     _check("convrot_quantize_act", load().convrot_quantize_act(_ptr(x), M, K, x.stride(0), block, _ptr(q), _ptr(s),
                                                                _stream(stream)))
     return q, s
+
+
+def _act_width(h: torch.Tensor, act: int) -> int:
+    if h.dim() != 2 or h.stride(1) != 1:
+        raise ValueError("h must be 2-D with unit column stride")
+    if act == ACT_SWIGLU:
+        if h.shape[1] % 2:
+            raise ValueError("a SwiGLU input holds gate and up halves: an even number of columns")
+        return h.shape[1] // 2
+    return h.shape[1]
+
+
+def act_quantize(h: torch.Tensor, act: int, block: int = 128, q: torch.Tensor | None = None,
+                 s: torch.Tensor | None = None, stream=None):
+    """The down projection's input: rotate + quantise act(h) (ACT_GELU on
+    h [M, K], or ACT_SWIGLU on h [M, 2K] = [gate | up]) -> (q [M, K], s [M])."""
+    _need(h, torch.bfloat16, "h")
+    K = _act_width(h, act)
+    M = h.shape[0]
+    q = torch.empty((M, K), dtype=torch.int8, device=h.device) if q is None else q
+    s = torch.empty((M,), dtype=torch.float32, device=h.device) if s is None else s
+    _check("convrot_act_quantize", load().convrot_act_quantize(_ptr(h), M, K, h.stride(0), act, block, _ptr(q),
+                                                               _ptr(s), _stream(stream)))
+    return q, s
+
+
+def linear_act(h: torch.Tensor, act: int, pw: PackedWeight, bias: torch.Tensor | None = None, gelu: bool = False,
+               workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Down projection with the activation prologue: y = act(h) W^T (+ bias)."""
+    _need(h, torch.bfloat16, "h")
+    K = _act_width(h, act)
+    if K != pw.K:
+        raise ValueError(f"act(h) has {K} columns, the weights {pw.K}")
+    M = h.shape[0]
+    ws = alloc_workspace(M, pw.K, h.device) if workspace is None else workspace
+    y = torch.empty((M, pw.N), dtype=torch.bfloat16, device=h.device) if out is None else out
+    _check("convrot_linear_act", load().convrot_linear_act(
+        _ptr(h), M, h.stride(0), act, _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias),
+        EPI_GELU if gelu else EPI_NONE, _ptr(ws), ws.numel(), _ptr(y), y.stride(0), _stream(stream)))
+    return y
 
 
 def w8a8_linear(qx: torch.Tensor, sx: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None,

@@ -112,21 +112,26 @@ bool decode_block(int32_t block, int* b, int* kind) {
     return true;
 }
 
-// Shared by activations (bf16) and weights (f32).
+// Shared by activations (bf16, optionally behind an activation prologue)
+// and weights (f32).  act: CONVROT_ACT_*; with SwiGLU each row of x holds
+// 2K elements (gate, then up).
 convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t K, int64_t ldx, int32_t block,
-                            int8_t* q, float* s, cudaStream_t stream) {
+                            int8_t* q, float* s, cudaStream_t stream, int32_t act = CONVROT_ACT_NONE) {
     if (!x || !q || !s) return CONVROT_EINVAL;
     if (M <= 0 || M > kMaxI32 || K <= 0) return CONVROT_EINVAL;
     int b = 1, kind = kRotNone;
     if (!decode_block(block, &b, &kind)) return CONVROT_EUNSUPPORTED;
+    if (act != CONVROT_ACT_NONE && act != CONVROT_ACT_GELU && act != CONVROT_ACT_SWIGLU) return CONVROT_EINVAL;
+    if (act != CONVROT_ACT_NONE && in_elem_bytes != 2) return CONVROT_EINVAL;
+    const int64_t row_elems = act == CONVROT_ACT_SWIGLU ? 2 * K : K;
     if (K % 64 != 0 || K > 32768 || K % b != 0) return CONVROT_EINVAL;
-    if (ldx < K || (ldx * in_elem_bytes) % 16 != 0) return CONVROT_EINVAL;
+    if (ldx < row_elems || (ldx * in_elem_bytes) % 16 != 0) return CONVROT_EINVAL;
     if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u) != 0) return CONVROT_EINVAL;
     const DeviceInfo* d = device_info();
     if (!d) return CONVROT_ECUDA;
     if (!d->supported) return CONVROT_EUNSUPPORTED;
     RqGeometry g;
-    if (!rq_geometry(K, in_elem_bytes, &g)) return CONVROT_EINVAL;
+    if (!rq_geometry(K, row_elems, in_elem_bytes, &g)) return CONVROT_EINVAL;
     CUtensorMap xmap;
     const uint32_t inner = 128u / static_cast<uint32_t>(in_elem_bytes);
     const CUtensorMapDataType dt =
@@ -135,7 +140,8 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
                    static_cast<uint64_t>(ldx) * in_elem_bytes, inner, static_cast<uint32_t>(g.box1),
                    static_cast<uint32_t>(g.rows_per_cta), CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
-    return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, kind, M, K, g, q, K, s, g_limit_ns.load(),
+    const int ak = act == CONVROT_ACT_GELU ? kActGelu : act == CONVROT_ACT_SWIGLU ? kActSwiglu : kActNone;
+    return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, kind, ak, M, K, g, q, K, s, g_limit_ns.load(),
                                            d->err, d->num_sms, stream));
 }
 
@@ -346,6 +352,30 @@ convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, c
         return linear_one_kernel(x, M, ldx, qw, s_w, desc, bias, epi, qx, sx, ready, y, ldy, s);
     st = rotate_quant(x, 2, M, desc->K, ldx, desc->block, qx, sx, s);
     if (st != CONVROT_OK) return st;
+    return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block), epi, 1, M, desc->N, desc->K, y, ldy, true, s);
+}
+
+convrot_status convrot_act_quantize(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, int32_t act,
+                                    int32_t block, int8_t* q, float* s_x, void* stream) {
+    if (act != CONVROT_ACT_GELU && act != CONVROT_ACT_SWIGLU) return CONVROT_EINVAL;
+    return rotate_quant(h, 2, M, K, ldh, block, q, s_x, static_cast<cudaStream_t>(stream), act);
+}
+
+convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int32_t act, const int8_t* qw,
+                                  const float* s_w, const convrot_wdesc* desc, const float* bias, int32_t epilogue,
+                                  void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy, void* stream) {
+    convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y, ldy, bias);
+    if (st != CONVROT_OK) return st;
+    if (act != CONVROT_ACT_GELU && act != CONVROT_ACT_SWIGLU) return CONVROT_EINVAL;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CONVROT_EINVAL;
+    if (ws_bytes < convrot_workspace_bytes(M, desc->K)) return CONVROT_EINVAL;
+    int8_t* qx = static_cast<int8_t*>(workspace);
+    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         round256(static_cast<size_t>(M) * static_cast<size_t>(desc->K)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = rotate_quant(h, 2, M, desc->K, ldh, desc->block, qx, sx, s, act);
+    if (st != CONVROT_OK) return st;
+    const int epi = epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16;
     return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block), epi, 1, M, desc->N, desc->K, y, ldy, true, s);
 }
 

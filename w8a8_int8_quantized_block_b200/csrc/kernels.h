@@ -16,15 +16,17 @@ struct RqGeometry {
     int tpr_pad;       // threads per row including idle ones (long rows: = tpr, packed back to back)
     int rows_per_cta;  // rows one CTA handles
     int threads;       // CTA size
-    int rows128;       // 128-byte shared-memory rows per input row
+    int rows128;       // 128-byte shared-memory rows per input row (all row_elems)
     int box1;          // TMA box extent along the 128-byte-row dimension
     int nbox;          // TMA boxes per input row
     int nstage;        // shared-memory ring slots (row groups in flight per CTA)
     size_t smem_bytes; // dynamic shared memory requested
 };
 
-// in_elem_bytes: 2 for bf16 activations, 4 for f32 weights.
-bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g);
+// K: elements quantised per row; row_elems: elements loaded per row (K, or
+// 2K for the SwiGLU prologue); in_elem_bytes: 2 for bf16 activations, 4 for
+// f32 weights.
+bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g);
 
 // The rotations a row can get: none, Sylvester H_b (b = 64, 128, 256) or the
 // regular H_4^(x)k (b = 16, 64, 256).
@@ -38,9 +40,14 @@ enum RotKind : int {
     kRotReg256 = 6,
 };
 
+// The activation applied before the rotation (the down projection's input):
+// none, x = gelu(h), or x = silu(g) * u with [g | u] the halves of h's row.
+enum ActKind : int { kActNone = 0, kActGelu = 1, kActSwiglu = 2 };
+
 // x: bf16 (bits) or f32 rows, described by `xmap` (3D: 128-byte inner rows,
-// rows128, M) with 128-byte swizzling.  kind: a RotKind.
-cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int64_t M, int64_t K,
+// rows128, M) with 128-byte swizzling.  kind: a RotKind; act: an ActKind
+// (bf16 rows only; with kActSwiglu each row holds 2K elements).
+cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int act, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
                                 unsigned int* err, int num_sms, cudaStream_t stream);
 

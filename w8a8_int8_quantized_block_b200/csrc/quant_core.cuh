@@ -123,6 +123,47 @@ __device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, u
     }
 }
 
+// ---- the activation prologue of the down projection
+
+// gelu(x) = x Phi(x) = 0.5 x erfc(-x / sqrt 2) (the erfc form has no
+// cancellation for negative x).
+__device__ __forceinline__ float gelu_prologue(float x) { return 0.5f * x * erfcf(-0.70710678118654752f * x); }
+
+// silu(g) = g / (1 + e^-g), IEEE division.
+__device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, 1.0f + expf(-g)); }
+
+__device__ __forceinline__ void gelu_pairs(uint64_t (&P)[kPairs]) {
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        float a, b;
+        upk(P[j], a, b);
+        P[j] = pk(gelu_prologue(a), gelu_prologue(b));
+    }
+}
+
+// x = silu(g) * u for this thread's 64 elements: P holds g; the matching u
+// are the thread's 64 bf16 of the row's second half, one 128-byte shared row
+// at 128-byte row `Ru` of the swizzled slot, read one 16-byte chunk (eight
+// elements) at a time.
+__device__ __forceinline__ void swiglu_pairs(uint64_t (&P)[kPairs], const uint8_t* slot, int Ru) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(slot + Ru * 128 + ((c ^ (Ru & 7)) << 4));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = 8 * c + i;  // element of the thread's piece
+            const float u = __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16));
+            const int j = e & (kPairs - 1);
+            float a, b;
+            upk(P[j], a, b);
+            if (e < kPairs) a = silu(a) * u;
+            else b = silu(b) * u;
+            P[j] = pk(a, b);
+        }
+    }
+}
+
 // Stages h = 1, 2, ..., kPairs/2 (packed, both halves at once) then
 // h = kPairs (inside each pair).  Butterfly (u, w) -> (u + w, u - w), u the
 // lower index.

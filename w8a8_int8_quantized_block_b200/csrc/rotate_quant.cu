@@ -55,7 +55,12 @@ constexpr int kMaxThreads = 512;
 #ifndef CONVROT_RQ_MAXREG
 #define CONVROT_RQ_MAXREG 80
 #endif
-#define CONVROT_RQ_BOUNDS __maxnreg__(CONVROT_RQ_MAXREG)
+// The activation prologues (erfc / exp per element next to 64 live values)
+// need more registers than 80; they are compute-heavy, so fewer resident
+// CTAs cost them little.
+#ifndef CONVROT_RQ_MAXREG_ACT
+#define CONVROT_RQ_MAXREG_ACT 128
+#endif
 #ifndef CONVROT_RQ_STAGES
 #define CONVROT_RQ_STAGES 2  // ring slots (row groups in flight) per CTA
 #endif
@@ -70,8 +75,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-template <typename Tin, int KIND>
-__global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
+template <typename Tin, int KIND, int ACT>
+__global__ void __maxnreg__(ACT == kActNone ? CONVROT_RQ_MAXREG : CONVROT_RQ_MAXREG_ACT) rotate_quant_kernel(const __grid_constant__ CUtensorMap xmap, int64_t M,
                                                             int tpr, int tpr_pad, int rows_per_cta, int rows128,
                                                             int box1, int nbox, int nstage, int64_t num_groups,
                                                             int8_t* __restrict__ q, int64_t ldq,
@@ -136,7 +141,10 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
 
         uint64_t P[kPairs];
         if (active) {
-            load_pairs<Tin>(ring + static_cast<size_t>(slot) * slot_bytes, rloc * row_pitch, t, P);
+            const uint8_t* sl = ring + static_cast<size_t>(slot) * slot_bytes;
+            load_pairs<Tin>(sl, rloc * row_pitch, t, P);
+            if constexpr (ACT == kActGelu) gelu_pairs(P);
+            if constexpr (ACT == kActSwiglu) swiglu_pairs(P, sl, rloc * row_pitch + tpr + t);  // u: second half
         } else {
 #pragma unroll
             for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
@@ -180,10 +188,10 @@ __global__ void CONVROT_RQ_BOUNDS rotate_quant_kernel(const __grid_constant__ CU
     }
 }
 
-template <typename Tin, int KIND>
+template <typename Tin, int KIND, int ACT>
 cudaError_t launch_typed(const CUtensorMap& xmap, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
                          float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
-    auto kern = rotate_quant_kernel<Tin, KIND>;
+    auto kern = rotate_quant_kernel<Tin, KIND, ACT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(g.smem_bytes));
     if (e != cudaSuccess) return e;
@@ -208,11 +216,11 @@ int next_pow2(int v) {
 
 }  // namespace
 
-bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
+bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g) {
     if (K <= 0 || K % 64 != 0 || K > 32768) return false;
-    if ((K * in_elem_bytes) % 128 != 0) return false;
+    if (row_elems != K && row_elems != 2 * K) return false;
     g->tpr = static_cast<int>(K / kPerThread);
-    g->rows128 = static_cast<int>(K * in_elem_bytes / 128);
+    g->rows128 = static_cast<int>(row_elems * in_elem_bytes / 128);
     if (g->tpr <= 32) {
         // Short rows: a power-of-two lane group per row, 256 threads per CTA.
         g->tpr_pad = next_pow2(g->tpr);
@@ -262,28 +270,40 @@ bool rq_geometry(int64_t K, int in_elem_bytes, RqGeometry* g) {
     return g->smem_bytes <= budget;
 }
 
-template <typename Tin>
+template <typename Tin, int ACT>
 cudaError_t launch_kind(const CUtensorMap& xmap, int kind, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
                         float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
     switch (kind) {
-        case kRotNone: return launch_typed<Tin, kRotNone>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-        case kRotSyl64: return launch_typed<Tin, kRotSyl64>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-        case kRotSyl128: return launch_typed<Tin, kRotSyl128>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-        case kRotSyl256: return launch_typed<Tin, kRotSyl256>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-        case kRotReg16: return launch_typed<Tin, kRotReg16>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-        case kRotReg64: return launch_typed<Tin, kRotReg64>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-        case kRotReg256: return launch_typed<Tin, kRotReg256>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotNone: return launch_typed<Tin, kRotNone, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotSyl64: return launch_typed<Tin, kRotSyl64, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotSyl128: return launch_typed<Tin, kRotSyl128, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotSyl256: return launch_typed<Tin, kRotSyl256, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotReg16: return launch_typed<Tin, kRotReg16, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotReg64: return launch_typed<Tin, kRotReg64, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+        case kRotReg256: return launch_typed<Tin, kRotReg256, ACT>(xmap, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int64_t M, int64_t K,
+cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int act, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
                                 unsigned int* err, int num_sms, cudaStream_t stream) {
     (void)K;
-    if (in_elem_bytes == 2)
-        return launch_kind<__nv_bfloat16>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
-    return launch_kind<float>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+    if (in_elem_bytes == 2) {
+        switch (act) {
+            case kActNone:
+                return launch_kind<__nv_bfloat16, kActNone>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+            case kActGelu:
+                return launch_kind<__nv_bfloat16, kActGelu>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
+            case kActSwiglu:
+                return launch_kind<__nv_bfloat16, kActSwiglu>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms,
+                                                              stream);
+            default:
+                return cudaErrorInvalidValue;
+        }
+    }
+    if (act != kActNone) return cudaErrorInvalidValue;  // weights take no activation
+    return launch_kind<float, kActNone>(xmap, kind, M, g, q, ldq, s, limit_ns, err, num_sms, stream);
 }
 
 namespace {
