@@ -77,6 +77,9 @@ def parse():
     ap.add_argument("--mlp-route", choices=["prologue", "epilogue"], default="prologue",
                     help="the route the mlp line's value is for: GELU as the down projection's prologue "
                          "(convrot_linear_act) or in the up projection's epilogue; both are timed")
+    ap.add_argument("--context-parallel", action="store_true",
+                    help="strong scaling: the 38656 tokens split across the ranks, each step the rank's linear "
+                         "then an NCCL all-gather of the bf16 rows so every rank holds the whole output")
     ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm"], default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
                          "(for profiler captures; prints no result line)")
@@ -274,9 +277,11 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(spec, n):
+def config_dict(spec, n, context_parallel=False):
+    par = (f"cp{n} (the tokens split across GPUs, then an all-gather of the output rows)" if context_parallel
+           else f"dp{n} (independent token batches per GPU)")
     return {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "block": spec.block,
-            "parallelism": f"dp{n} (independent token batches per GPU)",
+            "parallelism": par,
             "l2": "inputs larger than L2: x and y are 415.6 MB each per step; the 28.9 MB packed weights "
                   "stay L2-resident across steps as they do when one layer serves many batches"}
 
@@ -406,6 +411,13 @@ def main():
         return run_mlp(args, rank, world)
     spec = workload(args)
     x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
+    job = spec  # the whole job's tokens
+    if args.context_parallel:
+        import dataclasses
+        from w8a8_int8_quantized_block_b200 import context_parallel as CP
+        lo, hi = CP.token_shard(spec.M, world, rank)
+        x_cpu = x_cpu[lo:hi].contiguous()
+        spec = dataclasses.replace(spec, M=hi - lo)  # this rank's shard: the per-kernel and end-to-end legs
     x = x_cpu.cuda()
     bias = b_cpu.cuda()
     pw = C.pack_weight(w_cpu.cuda(), spec.block)
@@ -419,8 +431,17 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    def step():
-        C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream)
+    if args.context_parallel:
+        y_full = torch.empty(job.M, job.N, dtype=torch.bfloat16, device="cuda")
+
+        def shard_linear(xs, out):
+            C.linear_fused(xs, pw, bias, workspace=ws, out=out, stream=stream)
+
+        def step():
+            CP.linear_context_parallel(x, job.M, job.N, shard_linear, out=y_full)
+    else:
+        def step():
+            C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream)
 
     if args.kernel_only:
         C.quantize_act(x, spec.block, q, s, stream=stream)
@@ -454,7 +475,10 @@ def main():
     st, code = C.last_device_status()
     if st != C.OK:
         raise RuntimeError(f"device status {st} (code {code}) after the timed region")
-    value = job_tops(spec.ops, args.steps, world, elapsed_s)
+    if args.context_parallel:
+        value = job.ops * args.steps / elapsed_s / 1e12  # strong scaling: the ranks share one job
+    else:
+        value = job_tops(spec.ops, args.steps, world, elapsed_s)
 
     # Per-kernel durations, same stream, CUDA events around each launch: the
     # one-kernel step (its ready-counter memset included), then the two
@@ -501,8 +525,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_s / args.steps * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": config_dict(spec, world),
+            "scaling": "strong" if args.context_parallel else "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "config": config_dict(job, world, args.context_parallel),
             "pct_of_int8_peak": round(100.0 * value / world / int8_peak, 2),
             "roofline": {"bound": "tensor",
                          "kernel": "linear_fused_kernel (rotate + quantise + int8 GEMM + dequant epilogue, one launch)",

@@ -81,3 +81,65 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_zero():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+
+
+# ------------------------------------------------------------ token-sharded linear with an all-gather
+
+
+def _cp_worker(rank: int, world: int, port: int, out, cases):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    from w8a8_int8_quantized_block_b200 import context_parallel as CP
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        res = []
+        for M, K, N in cases:
+            g = torch.Generator().manual_seed(M * 100 + N)
+            x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+            w = torch.randn(N, K, generator=g)
+
+            def linear(xs, y):  # a CPU stand-in for the GPU linear: same rows in, same rows out
+                y.copy_((xs.float() @ w.T).to(torch.bfloat16))
+
+            s, e = CP.token_shard(M, world, rank)
+            y = CP.linear_context_parallel(x[s:e].clone(), M, N, linear)
+            ref = (x.float() @ w.T).to(torch.bfloat16)
+            res.append(bool(torch.equal(y.view(torch.int16), ref.view(torch.int16))) and tuple(y.shape) == (M, N))
+        dist.barrier()
+        out.put((rank, res))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_token_shard_covers_every_row_once():
+    sys.path.insert(0, ROOT)
+    from w8a8_int8_quantized_block_b200 import context_parallel as CP
+
+    for M in (0, 1, 7, 8, 38656, 38657):
+        for world in (1, 2, 3, 8):
+            rows = []
+            for r in range(world):
+                s, e = CP.token_shard(M, world, r)
+                assert 0 <= s <= e <= M and e - s <= -(-M // world)
+                rows.extend(range(s, e))
+            assert rows == list(range(M))
+
+
+def test_context_parallel_gather_on_two_gloo_ranks():
+    # even and uneven token counts, and a rank whose shard is empty (M = 1)
+    cases = [(10, 16, 6), (11, 16, 6), (1, 8, 4), (300, 64, 24)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, 2, port, q, cases)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok in res:
+        assert all(ok), (rank, ok)
