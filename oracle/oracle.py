@@ -18,6 +18,10 @@ Every function cites the passage it follows (page title and section):
 * the activation prologue of the down projection ("SwiGLU + ConvRot64 +
   Rowwise INT8 Quantize" in MLP.fc2) -- MiniMax-H3-Rung-Omega README,
   "Technical Architecture Overview", item 2;
+* int8 attention ("sageattn_qk_int8_pv_fp16_cuda" in the Rung-Omega engine's
+  Floor 1 -- MiniMax-H3-Rung-Omega README, "Technical Architecture
+  Overview", item 2): Q and K quantised per token row to int8, P V in
+  16-bit floating point;
 * the regular rotation H_4^(x)k ("DC-balanced regular orthogonal Hadamard
   matrix H_256 = H_4^(x)4") -- MiniMax-H3-Rung-Omega README, "Technical
   Architecture Overview", item 1.
@@ -48,7 +52,7 @@ CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-s
 __all__ = [
     "build", "lib", "num_threads", "hadamard", "hadamard_sylvester", "hadamard_regular_kron", "fwht",
     "quantize_rows", "quantize_act", "act_f32", "act_quantize", "ACT_NONE", "ACT_GELU", "ACT_SWIGLU",
-    "pack_weight", "igemm", "igemm_pairs",
+    "pack_weight", "igemm", "igemm_pairs", "attention", "attention_rows",
     "dequant", "dequant_pairs", "linear", "rotate_explicit_f64",
     "bf16_bits", "bf16_bits_to_f32", "py_fwht_exact", "py_quantize_row_exact",
     "py_igemm",
@@ -306,6 +310,47 @@ def linear(x_bits: np.ndarray, w: np.ndarray, bias: np.ndarray | None, b: int, g
     return y, qx, sx, qw, sw, acc
 
 
+# ---------------------------------------------------------------- attention
+
+
+def _attention_head(qx, sq, kx, sk, v, scale):
+    """One head: S = (q . k) s_q s_k scale from exact int64 dot products,
+    P = softmax over the keys, O = P V, all in fp64."""
+    S = igemm(qx, kx).astype(np.float64) * sq.astype(np.float64)[:, None] * sk.astype(np.float64)[None, :] * scale
+    S -= S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P /= P.sum(axis=1, keepdims=True)
+    return P @ v
+
+
+def attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, scale: float | None = None):
+    """int8 attention: q, k, v bf16 bits [H, L, d] (k and v share their L).
+    Q and K are quantised per token row (the rowwise int8 quantiser, no
+    rotation); O = softmax(S) V with S = (q . k) s_q s_k * scale, scale
+    1/sqrt(d) unless given; returns O fp64 [H, Lq, d] and the codes and
+    scales (qx, sq, kx, sk)."""
+    H, Lq, d = q_bits.shape
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    qx, sq = quantize_act(q_bits.reshape(H * Lq, d), 0)
+    kx, sk = quantize_act(k_bits.reshape(-1, d), 0)
+    Lk = k_bits.shape[1]
+    qx, sq = qx.reshape(H, Lq, d), sq.reshape(H, Lq)
+    kx, sk = kx.reshape(H, Lk, d), sk.reshape(H, Lk)
+    v = bf16_bits_to_f32(v_bits).astype(np.float64)
+    O = np.stack([_attention_head(qx[h], sq[h], kx[h], sk[h], v[h], scale) for h in range(H)])
+    return O, (qx, sq, kx, sk)
+
+
+def attention_rows(qx, sq, kx, sk, v_bits, heads: np.ndarray, rows: np.ndarray, scale: float) -> np.ndarray:
+    """O for a sample of (head, query row) pairs, from given codes and scales
+    (qx [H, Lq, d], kx [H, Lk, d] int8; sq, sk f32): each row in full."""
+    out = np.empty((len(heads), qx.shape[2]), dtype=np.float64)
+    for t, (h, i) in enumerate(zip(heads, rows)):
+        v = bf16_bits_to_f32(v_bits[h]).astype(np.float64)
+        out[t] = _attention_head(qx[h, i:i + 1], sq[h, i:i + 1], kx[h], sk[h], v, scale)[0]
+    return out
+
+
 # ---------------------------------------------------------------- pure-Python references (tiny inputs)
 
 
@@ -370,3 +415,16 @@ def py_quantize_row_exact(z: list):
 def py_igemm(qa: list, qb: list) -> list:
     """Brute-force integer dot products in Python ints."""
     return [[sum(int(a) * int(b) for a, b in zip(ra, rb)) for rb in qb] for ra in qa]
+
+
+def py_attention_exact_scores(qx: list, sq: list, kx: list, sk: list, v: list, scale: float) -> list:
+    """One head by plain Python loops (math.exp), for tiny inputs."""
+    import math
+    out = []
+    for i in range(len(qx)):
+        s = [sum(a * b for a, b in zip(qx[i], kx[j])) * sq[i] * sk[j] * scale for j in range(len(kx))]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        t = sum(e)
+        out.append([sum(e[j] * v[j][c] for j in range(len(kx))) / t for c in range(len(v[0]))])
+    return out

@@ -483,3 +483,70 @@ def test_down_projection_with_prologue_matches_unquantised_product(act):
         y = O.dequant(O.igemm(qx, qw), sx, sw, None, b)
         ref = x @ w.T.astype(np.float64)
         assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.02
+
+
+# ------------------------------------------------------------ int8 attention (f3)
+
+
+def _qkv(H, Lq, Lk, d, seed, qs=1.0):
+    rng = np.random.default_rng(seed)
+    q = _bf16(rng.standard_normal((H * Lq, d)) * qs).reshape(H, Lq, d)
+    k = _bf16(rng.standard_normal((H * Lk, d))).reshape(H, Lk, d)
+    v = _bf16(rng.standard_normal((H * Lk, d))).reshape(H, Lk, d)
+    return q, k, v
+
+
+def test_attention_matches_plain_python_loops():
+    q, k, v = _qkv(1, 5, 7, 8, 31)
+    att, (qx, sq, kx, sk) = O.attention(q, k, v)
+    ref = O.py_attention_exact_scores(qx[0].astype(int).tolist(), sq[0].astype(float).tolist(),
+                                      kx[0].astype(int).tolist(), sk[0].astype(float).tolist(),
+                                      O.bf16_bits_to_f32(v[0]).astype(float).tolist(), 1.0 / np.sqrt(8))
+    assert np.allclose(att[0], np.array(ref), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_of_constant_values_is_that_constant():
+    # softmax rows sum to one: V = c everywhere gives O = c
+    q, k, _ = _qkv(2, 16, 24, 32, 32)
+    v = _bf16(np.full((2 * 24, 32), 0.625)).reshape(2, 24, 32)
+    att, _ = O.attention(q, k, v)
+    assert np.allclose(att, 0.625, rtol=0, atol=1e-14)
+
+
+def test_attention_of_zero_queries_is_the_mean_of_values():
+    # a zero query row has s_q = 0: every score is 0, P is uniform
+    q, k, v = _qkv(1, 4, 20, 16, 33)
+    q[:] = 0
+    att, _ = O.attention(q, k, v)
+    assert np.allclose(att[0], O.bf16_bits_to_f32(v[0]).astype(np.float64).mean(axis=0), atol=1e-14)
+
+
+def test_attention_is_invariant_to_a_joint_permutation_of_keys_and_values():
+    q, k, v = _qkv(1, 8, 40, 16, 34)
+    perm = np.random.default_rng(0).permutation(40)
+    a1, _ = O.attention(q, k, v)
+    a2, _ = O.attention(q, k[:, perm], v[:, perm])
+    assert np.allclose(a1, a2, rtol=1e-12, atol=1e-14)
+
+
+def test_attention_picks_out_a_dominant_key():
+    # query and one key along the same axis with a large scale: the softmax
+    # puts almost all weight on that key
+    d = 16
+    q = np.zeros((1, 2, d)); q[0, :, 0] = 16.0
+    k = np.random.default_rng(35).standard_normal((1, 10, d)) * 0.1
+    k[0, 6, :] = 0.0; k[0, 6, 0] = 16.0  # score 16 * 16 / sqrt(16) = 64 against ~0.3
+    v = np.random.default_rng(36).standard_normal((1, 10, d))
+    att, _ = O.attention(_bf16(q.reshape(2, d)).reshape(1, 2, d), _bf16(k.reshape(10, d)).reshape(1, 10, d),
+                       _bf16(v.reshape(10, d)).reshape(1, 10, d))
+    v6 = O.bf16_bits_to_f32(_bf16(v[0, 6:7]))[0]
+    assert np.abs(att[0] - v6).max() < 1e-12
+
+
+def test_attention_scores_are_the_dequantised_qk_product():
+    # S is the config-5 skinny-K GEMM's output (before bf16) times the scale
+    q, k, v = _qkv(1, 6, 9, 128, 37)
+    a1, (qx, sq, kx, sk) = O.attention(q, k, v, scale=0.5)
+    S = O.dequant(O.igemm(qx[0], kx[0]), sq[0], sk[0], None, 0) * 0.5
+    P = np.exp(S - S.max(1, keepdims=True)); P /= P.sum(1, keepdims=True)
+    assert np.allclose(a1[0], P @ O.bf16_bits_to_f32(v[0]).astype(np.float64), rtol=1e-12, atol=1e-14)
