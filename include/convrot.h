@@ -172,6 +172,32 @@ convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int
                                   const float* s_w, const convrot_wdesc* desc, const float* bias, int32_t epilogue,
                                   void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy, void* stream);
 
+/* int8 attention without materialising the scores ("sageattn_qk_int8_pv_fp16_cuda"
+ * in the Rung-Omega engine's Floor 1 -- MiniMax-H3-Rung-Omega README,
+ * "Technical Architecture Overview", item 2: int8 Q K^T, 16-bit P V).  The
+ * pages give no formula; the reading here, per head h and query row i:
+ *   S_ij = (q_i . k_j) * s_q[i] * s_k[j] * scale,  O_i = sum_j softmax_j(S_i.) v_j
+ * with q, k the rows of Q and K quantised by the rowwise int8 quantiser (no
+ * rotation), v the bf16 rows of V, P rounded to bf16 for the P V product,
+ * f32 accumulation, O stored as bf16.  No mask.  Head dimension 128.
+ *
+ * convrot_attention: q [H][Lq][128], k and v [H][Lk][128], bf16, contiguous;
+ * o [H][Lq][128] bf16 (32-byte aligned).  Lq and Lk multiples of 128, scale > 0
+ * (1/sqrt(128) for the usual softmax scale).  `workspace` (256-byte aligned,
+ * >= convrot_attention_workspace_bytes(H, Lq, Lk)) receives the Q and K codes
+ * and scales and V^T.  Four kernels on `stream`. */
+size_t convrot_attention_workspace_bytes(int64_t H, int64_t Lq, int64_t Lk);
+convrot_status convrot_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t H, int64_t Lq,
+                                 int64_t Lk, float scale, void* workspace, size_t ws_bytes, uint16_t* o,
+                                 void* stream);
+
+/* The attention kernel alone, on quantised inputs: qx int8 [H][Lq][128] and
+ * s_q f32 [H][Lq]; kx int8 [H][Lk][128] and s_k f32 [H][Lk] (16-byte
+ * aligned); vt = V^T, bf16 [H][128][Lk]; o as above. */
+convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const int8_t* kx, const float* s_k,
+                                      const uint16_t* vt, int64_t H, int64_t Lq, int64_t Lk, float scale,
+                                      uint16_t* o, void* stream);
+
 /* End-to-end form of convrot_linear_fused for callers whose activations live
  * in host memory: copies x_host (bf16 [M][K], contiguous; pinned for overlap)
  * into the caller's device buffer x_dev, runs the fused linear into y_dev

@@ -40,6 +40,7 @@ EXPORTS = (
     "convrot_w8a8_linear", "convrot_workspace_bytes", "convrot_linear_fused", "convrot_linear_fused_host",
     "convrot_w8a8_bmm", "convrot_igemm_s32", "convrot_last_device_status", "convrot_set_wait_limit_ns",
     "convrot_selftest_wait_timeout", "convrot_linear_fused_noalloc", "convrot_act_quantize", "convrot_linear_act",
+    "convrot_attention_workspace_bytes", "convrot_attention", "convrot_attention_int8",
 )
 
 
@@ -93,6 +94,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "convrot_linear_fused_noalloc": ([P, I64, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, I64, P],
                                          ctypes.c_int),
         "convrot_act_quantize": ([P, I64, I64, I64, I32, I32, P, P, P], ctypes.c_int),
+        "convrot_attention_workspace_bytes": ([I64, I64, I64], ctypes.c_size_t),
+        "convrot_attention": ([P, P, P, I64, I64, I64, ctypes.c_float, P, ctypes.c_size_t, P, P], ctypes.c_int),
+        "convrot_attention_int8": ([P, P, P, P, P, I64, I64, I64, ctypes.c_float, P, P], ctypes.c_int),
         "convrot_linear_act": ([P, I64, I64, I32, P, P, ctypes.POINTER(WDesc), P, I32, P, ctypes.c_size_t, P, I64,
                                 P], ctypes.c_int),
     }
@@ -208,6 +212,40 @@ def linear_act(h: torch.Tensor, act: int, pw: PackedWeight, bias: torch.Tensor |
         _ptr(h), M, h.stride(0), act, _ptr(pw.q), _ptr(pw.s), ctypes.byref(pw.desc), _ptr(bias),
         EPI_GELU if gelu else EPI_NONE, _ptr(ws), ws.numel(), _ptr(y), y.stride(0), _stream(stream)))
     return y
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+              workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """int8 attention: q [H, Lq, 128], k and v [H, Lk, 128] bf16 -> O [H, Lq, 128]
+    bf16 (scale defaults to 1/sqrt(128))."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    H, Lq, d = q.shape
+    Lk = k.shape[1]
+    if d != 128 or tuple(k.shape) != (H, Lk, d) or tuple(v.shape) != (H, Lk, d):
+        raise ValueError("q [H, Lq, 128], k and v [H, Lk, 128]")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    L = load()
+    if workspace is None:
+        workspace = torch.empty((L.convrot_attention_workspace_bytes(H, Lq, Lk),), dtype=torch.uint8, device=q.device)
+    o = torch.empty((H, Lq, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    _check("convrot_attention", L.convrot_attention(_ptr(q), _ptr(k), _ptr(v), H, Lq, Lk,
+                                                    (d ** -0.5) if scale is None else scale, _ptr(workspace),
+                                                    workspace.numel(), _ptr(o), _stream(stream)))
+    return o
+
+
+def attention_int8(qx, sq, kx, sk, vt, scale: float | None = None, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """The attention kernel on quantised inputs: qx [H, Lq, 128] int8, sq [H, Lq],
+    kx [H, Lk, 128] int8, sk [H, Lk], vt = V^T [H, 128, Lk] bf16."""
+    H, Lq, d = qx.shape
+    Lk = kx.shape[1]
+    o = torch.empty((H, Lq, d), dtype=torch.bfloat16, device=qx.device) if out is None else out
+    _check("convrot_attention_int8", load().convrot_attention_int8(
+        _ptr(qx), _ptr(sq), _ptr(kx), _ptr(sk), _ptr(vt), H, Lq, Lk, (d ** -0.5) if scale is None else scale,
+        _ptr(o), _stream(stream)))
+    return o
 
 
 def w8a8_linear(qx: torch.Tensor, sx: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None,
