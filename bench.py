@@ -71,9 +71,10 @@ def parse():
     ap.add_argument("--block", choices=sorted(BLOCK_CHOICES), default="128",
                     help="rotation of the step: Sylvester H_b (64, 128, 256) or the regular H_4^(x)k "
                          "(reg16, reg64, reg256); the headline is 128")
-    ap.add_argument("--workload", choices=["proj", "mlp"], default="proj",
+    ap.add_argument("--workload", choices=["proj", "mlp", "attention"], default="proj",
                     help="proj: the 768p projection (the headline); mlp: the 768p MLP, up 5376 -> 21504 with "
-                         "GELU, then down, timed by both routes of the activation (see --mlp-route)")
+                         "GELU, then down, timed by both routes of the activation (see --mlp-route); "
+                         "attention: int8 attention over 42 heads of 8192 tokens, head dim 128")
     ap.add_argument("--mlp-route", choices=["prologue", "epilogue"], default="prologue",
                     help="the route the mlp line's value is for: GELU as the down projection's prologue "
                          "(convrot_linear_act) or in the up projection's epilogue; both are timed")
@@ -289,6 +290,102 @@ def config_dict(spec, n, context_parallel=False):
 # ---------------------------------------------------------------------------- GPU path
 
 
+ATTN_METRIC = "int8 attention TFLOP/s at 42 heads x 8192 tokens, d=128 (Q K^T int8 + P V bf16)"
+
+
+def run_attention(args, rank: int, world: int):
+    """int8 attention on the 42-head, 8192-token workload: the whole entry
+    (quantise Q and K, transpose V, attend) and the attention kernel alone.
+    Work = 2 H L^2 d int8 ops (Q K^T) + 2 H L^2 d bf16 flops (P V)."""
+    import torch
+    import torch.distributed as dist
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+
+    spec = W.QK_BMM
+    H, L, d = spec.batch, spec.M, spec.K
+    q_cpu, k_cpu = W.bmm_inputs(spec)
+    v_cpu = torch.randn(H, L, d, generator=torch.Generator().manual_seed(44)).to(torch.bfloat16)
+    q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
+    Lib = C.load()
+    ws = torch.empty((Lib.convrot_attention_workspace_bytes(H, L, L),), dtype=torch.uint8, device="cuda")
+    o = torch.empty(H, L, d, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    r256 = lambda n: (n + 255) // 256 * 256
+    off_sq = r256(H * L * d)
+    off_kx = off_sq + r256(H * L * 4)
+    off_sk = off_kx + r256(H * L * d)
+    off_vt = off_sk + r256(H * L * 4)
+    qx, sq = ws[:H * L * d].view(torch.int8).view(H, L, d), ws[off_sq:off_sq + H * L * 4].view(torch.float32)
+    kx, sk = ws[off_kx:off_kx + H * L * d].view(torch.int8).view(H, L, d), ws[off_sk:off_sk + H * L * 4].view(
+        torch.float32)
+    vt = ws[off_vt:off_vt + H * d * L * 2].view(torch.bfloat16).view(H, d, L)
+
+    def full():
+        C.attention(q, k, v, workspace=ws, out=o, stream=stream)
+
+    def kernel():
+        C.attention_int8(qx, sq, kx, sk, vt, out=o, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        full()
+    barrier()
+    times = {}
+    clk_summary = None
+    for name, fn in (("kernel", kernel), ("full", full)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            barrier()
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            barrier()
+        times[name] = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / args.steps
+        if name == "kernel":
+            clk_summary = clk.summary()
+    st, code = C.last_device_status()
+    if st != C.OK:
+        raise RuntimeError(f"device status {st} (code {code})")
+    if rank == 0:
+        hbm, bf16, kind = peaks()
+        int8_peak = bf16 * INT8_PER_BF16
+        half = 2.0 * H * L * L * d          # each of the two products
+        ops = 2 * half
+        t_tensor = half / (int8_peak * 1e12) + half / (bf16 * 1e12)   # both products at their peaks
+        mufu = 16 * 148 * 1.965e9                                      # 2^x per second (SFU, nominal)
+        t_exp = H * L * L / mufu
+        value = world * ops / times["full"] / 1e12
+        line = {
+            "metric": ATTN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": times["full"] * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
+            "config": {"workload": "attention_h42_l8192_d128", "heads": H, "Lq": L, "Lk": L, "d": d,
+                       "parallelism": f"dp{world} (independent heads and sequences per GPU)",
+                       "l2": "inputs larger than L2: Q, K, V are 88 MB each, O 88 MB; the score matrix (11.3 GB "
+                             "as bf16) is never stored"},
+            "roofline": {"bound": "tensor", "kernel": "attention_kernel (Q K^T, softmax, P V; one launch)",
+                         "achieved": ops / times["kernel"] / 1e12, "peak": ops / t_tensor / 1e12,
+                         "unit": "TFLOP/s", "frac": t_tensor / times["kernel"], "traffic": None,
+                         "peak_source": f"{kind}: Q K^T at bf16 burst x {INT8_PER_BF16}, P V at the bf16 burst "
+                                        f"{bf16} TFLOP/s; the 2^x of the softmax alone would take "
+                                        f"{t_exp * 1e3:.3f} ms on the special-function units (nominal 16/clk/SM)"},
+            "kernels": {"attention_kernel_us": times["kernel"] * 1e6,
+                        "quantise_transpose_us": (times["full"] - times["kernel"]) * 1e6},
+            "clocks": clk_summary,
+            "gpu_launches": 4 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 MLP_METRIC = "ConvRot W8A8 MLP TOPS at M=38656, K=5376, H=21504 (up + GELU + down)"
 
 
@@ -407,6 +504,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+    if args.workload == "attention":
+        return run_attention(args, rank, world)
     if args.workload == "mlp":
         return run_mlp(args, rank, world)
     spec = workload(args)

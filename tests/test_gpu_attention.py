@@ -56,7 +56,7 @@ def _check_codes(ws, q, k):
     assert np.array_equal(kx, kr) and np.array_equal(sk.view(np.uint32), skr.view(np.uint32))
 
 
-@pytest.mark.parametrize("H,Lq,Lk", [(2, 256, 384), (1, 128, 128), (3, 128, 1024)])
+@pytest.mark.parametrize("H,Lq,Lk", [(2, 256, 384), (1, 128, 128), (3, 128, 1024), (2, 640, 256), (1, 384, 512)])
 def test_attention_matches_oracle(H, Lq, Lk):
     q, k, v = _qkv(H, Lq, Lk, seed=H * 1000 + Lq + Lk)
     o, ws = _run(q, k, v)

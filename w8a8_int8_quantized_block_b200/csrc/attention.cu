@@ -12,25 +12,33 @@
 // rescaled by 2^(m_old - m_new) whenever m grows), so S only ever lives one
 // 128 x 128 tile at a time in tensor memory.
 //
-// One CTA per (head, 128-query tile), 192 threads:
-//   warp 0     TMA producer: the Q tile once, then for each 128-key tile its
-//              K codes, the two halves of V^T and the 128 key scales into one
-//              of two ring stages
-//   warp 1     TMEM owner and MMA issuer (one thread):
-//                S_b = Q K_j^T      kind::i8, M = N = 128, 4 MMAs of K = 32,
-//                                   into S buffer b = j % 2 (TMEM columns 128 b)
-//                O  += P_j V_j      kind::f16 (bf16 in, f32 accumulate),
-//                                   8 MMAs of K = 16, into TMEM columns 256..383
-//              QK_{j+1} is issued before P V_j, so the next scores are being
-//              computed while the softmax works on this tile.
-//   warps 2-5  softmax, one thread per query row (TMEM lane quadrant =
-//              warp % 4): scores from TMEM into registers, scaled to log2
-//              units, the row maximum, p = 2^(x - m) on the special-function
-//              unit, p rounded to bf16 into the P buffer (128-byte swizzle,
-//              the A operand's canonical K-major layout), the row sum; then,
-//              once P V_{j-1} is done, O *= 2^(m_old - m_new) in TMEM (skipped
-//              when no row of the warp changed its maximum); finally O / l,
-//              bf16, to global memory.
+// One CTA per (head, pair of 128-query tiles A and B), 320 threads:
+//   warp 0     TMA producer: the two Q tiles once, then for each 128-key tile
+//              its K codes, the two halves of V^T and the 128 key scales into
+//              one of two ring stages (shared by both query tiles)
+//   warp 1     TMEM owner and MMA issuer (one thread), per key tile j and
+//              query tile t = A, B in turn:
+//                S_t = Q_t K_{j+1}^T  kind::i8, M = N = 128, 4 MMAs of K = 32
+//                O_t += P_t V_j       kind::f16 (bf16 in, f32 accumulate), 8
+//                                     MMAs of K = 16
+//              TMEM holds S_A, O_A, S_B, O_B (128 columns each).  The next
+//              scores of a tile are issued before its P V, and the tensor
+//              cores work on one query tile while the softmax works on the
+//              other.  (One issuer serving both tiles in turn measured faster
+//              than one issuer per tile: 1.90 vs 2.01 ms on 42 heads of 8192.)
+//   warps 2-9  softmax, four warps per query tile, one thread per query row
+//              (TMEM lane quadrant = warp % 4).  The score buffers are seeded
+//              so that the int8 MMAs leave float bits behind (see kScoreSeed).
+//              Pass 1 reads the scores from TMEM for the row maximum (packed
+//              f32x2 arithmetic, three-input max); pass 2 reads them again,
+//              p = 2^(x - m) on the special-function unit, p rounded to bf16
+//              into the tile's P buffer (128-byte swizzle, the A operand's
+//              canonical K-major layout), the row sum.  Then O *=
+//              2^(m_old - m_new) in TMEM (the reference maximum moves only
+//              when a row's scores exceed it by more than 8 in log2 units, and
+//              the rescale is skipped when no row of the warp moved); finally
+//              O / l, bf16, to global memory.
+// Two softmax warps per SM sub-partition hide each other's latencies.
 // Every wait is bounded (a time-out records kErrTimeoutAttn and the CTA
 // unwinds).  V arrives as V^T [h][d][key] (K-major for the P V product),
 // written by transpose_kernel below.
@@ -46,8 +54,9 @@ namespace convrot {
 namespace {
 
 constexpr int kD = 128;        // head dimension
-constexpr int kTile = 128;     // queries per CTA and keys per tile
-constexpr int kThreadsA = 192;
+constexpr int kTile = 128;     // queries per tile and keys per tile
+constexpr int kQTiles = 2;     // query tiles per CTA
+constexpr int kThreadsA = (2 + 4 * kQTiles) * 32;
 constexpr int kQBytes = kTile * kD;           // int8 Q tile: 16 KB
 constexpr int kKBytes = kTile * kD;           // int8 K tile: 16 KB
 constexpr int kAtomBytes = 128 * 128;         // one 128-row x 128-byte swizzle column: 16 KB
@@ -56,16 +65,16 @@ constexpr int kPBytes = 2 * kAtomBytes;       // P tile (128 queries x 128 keys 
 constexpr int kSkBytes = kTile * 4;           // the tile's key scales
 constexpr int kStages = 2;
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffK = kOffQ + kQTiles * kQBytes;
 constexpr int kOffV = kOffK + kStages * kKBytes;
 constexpr int kOffP = kOffV + kStages * kVBytes;
-constexpr int kOffSk = kOffP + 2 * kPBytes;
+constexpr int kOffSk = kOffP + kQTiles * kPBytes;
 constexpr int kOffBar = kOffSk + kStages * kSkBytes;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2;
+constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles;
 constexpr int kSmemA = kOffBar + kNumBars * 8 + 16 + 1024;  // + TMEM slot, + 1024-byte alignment slack
 static_assert(kSmemA <= 227 * 1024, "shared memory budget");
-constexpr uint32_t kTmemColsA = 512;          // S0, S1, O (384 used)
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kTmemColsA = 512;          // per query tile: S (128 columns), O (128 columns)
+constexpr float kRescaleLog2 = 8.0f;          // the running maximum moves only by more than this
 
 struct AttnArgs {
     int H, Lq, Lk;
@@ -77,16 +86,52 @@ struct AttnArgs {
     unsigned int* err;
 };
 
-__device__ __forceinline__ float int_to_float_exact(uint32_t s) {
-    // |s| < 2^22 (|q . k| <= 127^2 * 128): adding 1.5 * 2^23 in the integer
-    // domain puts s in the mantissa of a float near 2^23 + 2^22, exactly.
-    return __uint_as_float(s + 0x4B400000u) - 12582912.0f;
+// Each score buffer starts every tile at the integer 0x4B400000 = the bits of
+// the float 1.5 * 2^23, and the int8 MMAs accumulate onto it: since
+// |q . k| <= 127^2 * 128 < 2^22, the int32 result is exactly the bits of the
+// float 1.5 * 2^23 + (q . k).  So x = fma(bits, s_k, -fl(1.5 * 2^23 * s_k))
+// is float(q . k) * s_k up to the rounding of fl(1.5 * 2^23 * s_k), at most
+// one unit of q . k times s_k (about 3e-5 of p's relative size at the usual
+// scales, far below p's bf16 rounding of 2^-9).
+constexpr uint32_t kScoreSeed = 0x4B400000u;
+constexpr float kSeedValue = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk2(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&v);
 }
+
+__device__ __forceinline__ uint32_t col_s(int t) { return static_cast<uint32_t>(t * 2 * kTile); }
+__device__ __forceinline__ uint32_t col_o(int t) { return static_cast<uint32_t>(t * 2 * kTile + kTile); }
 
 __global__ void __launch_bounds__(kThreadsA, 1)
     attention_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -100,19 +145,20 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     float* sSk = reinterpret_cast<float*>(smem + kOffSk);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;             // [2]
-    uint64_t* kv_empty = kv_full + kStages;   // [2]
-    uint64_t* s_full = kv_empty + kStages;    // [2]
-    uint64_t* s_free = s_full + 2;            // [2]
-    uint64_t* p_ready = s_free + 2;           // [2]
-    uint64_t* pv_done = p_ready + 2;          // [2]
+    uint64_t* kv_full = bars + 1;             // [stage]
+    uint64_t* kv_empty = kv_full + kStages;   // [stage]
+    uint64_t* s_full = kv_empty + kStages;    // [query tile]
+    uint64_t* s_free = s_full + kQTiles;      // [query tile]
+    uint64_t* p_ready = s_free + kQTiles;     // [query tile]
+    uint64_t* pv_done = p_ready + kQTiles;    // [query tile]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int q_tiles = a.Lq / kTile;
-    const int h = blockIdx.x / q_tiles;
-    const int q0 = (blockIdx.x - h * q_tiles) * kTile;
+    const int pairs = (a.Lq / kTile + kQTiles - 1) / kQTiles;
+    const int h = blockIdx.x / pairs;
+    const int q0 = (blockIdx.x - h * pairs) * kQTiles * kTile;
+    const int nq = min(kQTiles, (a.Lq - q0) / kTile);  // 1 when Lq / 128 is odd and this is the last pair
     const int T = a.Lk / kTile;  // key tiles
 
     if (threadIdx.x == 0) {
@@ -122,13 +168,13 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         mbar_init(q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&kv_empty[s], nq);  // one commit per query tile's P V
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&s_free[b], 4);   // one arrival per softmax warp
-            mbar_init(&p_ready[b], 4);
-            mbar_init(&pv_done[b], 1);
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&s_free[t], 4);   // one arrival per softmax warp of the tile
+            mbar_init(&p_ready[t], 4);
+            mbar_init(&pv_done[t], 1);
         }
         fence_mbar_init();
     }
@@ -147,8 +193,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         if (lane == 0) {
             // ---------------------------------------------------------- producer
             bool ok = true;
-            mbar_arrive_expect_tx(q_full, kQBytes);
-            tma_load_3d(sQ, &qmap, q_full, 0, q0, h);
+            mbar_arrive_expect_tx(q_full, nq * kQBytes);
+            for (int t = 0; t < nq; ++t) tma_load_3d(sQ + t * kQBytes, &qmap, q_full, 0, q0 + t * kTile, h);
             for (int j = 0; j < T && ok; ++j) {
                 const int st = j % kStages;
                 if (!mbar_wait_bounded(&kv_empty[st], ((j / kStages) & 1) ^ 1u, a.limit_ns, kErrTimeoutAttn,
@@ -167,166 +213,212 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ---------------------------------------------------------- MMA issuer
+            // ---------------------------------------------------------- MMA issuer (both tiles)
             constexpr uint32_t idesc_qk = umma_idesc_i8(kTile, kTile);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kTile, kD);
-            bool ok = mbar_wait_bounded(q_full, 0, a.limit_ns, kErrTimeoutAttn, a.err);
-            const uint32_t q_addr = smem_u32(sQ);
-            auto issue_pv = [&](int i) -> bool {
-                const int pb = i & 1;
-                if (!mbar_wait_bounded(&p_ready[pb], (i >> 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err)) return false;
-                tc_fence_after_sync();
-                const uint32_t p_addr = smem_u32(sP + pb * kPBytes);
-                const uint32_t v_addr = smem_u32(sV + (i % kStages) * kVBytes);
+            auto issue_qk = [&](int t, int j) {
+                const uint32_t q_addr = smem_u32(sQ + t * kQBytes);
+                const uint32_t k_addr = smem_u32(sK + (j % kStages) * kKBytes);
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {  // K = 16 keys per MMA
-                    const uint32_t off = static_cast<uint32_t>((kk >> 2) * kAtomBytes + (kk & 3) * 32);
-                    mma_bf16(tmem + kColO, umma_desc_sw128_kmajor(p_addr + off), umma_desc_sw128_kmajor(v_addr + off),
-                             idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&pv_done[pb]);
-                mma_commit(&kv_empty[i % kStages]);
-                return true;
+                for (int k = 0; k < kD / 32; ++k)
+                    mma_i8(tmem + col_s(t), umma_desc_sw128_kmajor(q_addr + k * 32),
+                           umma_desc_sw128_kmajor(k_addr + k * 32), idesc_qk, 1u);
+                mma_commit(&s_full[t]);
             };
-            for (int j = 0; j < T && ok; ++j) {
-                const int st = j % kStages;
-                const int b = j & 1;
-                if (!mbar_wait_bounded(&kv_full[st], (j / kStages) & 1, a.limit_ns, kErrTimeoutAttn, a.err)) {
-                    ok = false;
-                    break;
-                }
-                if (j >= 2 && !mbar_wait_bounded(&s_free[b], ((j - 2) >> 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t k_addr = smem_u32(sK + st * kKBytes);
+            auto issue_pv = [&](int t, int j) {
+                const uint32_t p_addr = smem_u32(sP + t * kPBytes);
+                const uint32_t v_addr = smem_u32(sV + (j % kStages) * kVBytes);
 #pragma unroll
-                for (int k = 0; k < kD / 32; ++k)  // K = 32 int8 per MMA
-                    mma_i8(tmem + static_cast<uint32_t>(b * kTile), umma_desc_sw128_kmajor(q_addr + k * 32),
-                           umma_desc_sw128_kmajor(k_addr + k * 32), idesc_qk, k > 0 ? 1u : 0u);
-                mma_commit(&s_full[b]);
-                if (j >= 1 && !issue_pv(j - 1)) {
-                    ok = false;
-                    break;
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    const uint32_t off = static_cast<uint32_t>((kk >> 2) * kAtomBytes + (kk & 3) * 32);
+                    mma_bf16(tmem + col_o(t), umma_desc_sw128_kmajor(p_addr + off),
+                             umma_desc_sw128_kmajor(v_addr + off), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&pv_done[t]);
+                mma_commit(&kv_empty[j % kStages]);
+            };
+            bool ok = mbar_wait_bounded(q_full, 0, a.limit_ns, kErrTimeoutAttn, a.err) &&
+                      mbar_wait_bounded(&kv_full[0], 0, a.limit_ns, kErrTimeoutAttn, a.err);
+            for (int t = 0; t < nq && ok; ++t) {
+                ok = mbar_wait_bounded(&s_free[t], 0, a.limit_ns, kErrTimeoutAttn, a.err);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_qk(t, 0);
                 }
             }
-            if (ok) issue_pv(T - 1);
+            for (int j = 0; j < T && ok; ++j) {
+                if (j + 1 < T)
+                    ok = mbar_wait_bounded(&kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, a.limit_ns,
+                                           kErrTimeoutAttn, a.err);
+                for (int t = 0; t < nq && ok; ++t) {
+                    if (j + 1 < T) {
+                        ok = mbar_wait_bounded(&s_free[t], (j + 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
+                        if (!ok) break;
+                        tc_fence_after_sync();
+                        issue_qk(t, j + 1);
+                    }
+                    ok = mbar_wait_bounded(&p_ready[t], j & 1, a.limit_ns, kErrTimeoutAttn, a.err);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_pv(t, j);
+                }
+            }
         }
     } else {
-        // -------------------------------------------------------------- softmax (warps 2..5)
+        // -------------------------------------------------------------- softmax (warps 2..9)
+        const int t = (warp - 2) >> 2;     // query tile
         const int quad = warp & 3;
         const int row = quad * 32 + lane;  // query row within the tile
-        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        const float rs = a.s_q[static_cast<int64_t>(h) * a.Lq + q0 + row] * a.scale_log2;
-        float m = -INFINITY, l = 0.0f;
-        bool ok = true;
-        for (int j = 0; j < T; ++j) {
-            const int b = j & 1;
-            const int st = j % kStages;
-            // the stage's key scales (bulk copy) and the tile's scores
-            ok = mbar_wait_bounded(&kv_full[st], (j / kStages) & 1, a.limit_ns, kErrTimeoutAttn, a.err) &&
-                 mbar_wait_bounded(&s_full[b], (j >> 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (!ok) break;
-            tc_fence_after_sync();
-            // the tile's scores, scaled to log2 units: x = float(q.k) * s_k[c] * s_q * scale * log2(e)
-            const float* cs = sSk + st * kTile;
-            float x[kTile];
-            float mx = -INFINITY;
+        if (t < nq) {
+            const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+            const uint32_t ts = tmem + lane_base + col_s(t);
+            const uint32_t to = tmem + lane_base + col_o(t);
+            const float rs = a.s_q[static_cast<int64_t>(h) * a.Lq + q0 + t * kTile + row] * a.scale_log2;
+            const uint64_t rs2 = pk2(rs, rs);
+            const uint64_t neg_seed2 = pk2(-kSeedValue, -kSeedValue);
+            uint8_t* prow = sP + t * kPBytes + row * 128;
+            uint32_t seed[32];
 #pragma unroll
-            for (int c4 = 0; c4 < kTile / 32; ++c4) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + static_cast<uint32_t>(b * kTile + c4 * 32), r);
-                tmem_ld_wait();
+            for (int e = 0; e < 32; ++e) seed[e] = kScoreSeed;
+            auto seed_scores = [&]() {
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const float v = int_to_float_exact(r[t]) * cs[c4 * 32 + t] * rs;
-                    x[c4 * 32 + t] = v;
-                    mx = fmaxf(mx, v);
-                }
-            }
-            // S_b has been read: QK_{j+2} may overwrite it
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[b]);
-
-            const float m_new = fmaxf(m, mx);
-            const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf)
-            // P buffer b is free once P V_{j-2} is done
-            if (j >= 2) {
-                ok = mbar_wait_bounded(&pv_done[b], ((j - 2) >> 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
-                ok = __all_sync(0xFFFFFFFFu, ok);
-                if (!ok) break;
-            }
-            uint8_t* prow = sP + b * kPBytes + row * 128;
-            float sum = 0.0f;
-#pragma unroll
-            for (int c8 = 0; c8 < kTile / 8; ++c8) {  // 8 keys = one 16-byte chunk
-                float p[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    p[e] = ex2_approx(x[c8 * 8 + e] - m_new);
-                    sum += p[e];
-                }
-                const uint4 w = make_uint4(pack2_bf16(p[0], p[1]), pack2_bf16(p[2], p[3]), pack2_bf16(p[4], p[5]),
-                                           pack2_bf16(p[6], p[7]));
-                const int atom = c8 >> 3, chunk = c8 & 7;
-                *reinterpret_cast<uint4*>(prow + atom * kAtomBytes + ((chunk ^ (row & 7)) << 4)) = w;
-            }
-            l = l * alpha + sum;
-            m = m_new;
-            // O *= alpha once P V_{j-1} is done (O holds nothing before P V_0)
-            if (j >= 1) {
-                ok = mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
+                for (int c4 = 0; c4 < kTile / 32; ++c4) tmem_st_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), seed);
+                tmem_st_wait();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[t]);
+            };
+            seed_scores();  // before the first tile's scores
+            float m = -INFINITY, l = 0.0f;
+            bool ok = true;
+            for (int j = 0; j < T; ++j) {
+                const int st = j % kStages;
+                // the stage's key scales (bulk copy) and the tile's scores
+                ok = mbar_wait_bounded(&kv_full[st], (j / kStages) & 1, a.limit_ns, kErrTimeoutAttn, a.err) &&
+                     mbar_wait_bounded(&s_full[t], j & 1, a.limit_ns, kErrTimeoutAttn, a.err);
                 ok = __all_sync(0xFFFFFFFFu, ok);
                 if (!ok) break;
                 tc_fence_after_sync();
-                if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+                const float4* cs4 = reinterpret_cast<const float4*>(sSk + st * kTile);
+                // pass 1 (single-load variant)
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c4 = 0; c4 < kTile / 32; ++c4) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 c = cs4[c4 * 8 + q];
+                        const uint64_t ca = pk2(c.x, c.y), cb = pk2(c.z, c.w);
+                        float x0, x1, x2, x3;
+                        upk2(fma2(pk2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), ca,
+                                  mul2(ca, neg_seed2)), x0, x1);
+                        upk2(fma2(pk2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), cb,
+                                  mul2(cb, neg_seed2)), x2, x3);
+                        mx = max3(mx, max3(x0, x1, x2), x3);
+                    }
+                }
+                mx *= rs;
+                // The softmax is exact for any reference m (O / l cancels it); m
+                // only has to keep 2^(x - m) in range.  So m moves only when the
+                // tile's maximum exceeds it by more than 8 (p <= 2^8 otherwise,
+                // fine in bf16 and f32), which skips most rescales of O.
+                const float m_new = (mx > m + kRescaleLog2) ? mx : m;
+                const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf), 1 when m stays
+                const uint64_t nm2 = pk2(-m_new, -m_new);
+                // P_t is free, and O_t complete, once P V of tile j - 1 is done
+                if (j >= 1) {
+                    ok = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
+                    ok = __all_sync(0xFFFFFFFFu, ok);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                }
+                // pass 2 (single-load variant)
+                uint64_t sum2 = pk2(0.0f, 0.0f);
+#pragma unroll
+                for (int c4 = 0; c4 < kTile / 32; ++c4) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int hq = 0; hq < 2; ++hq) {
+                            const float4 c = cs4[c4 * 8 + c8 * 2 + hq];
+                            const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                            for (int pr = 0; pr < 2; ++pr) {
+                                const int e = c8 * 8 + hq * 4 + pr * 2;
+                                const uint64_t c2 = pk2(cc[2 * pr], cc[2 * pr + 1]);
+                                const uint64_t x2 = fma2(pk2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2,
+                                                         mul2(c2, neg_seed2));
+                                float y0, y1;
+                                upk2(fma2(x2, rs2, nm2), y0, y1);
+                                const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+                                sum2 = add2(sum2, pk2(p0, p1));
+                                w[hq * 2 + pr] = pack2_bf16(p0, p1);
+                            }
+                        }
+                        const int chunk16 = c4 * 4 + c8;
+                        const int atom = chunk16 >> 3, chunk = chunk16 & 7;
+                        *reinterpret_cast<uint4*>(prow + atom * kAtomBytes + ((chunk ^ (row & 7)) << 4)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+                // S_t has been read for the last time: seed it for the next scores
+                if (j + 1 < T) seed_scores();
+                float s0, s1;
+                upk2(sum2, s0, s1);
+                l = l * alpha + (s0 + s1);
+                m = m_new;
+                // O *= alpha (O holds nothing before the first P V)
+                if (j >= 1 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
 #pragma unroll
                     for (int c4 = 0; c4 < kD / 32; ++c4) {
                         uint32_t r[32];
-                        const uint32_t taddr = tmem + lane_base + kColO + static_cast<uint32_t>(c4 * 32);
+                        const uint32_t taddr = to + static_cast<uint32_t>(c4 * 32);
                         tmem_ld_32x32b_x32(taddr, r);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(__uint_as_float(r[t]) * alpha);
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
                         tmem_st_32x32b_x32(taddr, r);
                     }
                     tmem_st_wait();
                 }
+                // P (generic-proxy stores) and O are ready for the tensor cores
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_ready[t]);
             }
-            // P (generic-proxy stores) and O are ready for the tensor cores
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_ready[b]);
-        }
-        // ------------------------------------------------------------- epilogue: O / l -> bf16
-        if (ok) {
-            ok = mbar_wait_bounded(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-        }
-        if (ok) {
-            tc_fence_after_sync();
-            const float inv = 1.0f / l;
-            uint16_t* orow = a.o + (static_cast<int64_t>(h) * a.Lq + q0 + row) * kD;
+            // ------------------------------------------------------------- epilogue: O / l -> bf16
+            if (ok) {
+                ok = mbar_wait_bounded(&pv_done[t], (T - 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
+                ok = __all_sync(0xFFFFFFFFu, ok);
+            }
+            if (ok) {
+                tc_fence_after_sync();
+                const float inv = 1.0f / l;
+                uint16_t* orow = a.o + (static_cast<int64_t>(h) * a.Lq + q0 + t * kTile + row) * kD;
 #pragma unroll
-            for (int c4 = 0; c4 < kD / 32; ++c4) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + kColO + static_cast<uint32_t>(c4 * 32), r);
-                tmem_ld_wait();
-                uint32_t w[16];
+                for (int c4 = 0; c4 < kD / 32; ++c4) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(to + static_cast<uint32_t>(c4 * 32), r);
+                    tmem_ld_wait();
+                    uint32_t w[16];
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    w[t] = pack2_bf16(__uint_as_float(r[2 * t]) * inv, __uint_as_float(r[2 * t + 1]) * inv);
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack2_bf16(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
 #pragma unroll
-                for (int v = 0; v < 2; ++v)
-                    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
-                                     orow + c4 * 32 + v * 16),
-                                 "r"(w[8 * v]), "r"(w[8 * v + 1]), "r"(w[8 * v + 2]), "r"(w[8 * v + 3]),
-                                 "r"(w[8 * v + 4]), "r"(w[8 * v + 5]), "r"(w[8 * v + 6]), "r"(w[8 * v + 7])
-                                 : "memory");
+                    for (int v = 0; v < 2; ++v)
+                        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                                         orow + c4 * 32 + v * 16),
+                                     "r"(w[8 * v]), "r"(w[8 * v + 1]), "r"(w[8 * v + 2]), "r"(w[8 * v + 3]),
+                                     "r"(w[8 * v + 4]), "r"(w[8 * v + 5]), "r"(w[8 * v + 6]), "r"(w[8 * v + 7])
+                                     : "memory");
+                }
             }
         }
     }
@@ -369,7 +461,7 @@ cudaError_t launch_attention(const CUtensorMap& qmap, const CUtensorMap& kmap, c
     a.limit_ns = limit_ns;
     a.err = err;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(H * (Lq / kTile)));
+    cfg.gridDim = dim3(static_cast<unsigned>(H * ((Lq / kTile + kQTiles - 1) / kQTiles)));
     cfg.blockDim = dim3(kThreadsA);
     cfg.dynamicSmemBytes = kSmemA;
     cfg.stream = stream;
