@@ -29,11 +29,12 @@
 //   warps 2-9  softmax, four warps per query tile, one thread per query row
 //              (TMEM lane quadrant = warp % 4).  The score buffers are seeded
 //              so that the int8 MMAs leave float bits behind (see kScoreSeed).
-//              Pass 1 reads the scores from TMEM for the row maximum (packed
-//              f32x2 arithmetic, three-input max); pass 2 reads them again,
-//              p = 2^(x - m) on the special-function unit, p rounded to bf16
-//              into the tile's P buffer (128-byte swizzle, the A operand's
-//              canonical K-major layout), the row sum.  Then O *=
+//              One sweep over the scores in TMEM gives the row maximum and,
+//              against the running maximum m, p = 2^(x - m) on the
+//              special-function unit, rounded to bf16 (kept in registers) and
+//              summed; a second sweep runs only when a row's maximum moved
+//              (see below).  p goes to the tile's P buffer (128-byte swizzle,
+//              the A operand's canonical K-major layout).  Then O *=
 //              2^(m_old - m_new) in TMEM (the reference maximum moves only
 //              when a row's scores exceed it by more than 8 in log2 units, and
 //              the rescale is skipped when no row of the warp moved); finally
@@ -119,6 +120,16 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// A 16-byte shared load the compiler must issue where it stands (so values
+// read in a loop are not held in registers across its iterations).
+__device__ __forceinline__ float4 lds128(const float4* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -300,33 +311,55 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 if (!ok) break;
                 tc_fence_after_sync();
                 const float4* cs4 = reinterpret_cast<const float4*>(sSk + st * kTile);
-                // pass 1 (single-load variant)
-                float mx = -INFINITY;
-#pragma unroll
-                for (int c4 = 0; c4 < kTile / 32; ++c4) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 c = cs4[c4 * 8 + q];
-                        const uint64_t ca = pk2(c.x, c.y), cb = pk2(c.z, c.w);
-                        float x0, x1, x2, x3;
-                        upk2(fma2(pk2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), ca,
-                                  mul2(ca, neg_seed2)), x0, x1);
-                        upk2(fma2(pk2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), cb,
-                                  mul2(cb, neg_seed2)), x2, x3);
-                        mx = max3(mx, max3(x0, x1, x2), x3);
-                    }
-                }
-                mx *= rs;
+                // One sweep over the tile's scores from TMEM: x = float(q.k) * s_k[c]
+                // (the score in log2 units is x * rs, rs = s_q * scale * log2(e) >= 0),
+                // the tile's row maximum, and p = 2^(x rs - mref) as packed bf16 in
+                // registers with their sum.
                 // The softmax is exact for any reference m (O / l cancels it); m
-                // only has to keep 2^(x - m) in range.  So m moves only when the
-                // tile's maximum exceeds it by more than 8 (p <= 2^8 otherwise,
-                // fine in bf16 and f32), which skips most rescales of O.
-                const float m_new = (mx > m + kRescaleLog2) ? mx : m;
+                // only has to keep 2^(x - m) in range.  So the exponentials are
+                // taken against the running m right away, and m moves only when a
+                // row's maximum exceeds it by more than 8 (p <= 2^8 otherwise, fine
+                // in bf16 and f32): then, and on the first tile (m = -inf), a second
+                // sweep redoes the warp's rows against the new references (rows that
+                // did not move recompute the same values).
+                float mx = -INFINITY, m_new = m, mref = m;
+                uint64_t sum2 = pk2(0.0f, 0.0f);
+                uint32_t pw[kTile / 2];
+#pragma unroll 1
+                for (int sweep = 0; sweep < 2; ++sweep) {
+                    const uint64_t nm2 = pk2(-mref, -mref);
+                    float mxa = -INFINITY, mxb = -INFINITY;
+                    float4 cq;
+                    sum2 = pk2(0.0f, 0.0f);
+#pragma unroll
+                    for (int c4 = 0; c4 < kTile / 32; ++c4) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int pi = 0; pi < 16; ++pi) {  // column pairs (2 pi, 2 pi + 1) of the 32
+                            if ((pi & 1) == 0) cq = lds128(cs4 + c4 * 8 + (pi >> 1));
+                            const uint64_t c2 = (pi & 1) ? pk2(cq.z, cq.w) : pk2(cq.x, cq.y);
+                            const uint64_t x2 = fma2(pk2(__uint_as_float(r[2 * pi]), __uint_as_float(r[2 * pi + 1])),
+                                                     c2, mul2(c2, neg_seed2));
+                            float x0, x1, y0, y1;
+                            upk2(x2, x0, x1);
+                            if (pi & 1) mxb = max3(mxb, x0, x1);
+                            else mxa = max3(mxa, x0, x1);
+                            upk2(fma2(x2, rs2, nm2), y0, y1);
+                            const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+                            sum2 = add2(sum2, pk2(p0, p1));
+                            pw[c4 * 16 + pi] = pack2_bf16(p0, p1);
+                        }
+                    }
+                    mx = fmaxf(mxa, mxb) * rs;  // the tile's row maximum in log2 units
+                    m_new = (mx > m + kRescaleLog2) ? mx : m;
+                    if (sweep == 1 || !__any_sync(0xFFFFFFFFu, m_new != mref)) break;
+                    mref = m_new;
+                }
                 const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf), 1 when m stays
-                const uint64_t nm2 = pk2(-m_new, -m_new);
+                // S_t has been read for the last time: seed it for the next scores
+                if (j + 1 < T) seed_scores();
                 // P_t is free, and O_t complete, once P V of tile j - 1 is done
                 if (j >= 1) {
                     ok = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
@@ -334,41 +367,12 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                     if (!ok) break;
                     tc_fence_after_sync();
                 }
-                // pass 2 (single-load variant)
-                uint64_t sum2 = pk2(0.0f, 0.0f);
 #pragma unroll
-                for (int c4 = 0; c4 < kTile / 32; ++c4) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int hq = 0; hq < 2; ++hq) {
-                            const float4 c = cs4[c4 * 8 + c8 * 2 + hq];
-                            const float cc[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-                            for (int pr = 0; pr < 2; ++pr) {
-                                const int e = c8 * 8 + hq * 4 + pr * 2;
-                                const uint64_t c2 = pk2(cc[2 * pr], cc[2 * pr + 1]);
-                                const uint64_t x2 = fma2(pk2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2,
-                                                         mul2(c2, neg_seed2));
-                                float y0, y1;
-                                upk2(fma2(x2, rs2, nm2), y0, y1);
-                                const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-                                sum2 = add2(sum2, pk2(p0, p1));
-                                w[hq * 2 + pr] = pack2_bf16(p0, p1);
-                            }
-                        }
-                        const int chunk16 = c4 * 4 + c8;
-                        const int atom = chunk16 >> 3, chunk = chunk16 & 7;
-                        *reinterpret_cast<uint4*>(prow + atom * kAtomBytes + ((chunk ^ (row & 7)) << 4)) =
-                            make_uint4(w[0], w[1], w[2], w[3]);
-                    }
+                for (int chunk16 = 0; chunk16 < kTile / 8; ++chunk16) {  // 8 keys = one 16-byte chunk of P
+                    const int atom = chunk16 >> 3, chunk = chunk16 & 7;
+                    *reinterpret_cast<uint4*>(prow + atom * kAtomBytes + ((chunk ^ (row & 7)) << 4)) =
+                        make_uint4(pw[4 * chunk16], pw[4 * chunk16 + 1], pw[4 * chunk16 + 2], pw[4 * chunk16 + 3]);
                 }
-                // S_t has been read for the last time: seed it for the next scores
-                if (j + 1 < T) seed_scores();
                 float s0, s1;
                 upk2(sum2, s0, s1);
                 l = l * alpha + (s0 + s1);
