@@ -12,10 +12,15 @@
 // rescaled by 2^(m_old - m_new) whenever m grows), so S only ever lives one
 // 128 x 128 tile at a time in tensor memory.
 //
-// One CTA per (head, pair of 128-query tiles A and B), 320 threads:
-//   warp 0     TMA producer: the two Q tiles once, then for each 128-key tile
-//              its K codes, the two halves of V^T and the 128 key scales into
-//              one of two ring stages (shared by both query tiles)
+// One CTA per (head, pair of 128-query tiles A and B), 352 threads:
+//   warp 0     TMA producer of the keys: the two Q tiles once, then for each
+//              128-key tile its K codes and its 128 key scales into one of
+//              three ring stages (freed once both tiles' scores are computed
+//              and their softmax has read the scales)
+//   warp 10    TMA producer of the values: the two halves of V^T of each key
+//              tile into one of two ring stages (freed by both tiles' P V).
+//              With separate rings the next keys load while the current P V
+//              still holds its values, so no load waits on the P V chain.
 //   warp 1     TMEM owner and MMA issuer (one thread), per key tile j and
 //              query tile t = A, B in turn:
 //                S_t = Q_t K_{j+1}^T  kind::i8, M = N = 128, 4 MMAs of K = 32
@@ -57,21 +62,23 @@ namespace {
 constexpr int kD = 128;        // head dimension
 constexpr int kTile = 128;     // queries per tile and keys per tile
 constexpr int kQTiles = 2;     // query tiles per CTA
-constexpr int kThreadsA = (2 + 4 * kQTiles) * 32;
+constexpr int kThreadsA = (3 + 4 * kQTiles) * 32;  // key producer, MMA, softmax, value producer
+constexpr int kWarpV = 2 + 4 * kQTiles;             // the value producer's warp
 constexpr int kQBytes = kTile * kD;           // int8 Q tile: 16 KB
 constexpr int kKBytes = kTile * kD;           // int8 K tile: 16 KB
 constexpr int kAtomBytes = 128 * 128;         // one 128-row x 128-byte swizzle column: 16 KB
 constexpr int kVBytes = 2 * kAtomBytes;       // V^T tile (128 d x 128 keys bf16): 32 KB
 constexpr int kPBytes = 2 * kAtomBytes;       // P tile (128 queries x 128 keys bf16): 32 KB
 constexpr int kSkBytes = kTile * 4;           // the tile's key scales
-constexpr int kStages = 2;
+constexpr int kKStages = 3;                   // K codes + key scales
+constexpr int kVStages = 2;                   // V^T
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQTiles * kQBytes;
-constexpr int kOffV = kOffK + kStages * kKBytes;
-constexpr int kOffP = kOffV + kStages * kVBytes;
+constexpr int kOffV = kOffK + kKStages * kKBytes;
+constexpr int kOffP = kOffV + kVStages * kVBytes;
 constexpr int kOffSk = kOffP + kQTiles * kPBytes;
-constexpr int kOffBar = kOffSk + kStages * kSkBytes;
-constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles;
+constexpr int kOffBar = kOffSk + kKStages * kSkBytes;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * kQTiles;
 constexpr int kSmemA = kOffBar + kNumBars * 8 + 16 + 1024;  // + TMEM slot, + 1024-byte alignment slack
 static_assert(kSmemA <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kTmemColsA = 512;          // per query tile: S (128 columns), O (128 columns)
@@ -156,9 +163,11 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     float* sSk = reinterpret_cast<float*>(smem + kOffSk);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;             // [stage]
-    uint64_t* kv_empty = kv_full + kStages;   // [stage]
-    uint64_t* s_full = kv_empty + kStages;    // [query tile]
+    uint64_t* k_full = bars + 1;              // [key stage]
+    uint64_t* k_empty = k_full + kKStages;    // [key stage]
+    uint64_t* v_full = k_empty + kKStages;    // [value stage]
+    uint64_t* v_empty = v_full + kVStages;    // [value stage]
+    uint64_t* s_full = v_empty + kVStages;    // [query tile]
     uint64_t* s_free = s_full + kQTiles;      // [query tile]
     uint64_t* p_ready = s_free + kQTiles;     // [query tile]
     uint64_t* pv_done = p_ready + kQTiles;    // [query tile]
@@ -177,9 +186,13 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         tma_prefetch_desc(&kmap);
         tma_prefetch_desc(&vtmap);
         mbar_init(q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], nq);  // one commit per query tile's P V
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 5 * nq);  // per query tile: the scores' commit and 4 softmax warps
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], nq);  // one commit per query tile's P V
         }
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&s_full[t], 1);
@@ -207,19 +220,30 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             mbar_arrive_expect_tx(q_full, nq * kQBytes);
             for (int t = 0; t < nq; ++t) tma_load_3d(sQ + t * kQBytes, &qmap, q_full, 0, q0 + t * kTile, h);
             for (int j = 0; j < T && ok; ++j) {
-                const int st = j % kStages;
-                if (!mbar_wait_bounded(&kv_empty[st], ((j / kStages) & 1) ^ 1u, a.limit_ns, kErrTimeoutAttn,
+                const int st = j % kKStages;
+                if (!mbar_wait_bounded(&k_empty[st], ((j / kKStages) & 1) ^ 1u, a.limit_ns, kErrTimeoutAttn,
                                        a.err)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&kv_full[st], kKBytes + kVBytes + kSkBytes);
-                tma_load_3d(sK + st * kKBytes, &kmap, &kv_full[st], 0, j * kTile, h);
-                // V^T rows are the 128 d; each 64-key half is one 128-byte swizzle column
-                tma_load_3d(sV + st * kVBytes, &vtmap, &kv_full[st], j * kTile, 0, h);
-                tma_load_3d(sV + st * kVBytes + kAtomBytes, &vtmap, &kv_full[st], j * kTile + 64, 0, h);
+                mbar_arrive_expect_tx(&k_full[st], kKBytes + kSkBytes);
+                tma_load_3d(sK + st * kKBytes, &kmap, &k_full[st], 0, j * kTile, h);
                 bulk_load_g2s(sSk + st * kTile, a.s_k + static_cast<int64_t>(h) * a.Lk + j * kTile, kSkBytes,
-                              &kv_full[st]);
+                              &k_full[st]);
+            }
+        }
+    } else if (warp == kWarpV) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- value producer
+            for (int j = 0; j < T; ++j) {
+                const int st = j % kVStages;
+                if (!mbar_wait_bounded(&v_empty[st], ((j / kVStages) & 1) ^ 1u, a.limit_ns, kErrTimeoutAttn,
+                                       a.err))
+                    break;
+                mbar_arrive_expect_tx(&v_full[st], kVBytes);
+                // V^T rows are the 128 d; each 64-key half is one 128-byte swizzle column
+                tma_load_3d(sV + st * kVBytes, &vtmap, &v_full[st], j * kTile, 0, h);
+                tma_load_3d(sV + st * kVBytes + kAtomBytes, &vtmap, &v_full[st], j * kTile + 64, 0, h);
             }
         }
     } else if (warp == 1) {
@@ -229,16 +253,17 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kTile, kD);
             auto issue_qk = [&](int t, int j) {
                 const uint32_t q_addr = smem_u32(sQ + t * kQBytes);
-                const uint32_t k_addr = smem_u32(sK + (j % kStages) * kKBytes);
+                const uint32_t k_addr = smem_u32(sK + (j % kKStages) * kKBytes);
 #pragma unroll
                 for (int k = 0; k < kD / 32; ++k)
                     mma_i8(tmem + col_s(t), umma_desc_sw128_kmajor(q_addr + k * 32),
                            umma_desc_sw128_kmajor(k_addr + k * 32), idesc_qk, 1u);
                 mma_commit(&s_full[t]);
+                mma_commit(&k_empty[j % kKStages]);
             };
             auto issue_pv = [&](int t, int j) {
                 const uint32_t p_addr = smem_u32(sP + t * kPBytes);
-                const uint32_t v_addr = smem_u32(sV + (j % kStages) * kVBytes);
+                const uint32_t v_addr = smem_u32(sV + (j % kVStages) * kVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     const uint32_t off = static_cast<uint32_t>((kk >> 2) * kAtomBytes + (kk & 3) * 32);
@@ -246,10 +271,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                              umma_desc_sw128_kmajor(v_addr + off), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&pv_done[t]);
-                mma_commit(&kv_empty[j % kStages]);
+                mma_commit(&v_empty[j % kVStages]);
             };
             bool ok = mbar_wait_bounded(q_full, 0, a.limit_ns, kErrTimeoutAttn, a.err) &&
-                      mbar_wait_bounded(&kv_full[0], 0, a.limit_ns, kErrTimeoutAttn, a.err);
+                      mbar_wait_bounded(&k_full[0], 0, a.limit_ns, kErrTimeoutAttn, a.err);
             for (int t = 0; t < nq && ok; ++t) {
                 ok = mbar_wait_bounded(&s_free[t], 0, a.limit_ns, kErrTimeoutAttn, a.err);
                 if (ok) {
@@ -259,7 +284,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             }
             for (int j = 0; j < T && ok; ++j) {
                 if (j + 1 < T)
-                    ok = mbar_wait_bounded(&kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, a.limit_ns,
+                    ok = mbar_wait_bounded(&k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, a.limit_ns,
                                            kErrTimeoutAttn, a.err);
                 for (int t = 0; t < nq && ok; ++t) {
                     if (j + 1 < T) {
@@ -268,7 +293,9 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                         tc_fence_after_sync();
                         issue_qk(t, j + 1);
                     }
-                    ok = mbar_wait_bounded(&p_ready[t], j & 1, a.limit_ns, kErrTimeoutAttn, a.err);
+                    ok = mbar_wait_bounded(&p_ready[t], j & 1, a.limit_ns, kErrTimeoutAttn, a.err) &&
+                         (t > 0 || mbar_wait_bounded(&v_full[j % kVStages], (j / kVStages) & 1, a.limit_ns,
+                                                     kErrTimeoutAttn, a.err));
                     if (!ok) break;
                     tc_fence_after_sync();
                     issue_pv(t, j);
@@ -303,9 +330,9 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             float m = -INFINITY, l = 0.0f;
             bool ok = true;
             for (int j = 0; j < T; ++j) {
-                const int st = j % kStages;
+                const int st = j % kKStages;
                 // the stage's key scales (bulk copy) and the tile's scores
-                ok = mbar_wait_bounded(&kv_full[st], (j / kStages) & 1, a.limit_ns, kErrTimeoutAttn, a.err) &&
+                ok = mbar_wait_bounded(&k_full[st], (j / kKStages) & 1, a.limit_ns, kErrTimeoutAttn, a.err) &&
                      mbar_wait_bounded(&s_full[t], j & 1, a.limit_ns, kErrTimeoutAttn, a.err);
                 ok = __all_sync(0xFFFFFFFFu, ok);
                 if (!ok) break;
@@ -357,6 +384,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                     if (sweep == 1 || !__any_sync(0xFFFFFFFFu, m_new != mref)) break;
                     mref = m_new;
                 }
+                __syncwarp();  // the warp is done with the stage's key scales
+                if (lane == 0) mbar_arrive(&k_empty[st]);
                 const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf), 1 when m stays
                 // S_t has been read for the last time: seed it for the next scores
                 if (j + 1 < T) seed_scores();
