@@ -32,9 +32,9 @@
 //              other.  (One issuer serving both tiles in turn measured faster
 //              than one issuer per tile: 1.90 vs 2.01 ms on 42 heads of 8192.)
 //   warps 2-9  softmax, four warps per query tile, one thread per query row
-//              (TMEM lane quadrant = warp % 4).  The score buffers are seeded
-//              so that the int8 MMAs leave float bits behind (see kScoreSeed).
-//              One sweep over the scores in TMEM gives the row maximum and,
+//              (TMEM lane quadrant = warp % 4).  One sweep over the scores in
+//              TMEM (16-column loads, each overlapped with the arithmetic on
+//              the previous 16) gives the row maximum and,
 //              against the running maximum m, p = 2^(x - m) on the
 //              special-function unit, rounded to bf16 (kept in registers) and
 //              summed; a second sweep runs only when a row's maximum moved
@@ -93,16 +93,6 @@ struct AttnArgs {
     uint64_t limit_ns;
     unsigned int* err;
 };
-
-// Each score buffer starts every tile at the integer 0x4B400000 = the bits of
-// the float 1.5 * 2^23, and the int8 MMAs accumulate onto it: since
-// |q . k| <= 127^2 * 128 < 2^22, the int32 result is exactly the bits of the
-// float 1.5 * 2^23 + (q . k).  So x = fma(bits, s_k, -fl(1.5 * 2^23 * s_k))
-// is float(q . k) * s_k up to the rounding of fl(1.5 * 2^23 * s_k), at most
-// one unit of q . k times s_k (about 3e-5 of p's relative size at the usual
-// scales, far below p's bf16 rounding of 2^-9).
-constexpr uint32_t kScoreSeed = 0x4B400000u;
-constexpr float kSeedValue = 12582912.0f;  // 1.5 * 2^23
 
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
     uint64_t r;
@@ -257,7 +247,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 #pragma unroll
                 for (int k = 0; k < kD / 32; ++k)
                     mma_i8(tmem + col_s(t), umma_desc_sw128_kmajor(q_addr + k * 32),
-                           umma_desc_sw128_kmajor(k_addr + k * 32), idesc_qk, 1u);
+                           umma_desc_sw128_kmajor(k_addr + k * 32), idesc_qk, k > 0 ? 1u : 0u);
                 mma_commit(&s_full[t]);
                 mma_commit(&k_empty[j % kKStages]);
             };
@@ -313,20 +303,14 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             const uint32_t to = tmem + lane_base + col_o(t);
             const float rs = a.s_q[static_cast<int64_t>(h) * a.Lq + q0 + t * kTile + row] * a.scale_log2;
             const uint64_t rs2 = pk2(rs, rs);
-            const uint64_t neg_seed2 = pk2(-kSeedValue, -kSeedValue);
             uint8_t* prow = sP + t * kPBytes + row * 128;
-            uint32_t seed[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) seed[e] = kScoreSeed;
-            auto seed_scores = [&]() {
-#pragma unroll
-                for (int c4 = 0; c4 < kTile / 32; ++c4) tmem_st_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), seed);
-                tmem_st_wait();
+            // S_t may be overwritten by the next scores once the warp has read it
+            auto release_scores = [&]() {
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_free[t]);
             };
-            seed_scores();  // before the first tile's scores
+            release_scores();  // before the first tile's scores
             float m = -INFINITY, l = 0.0f;
             bool ok = true;
             for (int j = 0; j < T; ++j) {
@@ -338,7 +322,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 if (!ok) break;
                 tc_fence_after_sync();
                 const float4* cs4 = reinterpret_cast<const float4*>(sSk + st * kTile);
-                // One sweep over the tile's scores from TMEM: x = float(q.k) * s_k[c]
+                // One sweep over the tile's scores from TMEM: x = float(q . k) * s_k[c]
                 // (the score in log2 units is x * rs, rs = s_q * scale * log2(e) >= 0),
                 // the tile's row maximum, and p = 2^(x rs - mref) as packed bf16 in
                 // registers with their sum.
@@ -359,25 +343,34 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                     float4 cq;
                     sum2 = pk2(0.0f, 0.0f);
 #pragma unroll
-                    for (int c4 = 0; c4 < kTile / 32; ++c4) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(ts + static_cast<uint32_t>(c4 * 32), r);
-                        tmem_ld_wait();
+                    uint32_t rb[2][16];
+                    tmem_ld_32x32b_x16(ts, rb[0]);
+                    tmem_ld_wait_regs(rb[0]);
 #pragma unroll
-                        for (int pi = 0; pi < 16; ++pi) {  // column pairs (2 pi, 2 pi + 1) of the 32
-                            if ((pi & 1) == 0) cq = lds128(cs4 + c4 * 8 + (pi >> 1));
-                            const uint64_t c2 = (pi & 1) ? pk2(cq.z, cq.w) : pk2(cq.x, cq.y);
-                            const uint64_t x2 = fma2(pk2(__uint_as_float(r[2 * pi]), __uint_as_float(r[2 * pi + 1])),
-                                                     c2, mul2(c2, neg_seed2));
+                    for (int c = 0; c < kTile / 16; ++c) {
+                        if (c + 1 < kTile / 16)
+                            tmem_ld_32x32b_x16(ts + static_cast<uint32_t>((c + 1) * 16), rb[(c + 1) & 1]);
+                        const uint32_t(&r)[16] = rb[c & 1];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {  // column pairs (2 q, 2 q + 1) of the 16
+                            const int pi = c * 8 + q;
+                            if ((q & 1) == 0) cq = lds128(cs4 + (pi >> 1));
+                            const uint64_t c2 = (q & 1) ? pk2(cq.z, cq.w) : pk2(cq.x, cq.y);
+                            const uint64_t x2 = mul2(pk2(__int2float_rn(static_cast<int>(r[2 * q])),
+                                                         __int2float_rn(static_cast<int>(r[2 * q + 1]))),
+                                                     c2);
                             float x0, x1, y0, y1;
                             upk2(x2, x0, x1);
-                            if (pi & 1) mxb = max3(mxb, x0, x1);
-                            else mxa = max3(mxa, x0, x1);
+                            if (q & 1)
+                                mxb = max3(mxb, x0, x1);
+                            else
+                                mxa = max3(mxa, x0, x1);
                             upk2(fma2(x2, rs2, nm2), y0, y1);
                             const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
                             sum2 = add2(sum2, pk2(p0, p1));
-                            pw[c4 * 16 + pi] = pack2_bf16(p0, p1);
+                            pw[pi] = pack2_bf16(p0, p1);
                         }
+                        if (c + 1 < kTile / 16) tmem_ld_wait_regs(rb[(c + 1) & 1]);
                     }
                     mx = fmaxf(mxa, mxb) * rs;  // the tile's row maximum in log2 units
                     m_new = (mx > m + kRescaleLog2) ? mx : m;
@@ -387,8 +380,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 __syncwarp();  // the warp is done with the stage's key scales
                 if (lane == 0) mbar_arrive(&k_empty[st]);
                 const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf), 1 when m stays
-                // S_t has been read for the last time: seed it for the next scores
-                if (j + 1 < T) seed_scores();
+                // S_t has been read for the last time
+                if (j + 1 < T) release_scores();
                 // P_t is free, and O_t complete, once P V of tile j - 1 is done
                 if (j >= 1) {
                     ok = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
