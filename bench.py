@@ -75,6 +75,8 @@ def parse():
                     help="proj: the 768p projection (the headline); mlp: the 768p MLP, up 5376 -> 21504 with "
                          "GELU, then down, timed by both routes of the activation (see --mlp-route); "
                          "attention: int8 attention over 42 heads of 8192 tokens, head dim 128")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="attention workload only: number of heads (default 42; fewer for small profiling runs)")
     ap.add_argument("--mlp-route", choices=["prologue", "epilogue"], default="prologue",
                     help="the route the mlp line's value is for: GELU as the down projection's prologue "
                          "(convrot_linear_act) or in the up projection's epilogue; both are timed")
@@ -306,6 +308,11 @@ def run_attention(args, rank: int, world: int):
     H, L, d = spec.batch, spec.M, spec.K
     q_cpu, k_cpu = W.bmm_inputs(spec)
     v_cpu = torch.randn(H, L, d, generator=torch.Generator().manual_seed(44)).to(torch.bfloat16)
+    if args.heads is not None:  # a smaller case of the same workload: its first heads
+        if not 1 <= args.heads <= H:
+            raise SystemExit(f"--heads must be in [1, {H}]")
+        H = args.heads
+        q_cpu, k_cpu, v_cpu = q_cpu[:H].contiguous(), k_cpu[:H].contiguous(), v_cpu[:H].contiguous()
     q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
     Lib = C.load()
     ws = torch.empty((Lib.convrot_attention_workspace_bytes(H, L, L),), dtype=torch.uint8, device="cuda")
@@ -365,10 +372,11 @@ def run_attention(args, rank: int, world: int):
             "metric": ATTN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": times["full"] * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
-            "config": {"workload": "attention_h42_l8192_d128", "heads": H, "Lq": L, "Lk": L, "d": d,
+            "config": {"workload": f"attention_h{H}_l{L}_d{d}", "heads": H, "Lq": L, "Lk": L, "d": d,
                        "parallelism": f"dp{world} (independent heads and sequences per GPU)",
-                       "l2": "inputs larger than L2: Q, K, V are 88 MB each, O 88 MB; the score matrix (11.3 GB "
-                             "as bf16) is never stored"},
+                       "l2": f"Q, K, V are {H * L * d * 2 / 1e6:.0f} MB each (bf16), O the same"
+                             f"{'' if 4 * H * L * d * 2 > 126e6 else ' (together below L2: a small profiling case)'}; the score "
+                             f"matrix ({H * L * L * 2 / 1e9:.1f} GB as bf16) is never stored"},
             "roofline": {"bound": "tensor", "kernel": "attention_kernel (Q K^T, softmax, P V; one launch)",
                          "achieved": ops / times["kernel"] / 1e12, "peak": ops / t_tensor / 1e12,
                          "unit": "TFLOP/s", "frac": t_tensor / times["kernel"], "traffic": None,
