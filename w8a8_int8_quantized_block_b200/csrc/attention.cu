@@ -455,18 +455,36 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     if (warp == 1) tmem_dealloc(tmem, kTmemColsA);
 }
 
-// V [h][key][d] -> V^T [h][d][key], bf16, through 32 x 32 shared tiles.
-__global__ void transpose_kernel(const uint16_t* __restrict__ v, uint16_t* __restrict__ vt, int L) {
-    __shared__ uint16_t tile[32][33];
-    const int h = blockIdx.z;
-    const int key0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
-    const uint16_t* src = v + static_cast<int64_t>(h) * L * kD;
-    uint16_t* dst = vt + static_cast<int64_t>(h) * kD * L;
-    for (int r = threadIdx.y; r < 32; r += blockDim.y)
-        tile[r][threadIdx.x] = src[static_cast<int64_t>(key0 + r) * kD + d0 + threadIdx.x];
-    __syncthreads();
-    for (int r = threadIdx.y; r < 32; r += blockDim.y)
-        dst[static_cast<int64_t>(d0 + r) * L + key0 + threadIdx.x] = tile[threadIdx.x][r];
+// V [h][key][d] -> V^T [h][d][key], bf16.  Each thread moves one block of
+// 8 keys x 8 d through registers: 8 16-byte loads (one per key row), 32 byte
+// permutes, 8 16-byte stores (one per d row).  A warp covers 32 keys x 64 d:
+// 8 lanes read 128 contiguous bytes of a key row and 4 lanes write 64
+// contiguous bytes of a d row, so every access fills whole 32-byte sectors.
+constexpr int kTransposeThreads = 256;
+
+__global__ void __launch_bounds__(kTransposeThreads)
+    transpose_kernel(const uint16_t* __restrict__ v, uint16_t* __restrict__ vt, int L) {
+    const int h = blockIdx.y;
+    const int w = (blockIdx.x * kTransposeThreads + threadIdx.x) >> 5;  // warp within the head
+    const int lane = threadIdx.x & 31;
+    const int key0 = (w >> 1) * 32 + (lane >> 3) * 8;
+    const int d0 = (w & 1) * 64 + (lane & 7) * 8;
+    if (key0 >= L) return;
+    const uint4* src = reinterpret_cast<const uint4*>(v + (static_cast<int64_t>(h) * L + key0) * kD + d0);
+    uint4 r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = __ldg(src + i * (kD / 8));
+    auto word = [](const uint4& q, int k) { return k == 0 ? q.x : k == 1 ? q.y : k == 2 ? q.z : q.w; };
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // d0 + j: keys key0 .. key0 + 7, pairs (2k, 2k + 1) per word
+        const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+        uint4 o;
+        o.x = __byte_perm(word(r[0], j >> 1), word(r[1], j >> 1), sel);
+        o.y = __byte_perm(word(r[2], j >> 1), word(r[3], j >> 1), sel);
+        o.z = __byte_perm(word(r[4], j >> 1), word(r[5], j >> 1), sel);
+        o.w = __byte_perm(word(r[6], j >> 1), word(r[7], j >> 1), sel);
+        *reinterpret_cast<uint4*>(vt + (static_cast<int64_t>(h) * kD + d0 + j) * L + key0) = o;
+    }
 }
 
 }  // namespace
@@ -502,8 +520,11 @@ cudaError_t launch_attention(const CUtensorMap& qmap, const CUtensorMap& kmap, c
 }
 
 cudaError_t launch_transpose_v(const uint16_t* v, uint16_t* vt, int H, int L, cudaStream_t stream) {
-    transpose_kernel<<<dim3(static_cast<unsigned>(L / 32), kD / 32, static_cast<unsigned>(H)), dim3(32, 8), 0,
-                       stream>>>(v, vt, L);
+    // two warps (one per 64-d half) per 32 keys
+    const int warps = (L + 31) / 32 * 2;
+    const int blocks = (warps * 32 + kTransposeThreads - 1) / kTransposeThreads;
+    transpose_kernel<<<dim3(static_cast<unsigned>(blocks), static_cast<unsigned>(H)), kTransposeThreads, 0, stream>>>(
+        v, vt, L);
     return cudaGetLastError();
 }
 
