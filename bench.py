@@ -327,12 +327,21 @@ def run_attention(args, rank: int, world: int):
     kx, sk = ws[off_kx:off_kx + H * L * d].view(torch.int8).view(H, L, d), ws[off_sk:off_sk + H * L * 4].view(
         torch.float32)
     vt = ws[off_vt:off_vt + H * d * L * 2].view(torch.bfloat16).view(H, d, L)
+    off_part = off_vt + r256(H * d * L * 2)
+    part_bytes = C.attention_split_bytes(H, L, L)
+    part = ws[off_part:off_part + part_bytes] if part_bytes else None
+    # attention launches per call: the units of whole waves, and (when the last
+    # wave is split over its keys) the split units and the combine
+    units = H * ((L // 128 + 1) // 2)
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    main_units = units - units % sms if part_bytes else units
+    attn_launches = (1 if main_units > 0 else 0) + (2 if part_bytes else 0)
 
     def full():
         C.attention(q, k, v, workspace=ws, out=o, stream=stream)
 
     def kernel():
-        C.attention_int8(qx, sq, kx, sk, vt, out=o, stream=stream)
+        C.attention_int8(qx, sq, kx, sk, vt, out=o, stream=stream, split_ws=part)
 
     def barrier():
         if world > 1:
@@ -377,7 +386,9 @@ def run_attention(args, rank: int, world: int):
                        "l2": f"Q, K, V are {H * L * d * 2 / 1e6:.0f} MB each (bf16), O the same"
                              f"{'' if 4 * H * L * d * 2 > 126e6 else ' (together below L2: a small profiling case)'}; the score "
                              f"matrix ({H * L * L * 2 / 1e9:.1f} GB as bf16) is never stored"},
-            "roofline": {"bound": "tensor", "kernel": "attention_kernel (Q K^T, softmax, P V; one launch)",
+            "roofline": {"bound": "tensor",
+                         "kernel": f"attention_kernel (Q K^T, softmax, P V; {attn_launches} launch"
+                                   f"{'es: whole units, split units, combine' if attn_launches > 1 else ''})",
                          "achieved": ops / times["kernel"] / 1e12, "peak": ops / t_tensor / 1e12,
                          "unit": "TFLOP/s", "frac": t_tensor / times["kernel"], "traffic": None,
                          "peak_source": f"{kind}: Q K^T at bf16 burst x {INT8_PER_BF16}, P V at the bf16 burst "
@@ -386,7 +397,7 @@ def run_attention(args, rank: int, world: int):
             "kernels": {"attention_kernel_us": times["kernel"] * 1e6,
                         "quantise_transpose_us": (times["full"] - times["kernel"]) * 1e6},
             "clocks": clk_summary,
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (3 + attn_launches) * args.steps,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

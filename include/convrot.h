@@ -185,7 +185,8 @@ convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int
  * o [H][Lq][128] bf16 (32-byte aligned).  Lq and Lk multiples of 128, scale > 0
  * (1/sqrt(128) for the usual softmax scale).  `workspace` (256-byte aligned,
  * >= convrot_attention_workspace_bytes(H, Lq, Lk)) receives the Q and K codes
- * and scales and V^T.  Four kernels on `stream`. */
+ * and scales, V^T and the split parts (see convrot_attention_int8).  Four to
+ * six kernels on `stream`. */
 size_t convrot_attention_workspace_bytes(int64_t H, int64_t Lq, int64_t Lk);
 convrot_status convrot_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t H, int64_t Lq,
                                  int64_t Lk, float scale, void* workspace, size_t ws_bytes, uint16_t* o,
@@ -193,10 +194,21 @@ convrot_status convrot_attention(const uint16_t* q, const uint16_t* k, const uin
 
 /* The attention kernel alone, on quantised inputs: qx int8 [H][Lq][128] and
  * s_q f32 [H][Lq]; kx int8 [H][Lk][128] and s_k f32 [H][Lk] (16-byte
- * aligned); vt = V^T, bf16 [H][128][Lk]; o as above. */
+ * aligned); vt = V^T, bf16 [H][128][Lk]; o as above.
+ *
+ * The work runs as one CTA per SM for each head and pair of query tiles.
+ * When the last wave of those units would leave most SMs idle, the keys of
+ * its units are split over all SMs and a small kernel combines the parts
+ * (O = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p).  That needs
+ * `split_ws`, a caller-owned device buffer (16-byte aligned) of
+ * convrot_attention_split_bytes(H, Lq, Lk) bytes; pass NULL (or fewer bytes)
+ * to run every unit whole.  The split has no counterpart on the pages; it
+ * only changes the order of the f32 sums.  The size depends on the current
+ * device's SM count (0 when nothing would be split). */
+size_t convrot_attention_split_bytes(int64_t H, int64_t Lq, int64_t Lk);
 convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const int8_t* kx, const float* s_k,
                                       const uint16_t* vt, int64_t H, int64_t Lq, int64_t Lk, float scale,
-                                      uint16_t* o, void* stream);
+                                      void* split_ws, size_t split_bytes, uint16_t* o, void* stream);
 
 /* End-to-end form of convrot_linear_fused for callers whose activations live
  * in host memory: copies x_host (bf16 [M][K], contiguous; pinned for overlap)

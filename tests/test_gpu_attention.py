@@ -101,3 +101,44 @@ def test_attention_full_size_sampled_rows():
                            bits(v), heads, rows, 128 ** -0.5)
     got = o[torch.from_numpy(heads).to(DEV), torch.from_numpy(rows).to(DEV)].float().cpu().numpy()
     assert_close_bf16(got, ref, "attention full size (sampled rows)")
+
+
+def test_attention_splits_the_last_wave_over_the_keys():
+    # 150 units (heads x query-tile pairs) on 148 SMs: 148 run whole, the last
+    # two are split over their 4 key tiles and combined; rows of both kinds
+    # are checked against the oracle
+    H, Lq, Lk = 150, 256, 512
+    q, k, v = _qkv(H, Lq, Lk, seed=8)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    o, ws = _run(q, k, v)
+    assert C.attention_split_bytes(H, Lq, Lk) > 0 or sms >= H
+    qx, sq = O.quantize_act(bits(q.reshape(H * Lq, 128)), 0)
+    kx, sk = O.quantize_act(bits(k.reshape(H * Lk, 128)), 0)
+    rng = np.random.default_rng(9)
+    heads = np.concatenate([np.full(12, H - 1), np.full(12, H - 2), rng.integers(0, H - 2, 12)])
+    rows = rng.integers(0, Lq, heads.size)
+    ref = O.attention_rows(qx.reshape(H, Lq, 128), sq.reshape(H, Lq), kx.reshape(H, Lk, 128), sk.reshape(H, Lk),
+                           bits(v), heads, rows, 128 ** -0.5)
+    got = o[torch.from_numpy(heads).to(DEV), torch.from_numpy(rows).to(DEV)].float().cpu().numpy()
+    assert_close_bf16(got, ref, "attention, split last wave")
+
+
+def test_attention_int8_with_and_without_the_split_buffer():
+    # the kernel entry on quantised inputs: the split path (parts + combine)
+    # and every unit whole both match the oracle
+    H, Lq, Lk = 2, 256, 2048
+    q, k, v = _qkv(H, Lq, Lk, seed=10)
+    qx, sq = C.quantize_act(q.reshape(H * Lq, 128).to(DEV), 0)
+    kx, sk = C.quantize_act(k.reshape(H * Lk, 128).to(DEV), 0)
+    vt = v.transpose(1, 2).contiguous().to(DEV)
+    nbytes = C.attention_split_bytes(H, Lq, Lk)
+    assert nbytes > 0  # 2 units on one wave: split 8 ways over 16 key tiles
+    split_ws = torch.empty((nbytes,), dtype=torch.uint8, device=DEV)
+    args = (qx.view(H, Lq, 128), sq.view(H, Lq), kx.view(H, Lk, 128), sk.view(H, Lk), vt)
+    o_split = C.attention_int8(*args, split_ws=split_ws)
+    o_whole = C.attention_int8(*args)
+    torch.cuda.synchronize()
+    assert C.last_device_status() == (C.OK, 0)
+    ref, _ = O.attention(bits(q), bits(k), bits(v))
+    assert_close_bf16(o_split.float().cpu().numpy(), ref, "attention_int8 split")
+    assert_close_bf16(o_whole.float().cpu().numpy(), ref, "attention_int8 whole")

@@ -40,7 +40,8 @@ EXPORTS = (
     "convrot_w8a8_linear", "convrot_workspace_bytes", "convrot_linear_fused", "convrot_linear_fused_host",
     "convrot_w8a8_bmm", "convrot_igemm_s32", "convrot_last_device_status", "convrot_set_wait_limit_ns",
     "convrot_selftest_wait_timeout", "convrot_linear_fused_noalloc", "convrot_act_quantize", "convrot_linear_act",
-    "convrot_attention_workspace_bytes", "convrot_attention", "convrot_attention_int8",
+    "convrot_attention_workspace_bytes", "convrot_attention", "convrot_attention_split_bytes",
+    "convrot_attention_int8",
 )
 
 
@@ -96,7 +97,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "convrot_act_quantize": ([P, I64, I64, I64, I32, I32, P, P, P], ctypes.c_int),
         "convrot_attention_workspace_bytes": ([I64, I64, I64], ctypes.c_size_t),
         "convrot_attention": ([P, P, P, I64, I64, I64, ctypes.c_float, P, ctypes.c_size_t, P, P], ctypes.c_int),
-        "convrot_attention_int8": ([P, P, P, P, P, I64, I64, I64, ctypes.c_float, P, P], ctypes.c_int),
+        "convrot_attention_split_bytes": ([I64, I64, I64], ctypes.c_size_t),
+        "convrot_attention_int8": ([P, P, P, P, P, I64, I64, I64, ctypes.c_float, P, ctypes.c_size_t, P, P],
+                                   ctypes.c_int),
         "convrot_linear_act": ([P, I64, I64, I32, P, P, ctypes.POINTER(WDesc), P, I32, P, ctypes.c_size_t, P, I64,
                                 P], ctypes.c_int),
     }
@@ -235,16 +238,25 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | 
     return o
 
 
+def attention_split_bytes(H: int, Lq: int, Lk: int) -> int:
+    """Bytes of the buffer that lets attention_int8 split the last wave's units
+    over their keys on the current device (0: nothing to split)."""
+    return int(load().convrot_attention_split_bytes(H, Lq, Lk))
+
+
 def attention_int8(qx, sq, kx, sk, vt, scale: float | None = None, out: torch.Tensor | None = None,
-                   stream=None) -> torch.Tensor:
+                   stream=None, split_ws: torch.Tensor | None = None) -> torch.Tensor:
     """The attention kernel on quantised inputs: qx [H, Lq, 128] int8, sq [H, Lq],
-    kx [H, Lk, 128] int8, sk [H, Lk], vt = V^T [H, 128, Lk] bf16."""
+    kx [H, Lk, 128] int8, sk [H, Lk], vt = V^T [H, 128, Lk] bf16.  split_ws
+    (attention_split_bytes bytes, optional) lets the last wave's units run
+    split over their keys."""
     H, Lq, d = qx.shape
     Lk = kx.shape[1]
     o = torch.empty((H, Lq, d), dtype=torch.bfloat16, device=qx.device) if out is None else out
     _check("convrot_attention_int8", load().convrot_attention_int8(
         _ptr(qx), _ptr(sq), _ptr(kx), _ptr(sk), _ptr(vt), H, Lq, Lk, (d ** -0.5) if scale is None else scale,
-        _ptr(o), _stream(stream)))
+        _ptr(split_ws), 0 if split_ws is None else split_ws.numel() * split_ws.element_size(), _ptr(o),
+        _stream(stream)))
     return o
 
 

@@ -380,16 +380,27 @@ convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int
     return gemm(qx, qw, sx, s_w, bias, alpha_for_block(desc->block), epi, 1, M, desc->N, desc->K, y, ldy, true, s);
 }
 
+size_t convrot_attention_split_bytes(int64_t H, int64_t Lq, int64_t Lk) {
+    if (H <= 0 || Lq <= 0 || Lk <= 0 || Lq % 128 != 0 || Lk % 128 != 0) return 0;
+    if (H * Lq > kMaxI32 || H * Lk > kMaxI32) return 0;
+    const DeviceInfo* d = device_info();
+    if (!d) return 0;
+    const AttnSplit sp = attention_split_plan(static_cast<int>(H), static_cast<int>(Lq), static_cast<int>(Lk),
+                                              d->num_sms);
+    return sp.splits > 1 ? attention_split_bytes(sp.tail * sp.splits) : 0;
+}
+
 size_t convrot_attention_workspace_bytes(int64_t H, int64_t Lq, int64_t Lk) {
     if (H <= 0 || Lq <= 0 || Lk <= 0) return 0;
     const size_t hq = static_cast<size_t>(H) * static_cast<size_t>(Lq);
     const size_t hk = static_cast<size_t>(H) * static_cast<size_t>(Lk);
-    return round256(hq * 128) + round256(hq * 4) + round256(hk * 128) + round256(hk * 4) + round256(hk * 128 * 2);
+    return round256(hq * 128) + round256(hq * 4) + round256(hk * 128) + round256(hk * 4) + round256(hk * 128 * 2) +
+           round256(convrot_attention_split_bytes(H, Lq, Lk));
 }
 
 convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const int8_t* kx, const float* s_k,
                                       const uint16_t* vt, int64_t H, int64_t Lq, int64_t Lk, float scale,
-                                      uint16_t* o, void* stream) {
+                                      void* split_ws, size_t split_bytes, uint16_t* o, void* stream) {
     if (!qx || !s_q || !kx || !s_k || !vt || !o) return CONVROT_EINVAL;
     if (H <= 0 || Lq <= 0 || Lk <= 0 || Lq % 128 != 0 || Lk % 128 != 0) return CONVROT_EINVAL;
     if (H * Lq > kMaxI32 || H * Lk > kMaxI32 || Lk > (int64_t{1} << 24)) return CONVROT_EINVAL;
@@ -397,9 +408,15 @@ convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const 
     if (!aligned16(qx) || !aligned16(kx) || !aligned16(vt) || !aligned16(s_k)) return CONVROT_EINVAL;
     if ((reinterpret_cast<uintptr_t>(s_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(o) & 31u) != 0)
         return CONVROT_EINVAL;
+    if (split_ws != nullptr && !aligned16(split_ws)) return CONVROT_EINVAL;
     const DeviceInfo* d = device_info();
     if (!d) return CONVROT_ECUDA;
     if (!d->supported) return CONVROT_EUNSUPPORTED;
+    const AttnSplit plan = attention_split_plan(static_cast<int>(H), static_cast<int>(Lq), static_cast<int>(Lk),
+                                                d->num_sms);
+    void* part = nullptr;  // without room for the parts every unit runs whole
+    if (split_ws != nullptr && plan.splits > 1 && split_bytes >= attention_split_bytes(plan.tail * plan.splits))
+        part = split_ws;
     CUtensorMap qmap, kmap, vtmap;
     if (!encode_3d(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, 128, static_cast<uint64_t>(Lq), static_cast<uint64_t>(H),
                    128, static_cast<uint64_t>(Lq) * 128, 128, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -414,7 +431,7 @@ convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const 
     const float scale_log2 = scale * 1.4426950408889634f;
     return cuda_status(launch_attention(qmap, kmap, vtmap, static_cast<int>(H), static_cast<int>(Lq),
                                         static_cast<int>(Lk), s_q, s_k, scale_log2, o, g_limit_ns.load(), d->err, true,
-                                        static_cast<cudaStream_t>(stream)));
+                                        static_cast<cudaStream_t>(stream), plan, part));
 }
 
 convrot_status convrot_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t H, int64_t Lq,
@@ -438,6 +455,9 @@ convrot_status convrot_attention(const uint16_t* q, const uint16_t* k, const uin
     float* sk = reinterpret_cast<float*>(w);
     w += round256(hk * 4);
     uint16_t* vt = reinterpret_cast<uint16_t*>(w);
+    w += round256(hk * 128 * 2);
+    void* part = w;  // the parts of split units (convrot_attention_split_bytes)
+    const size_t part_bytes = convrot_attention_split_bytes(H, Lq, Lk);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // Q and K: the rowwise int8 quantiser without rotation, one row per token
     convrot_status st = rotate_quant(q, 2, static_cast<int64_t>(hq), 128, 128, 0, qx, sq, s);
@@ -446,7 +466,8 @@ convrot_status convrot_attention(const uint16_t* q, const uint16_t* k, const uin
     if (st != CONVROT_OK) return st;
     st = cuda_status(launch_transpose_v(v, vt, static_cast<int>(H), static_cast<int>(Lk), s));
     if (st != CONVROT_OK) return st;
-    return convrot_attention_int8(qx, sq, kx, sk, vt, H, Lq, Lk, scale, o, stream);
+    return convrot_attention_int8(qx, sq, kx, sk, vt, H, Lq, Lk, scale, part_bytes ? part : nullptr, part_bytes, o,
+                                  stream);
 }
 
 convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, const int8_t* qw, const float* s_w,

@@ -92,6 +92,13 @@ struct AttnArgs {
     uint16_t* o;           // [H][Lq][128] bf16
     uint64_t limit_ns;
     unsigned int* err;
+    // Work split: CTA i takes unit unit0 + i / splits (a head and a pair of
+    // query tiles) and the splits-th part (i % splits) of its key tiles.
+    // With splits > 1 it writes its unnormalised O and (m, l) per row to
+    // o_part / ml_part (slot i) for attention_combine_kernel instead of O.
+    int unit0, splits;
+    float* o_part;         // [slot][256][128] f32
+    float2* ml_part;       // [slot][256] (m, l)
 };
 
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -166,10 +173,14 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int pairs = (a.Lq / kTile + kQTiles - 1) / kQTiles;
-    const int h = blockIdx.x / pairs;
-    const int q0 = (blockIdx.x - h * pairs) * kQTiles * kTile;
+    const int unit = a.unit0 + static_cast<int>(blockIdx.x) / a.splits;
+    const int piece = static_cast<int>(blockIdx.x) % a.splits;
+    const int h = unit / pairs;
+    const int q0 = (unit - h * pairs) * kQTiles * kTile;
     const int nq = min(kQTiles, (a.Lq - q0) / kTile);  // 1 when Lq / 128 is odd and this is the last pair
-    const int T = a.Lk / kTile;  // key tiles
+    const int T_all = a.Lk / kTile;
+    const int j0 = piece * T_all / a.splits;           // this CTA's key tiles: [j0, j0 + T)
+    const int T = (piece + 1) * T_all / a.splits - j0;
 
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&qmap);
@@ -217,9 +228,9 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(&k_full[st], kKBytes + kSkBytes);
-                tma_load_3d(sK + st * kKBytes, &kmap, &k_full[st], 0, j * kTile, h);
-                bulk_load_g2s(sSk + st * kTile, a.s_k + static_cast<int64_t>(h) * a.Lk + j * kTile, kSkBytes,
-                              &k_full[st]);
+                tma_load_3d(sK + st * kKBytes, &kmap, &k_full[st], 0, (j0 + j) * kTile, h);
+                bulk_load_g2s(sSk + st * kTile, a.s_k + static_cast<int64_t>(h) * a.Lk + (j0 + j) * kTile,
+                              kSkBytes, &k_full[st]);
             }
         }
     } else if (warp == kWarpV) {
@@ -232,8 +243,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                     break;
                 mbar_arrive_expect_tx(&v_full[st], kVBytes);
                 // V^T rows are the 128 d; each 64-key half is one 128-byte swizzle column
-                tma_load_3d(sV + st * kVBytes, &vtmap, &v_full[st], j * kTile, 0, h);
-                tma_load_3d(sV + st * kVBytes + kAtomBytes, &vtmap, &v_full[st], j * kTile + 64, 0, h);
+                tma_load_3d(sV + st * kVBytes, &vtmap, &v_full[st], (j0 + j) * kTile, 0, h);
+                tma_load_3d(sV + st * kVBytes + kAtomBytes, &vtmap, &v_full[st], (j0 + j) * kTile + 64, 0, h);
             }
         }
     } else if (warp == 1) {
@@ -342,7 +353,6 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                     float mxa = -INFINITY, mxb = -INFINITY;
                     float4 cq;
                     sum2 = pk2(0.0f, 0.0f);
-#pragma unroll
                     uint32_t rb[2][16];
                     tmem_ld_32x32b_x16(ts, rb[0]);
                     tmem_ld_wait_regs(rb[0]);
@@ -424,7 +434,26 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 ok = mbar_wait_bounded(&pv_done[t], (T - 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
                 ok = __all_sync(0xFFFFFFFFu, ok);
             }
-            if (ok) {
+            if (ok && a.splits > 1) {
+                // a part of the keys: the unnormalised O rows and (m, l) for the combine
+                tc_fence_after_sync();
+                const int64_t slot_row = static_cast<int64_t>(blockIdx.x) * (kQTiles * kTile) + t * kTile + row;
+                float* prow_o = a.o_part + slot_row * kD;
+#pragma unroll 1
+                for (int c4 = 0; c4 < kD / 32; ++c4) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(to + static_cast<uint32_t>(c4 * 32), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                                         prow_o + c4 * 32 + v * 8),
+                                     "r"(r[8 * v]), "r"(r[8 * v + 1]), "r"(r[8 * v + 2]), "r"(r[8 * v + 3]),
+                                     "r"(r[8 * v + 4]), "r"(r[8 * v + 5]), "r"(r[8 * v + 6]), "r"(r[8 * v + 7])
+                                     : "memory");
+                }
+                a.ml_part[slot_row] = make_float2(m, l);
+            } else if (ok) {
                 tc_fence_after_sync();
                 const float inv = 1.0f / l;
                 uint16_t* orow = a.o + (static_cast<int64_t>(h) * a.Lq + q0 + t * kTile + row) * kD;
@@ -453,6 +482,49 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     __syncthreads();
     tc_fence_after_sync();
     if (warp == 1) tmem_dealloc(tmem, kTmemColsA);
+}
+
+// O rows of the split units from their parts: with m_p, l_p and the
+// unnormalised O_p of part p (each against its own reference m_p),
+// O = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p for M = max_p m_p.  One
+// warp per row, four columns per lane.
+constexpr int kCombineRows = 8;  // rows (warps) per CTA
+
+__global__ void __launch_bounds__(kCombineRows * 32)
+    attention_combine_kernel(const float* __restrict__ o_part, const float2* __restrict__ ml_part, int Lq,
+                             int unit0, int splits, uint16_t* __restrict__ o) {
+    pdl_wait_primary();  // the parts come from the previous kernel
+    const int lane = threadIdx.x & 31;
+    const int r = static_cast<int>(blockIdx.x) * kCombineRows + (threadIdx.x >> 5);  // row among the split units
+    const int u = r / (kQTiles * kTile);     // split unit, 0-based
+    const int rr = r - u * (kQTiles * kTile);  // row within the unit's query-tile pair
+    const int pairs = (Lq / kTile + kQTiles - 1) / kQTiles;
+    const int unit = unit0 + u;
+    const int h = unit / pairs;
+    const int q0 = (unit - h * pairs) * kQTiles * kTile;
+    if (rr >= min(kQTiles, (Lq - q0) / kTile) * kTile) return;  // past the unit's last query tile
+    const int q = q0 + rr;
+    const int64_t slot0 = static_cast<int64_t>(u) * splits;
+    float M = -INFINITY;
+    for (int p = 0; p < splits; ++p) M = fmaxf(M, ml_part[(slot0 + p) * (kQTiles * kTile) + rr].x);
+    float L = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int p = 0; p < splits; ++p) {
+        const int64_t sr = (slot0 + p) * (kQTiles * kTile) + rr;
+        const float2 ml = ml_part[sr];
+        const float w = ex2_approx(ml.x - M);
+        L = fmaf(w, ml.y, L);
+        const float4 v = reinterpret_cast<const float4*>(o_part + sr * kD)[lane];
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+    }
+    const float inv = 1.0f / L;
+    uint2 out;
+    out.x = pack2_bf16(acc.x * inv, acc.y * inv);
+    out.y = pack2_bf16(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(o + (static_cast<int64_t>(h) * Lq + q) * kD)[lane] = out;
 }
 
 // V [h][key][d] -> V^T [h][d][key], bf16.  Each thread moves one block of
@@ -489,9 +561,28 @@ __global__ void __launch_bounds__(kTransposeThreads)
 
 }  // namespace
 
+AttnSplit attention_split_plan(int H, int Lq, int Lk, int num_sms) {
+    AttnSplit sp;
+    sp.units = H * ((Lq / kTile + kQTiles - 1) / kQTiles);
+    sp.main = sp.units;
+    if (num_sms <= 0) return sp;
+    const int tail = sp.units % num_sms;
+    const int s = min(num_sms / max(tail, 1), (Lk / kTile) / 2);  // at least two key tiles per part
+    if (tail == 0 || s < 2) return sp;
+    sp.main = sp.units - tail;
+    sp.tail = tail;
+    sp.splits = s;
+    return sp;
+}
+
+size_t attention_split_bytes(int slots) {
+    return static_cast<size_t>(slots) * (kQTiles * kTile) * (kD * sizeof(float) + sizeof(float2));
+}
+
 cudaError_t launch_attention(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vtmap, int H,
                              int Lq, int Lk, const float* s_q, const float* s_k, float scale_log2, uint16_t* o,
-                             uint64_t limit_ns, unsigned int* err, bool pdl, cudaStream_t stream) {
+                             uint64_t limit_ns, unsigned int* err, bool pdl, cudaStream_t stream,
+                             const AttnSplit& sp, void* part) {
     cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA);
     if (e != cudaSuccess) return e;
     AttnArgs a;
@@ -504,8 +595,11 @@ cudaError_t launch_attention(const CUtensorMap& qmap, const CUtensorMap& kmap, c
     a.o = o;
     a.limit_ns = limit_ns;
     a.err = err;
+    a.unit0 = 0;
+    a.splits = 1;
+    a.o_part = nullptr;
+    a.ml_part = nullptr;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(H * ((Lq / kTile + kQTiles - 1) / kQTiles)));
     cfg.blockDim = dim3(kThreadsA);
     cfg.dynamicSmemBytes = kSmemA;
     cfg.stream = stream;
@@ -514,8 +608,35 @@ cudaError_t launch_attention(const CUtensorMap& qmap, const CUtensorMap& kmap, c
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, attention_kernel, qmap, kmap, vtmap, a);
-    if (e != cudaSuccess) return e;
+    const bool split = sp.splits > 1 && part != nullptr;
+    const int main_units = split ? sp.main : sp.units;
+    if (main_units > 0) {
+        cfg.gridDim = dim3(static_cast<unsigned>(main_units));
+        e = cudaLaunchKernelEx(&cfg, attention_kernel, qmap, kmap, vtmap, a);
+        if (e != cudaSuccess) return e;
+    }
+    if (split) {
+        // the units of the last, partly filled wave: their keys spread over all SMs
+        const int slots = sp.tail * sp.splits;
+        a.unit0 = sp.main;
+        a.splits = sp.splits;
+        a.o_part = static_cast<float*>(part);
+        a.ml_part = reinterpret_cast<float2*>(static_cast<uint8_t*>(part) +
+                                              static_cast<size_t>(slots) * (kQTiles * kTile) * kD * sizeof(float));
+        cfg.gridDim = dim3(static_cast<unsigned>(slots));
+        cfg.numAttrs = (main_units > 0 || pdl) ? 1 : 0;  // after the main launch (or the producers of Q, K, V^T)
+        e = cudaLaunchKernelEx(&cfg, attention_kernel, qmap, kmap, vtmap, a);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cc = {};
+        cc.gridDim = dim3(static_cast<unsigned>(sp.tail * kQTiles * kTile / kCombineRows));
+        cc.blockDim = dim3(kCombineRows * 32);
+        cc.stream = stream;
+        cc.attrs = attr;
+        cc.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cc, attention_combine_kernel, static_cast<const float*>(a.o_part),
+                               static_cast<const float2*>(a.ml_part), Lq, sp.main, sp.splits, o);
+        if (e != cudaSuccess) return e;
+    }
     return cudaGetLastError();
 }
 
