@@ -213,9 +213,13 @@ convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const 
 /* End-to-end form of convrot_linear_fused for callers whose activations live
  * in host memory: copies x_host (bf16 [M][K], contiguous; pinned for overlap)
  * into the caller's device buffer x_dev, runs the fused linear into y_dev
- * (bf16 [M][N], contiguous) and copies it back to y_host.  All enqueued on
- * `stream`; the host buffers must stay valid until the stream reaches the end
- * of the call. */
+ * (bf16 [M][N], contiguous) and copies it back to y_host.  The workspace is
+ * that of convrot_linear_fused (>= convrot_workspace_bytes(M, K)).  Rows of
+ * more than ~16 MiB of input run in chunks whose copy in, compute and copy
+ * out overlap: the copies go on two streams the library owns (one per
+ * direction and device), ordered by events, and `stream` waits for the last
+ * copy out, so the call is ordered on `stream` as one operation.  The host
+ * buffers must stay valid until the stream reaches the end of the call. */
 convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, const int8_t* qw, const float* s_w,
                                          const convrot_wdesc* desc, const float* bias, int32_t epilogue,
                                          uint16_t* x_dev, void* workspace, size_t ws_bytes, uint16_t* y_dev,

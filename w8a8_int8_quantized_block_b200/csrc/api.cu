@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -271,6 +272,43 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
                                            epi, d->num_sms, true, stream));
 }
 
+// Rows per chunk of convrot_linear_fused_host's copy/compute pipeline: about
+// 16 MiB of input per chunk, a multiple of the 256-row panel.
+int64_t host_chunk_rows(int64_t M, int64_t K) {
+    const int64_t rows = ((int64_t{16} << 20) / (K * 2) + 255) / 256 * 256;
+    return std::max<int64_t>(rows, 256) >= M ? M : std::max<int64_t>(rows, 256);
+}
+
+// The library's copy streams and events of the host-buffer pipeline, one set
+// per device, created on first use with that device current.
+struct HostPipe {
+    static constexpr int kEvents = 4;
+    std::mutex mutex;  // one call at a time enqueues on this device's set
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr, in[kEvents] = {}, out[kEvents] = {};
+    bool ready = false;
+};
+HostPipe g_host_pipe[kMaxDevices];
+
+HostPipe* host_pipe() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    HostPipe& hp = g_host_pipe[dev];
+    if (!hp.ready) {
+        bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.end, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; good && i < HostPipe::kEvents; ++i)
+            good = cudaEventCreateWithFlags(&hp.in[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&hp.out[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) return nullptr;  // the caller falls back to the one-piece form
+        hp.ready = true;
+    }
+    return &hp;
+}
+
 }  // namespace
 }  // namespace convrot
 
@@ -478,14 +516,52 @@ convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, cons
     if (st != CONVROT_OK) return st;
     if (!x_host || !y_host || !x_dev || !aligned16(x_dev)) return CONVROT_EINVAL;
     if (desc->N % 8 != 0) return CONVROT_EINVAL;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CONVROT_EINVAL;
+    if (ws_bytes < convrot_workspace_bytes(M, desc->K)) return CONVROT_EINVAL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t xbytes = static_cast<size_t>(M) * static_cast<size_t>(desc->K) * 2;
-    const size_t ybytes = static_cast<size_t>(M) * static_cast<size_t>(desc->N) * 2;
-    if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return CONVROT_ECUDA;
-    st = convrot_linear_fused(x_dev, M, desc->K, qw, s_w, desc, bias, epilogue, workspace, ws_bytes, y_dev,
-                              desc->N, stream);
-    if (st != CONVROT_OK) return st;
-    if (cudaMemcpyAsync(y_host, y_dev, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return CONVROT_ECUDA;
+    const int64_t K = desc->K, N = desc->N;
+    const int64_t chunk = host_chunk_rows(M, K);
+    HostPipe* hp = chunk < M ? host_pipe() : nullptr;
+    if (hp == nullptr) {  // one piece: copy in, compute, copy out, all on the caller's stream
+        if (cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(M * K) * 2, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+            return CONVROT_ECUDA;
+        st = convrot_linear_fused(x_dev, M, K, qw, s_w, desc, bias, epilogue, workspace, ws_bytes, y_dev, N,
+                                  stream);
+        if (st != CONVROT_OK) return st;
+        if (cudaMemcpyAsync(y_host, y_dev, static_cast<size_t>(M * N) * 2, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess)
+            return CONVROT_ECUDA;
+        return CONVROT_OK;
+    }
+    // Row chunks in a pipeline: chunk i's rows go in on the library's
+    // host-to-device stream while chunk i - 1 computes on the caller's stream
+    // and chunk i - 2's results come out on the device-to-host stream (the two
+    // copy directions run on separate copy engines).  Events order each
+    // chunk's three steps; the caller's stream waits for the last copy out, so
+    // the call stays ordered on `stream` like the one-piece form.
+    std::lock_guard<std::mutex> lock(hp->mutex);
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    if (!ok(cudaEventRecord(hp->start, s)) || !ok(cudaStreamWaitEvent(hp->h2d, hp->start, 0)) ||
+        !ok(cudaStreamWaitEvent(hp->d2h, hp->start, 0)))
+        return CONVROT_ECUDA;
+    int i = 0;
+    for (int64_t r0 = 0; r0 < M; r0 += chunk, ++i) {
+        const int64_t rows = std::min(chunk, M - r0);
+        cudaEvent_t in = hp->in[i % HostPipe::kEvents], out = hp->out[i % HostPipe::kEvents];
+        if (!ok(cudaMemcpyAsync(x_dev + r0 * K, x_host + r0 * K, static_cast<size_t>(rows * K) * 2,
+                                cudaMemcpyHostToDevice, hp->h2d)) ||
+            !ok(cudaEventRecord(in, hp->h2d)) || !ok(cudaStreamWaitEvent(s, in, 0)))
+            return CONVROT_ECUDA;
+        st = convrot_linear_fused(x_dev + r0 * K, rows, K, qw, s_w, desc, bias, epilogue, workspace, ws_bytes,
+                                  y_dev + r0 * N, N, stream);
+        if (st != CONVROT_OK) return st;
+        if (!ok(cudaEventRecord(out, s)) || !ok(cudaStreamWaitEvent(hp->d2h, out, 0)) ||
+            !ok(cudaMemcpyAsync(y_host + r0 * N, y_dev + r0 * N, static_cast<size_t>(rows * N) * 2,
+                                cudaMemcpyDeviceToHost, hp->d2h)))
+            return CONVROT_ECUDA;
+    }
+    if (!ok(cudaEventRecord(hp->end, hp->d2h)) || !ok(cudaStreamWaitEvent(s, hp->end, 0))) return CONVROT_ECUDA;
     return CONVROT_OK;
 }
 
