@@ -215,7 +215,7 @@ convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const 
  * into the caller's device buffer x_dev, runs the fused linear into y_dev
  * (bf16 [M][N], contiguous) and copies it back to y_host.  The workspace is
  * that of convrot_linear_fused (>= convrot_workspace_bytes(M, K)).  Rows of
- * more than ~16 MiB of input run in chunks whose copy in, compute and copy
+ * more than ~32 MiB of input run in chunks whose copy in, compute and copy
  * out overlap: the copies go on two streams the library owns (one per
  * direction and device), ordered by events, and `stream` waits for the last
  * copy out, so the call is ordered on `stream` as one operation.  The host

@@ -14,10 +14,10 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("M,gelu", [(4000, False), (3585, True), (700, False)])
+@pytest.mark.parametrize("M,gelu", [(7000, False), (6657, True), (700, False)])
 def test_host_pipeline_equals_device_call(M, gelu):
-    # K = 5376: about 1790 rows per 16 MiB chunk, so 4000 and 3585 rows run in
-    # three chunks (the last one ragged) and 700 rows in one piece
+    # K = 5376: 3328 rows per 32 MiB chunk, so 7000 and 6657 rows run in three
+    # chunks (the last one ragged, down to a single row) and 700 rows in one piece
     K, N = 5376, 320
     spec, (x, w, bias) = W.custom_linear(M, K, N, seed=M + 3)
     pw = C.pack_weight(w.to(DEV), 128)
