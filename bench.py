@@ -83,6 +83,9 @@ def parse():
     ap.add_argument("--context-parallel", action="store_true",
                     help="strong scaling: the 38656 tokens split across the ranks, each step the rank's linear "
                          "then an NCCL all-gather of the bf16 rows so every rank holds the whole output")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="with --kernel-only: only the first ROWS token rows of the projection (a smaller case "
+                         "of the same workload, for detailed profiler captures)")
     ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm"], default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
                          "(for profiler captures; prints no result line)")
@@ -529,6 +532,12 @@ def main():
         return run_mlp(args, rank, world)
     spec = workload(args)
     x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
+    if args.rows is not None:
+        import dataclasses
+        if not args.kernel_only or not 1 <= args.rows <= spec.M:
+            raise SystemExit(f"--rows needs --kernel-only and 1 <= ROWS <= {spec.M}")
+        spec = dataclasses.replace(spec, M=args.rows, name=f"{spec.name}_rows{args.rows}")
+        x_cpu = x_cpu[:args.rows].contiguous()
     job = spec  # the whole job's tokens
     if args.context_parallel:
         import dataclasses

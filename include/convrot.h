@@ -131,7 +131,8 @@ convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int
                                    uint16_t* y, int64_t ldy, void* stream);
 
 /* Bytes of device workspace convrot_linear_fused needs: the int8 codes
- * (M*K, rounded up to 256) plus the scales (4*M, rounded up to 256). */
+ * (M*K, rounded up to 256), the scales (4*M, rounded up to 256) and the
+ * one-kernel path's counters (4 * (2 * ceil(M/256) + 1), rounded up to 256). */
 size_t convrot_workspace_bytes(int64_t M, int64_t K);
 
 /* The whole linear, steps 1-4, on `stream`: one kernel (quantiser warps run
@@ -140,7 +141,10 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K);
  * GEMM starts while the quantiser drains).  x: bf16 [M][K] (row stride ldx);
  * the codes and scales go to `workspace` (>= convrot_workspace_bytes(M, K)
  * bytes, 256-byte aligned, caller-owned, must not be shared by calls that
- * overlap). */
+ * overlap).  The one-kernel path keeps the codes of at most 12 row panels of
+ * 256 rows at a time (a ring, reused as the tensor cores finish each panel),
+ * so after the call the workspace holds the scales of every row but not every
+ * row's codes. */
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw,
                                     const float* s_w, const convrot_wdesc* desc, const float* bias,
                                     int32_t epilogue, void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy,

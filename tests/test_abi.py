@@ -38,9 +38,9 @@ def test_abi_version_and_status_strings():
 
 def test_workspace_bytes():
     L = C.load()
-    # codes, scales, and one counter per 256-row panel plus one, each rounded to 256 bytes
+    # codes, scales, and two counters per 256-row panel plus one, each rounded to 256 bytes
     r = lambda v: (v + 255) // 256 * 256
-    assert L.convrot_workspace_bytes(38656, 5376) == 38656 * 5376 + r(38656 * 4) + r(152 * 4)
+    assert L.convrot_workspace_bytes(38656, 5376) == 38656 * 5376 + r(38656 * 4) + r((2 * 151 + 1) * 4)
     assert L.convrot_workspace_bytes(1, 128) == 256 + 256 + 256
     assert L.convrot_workspace_bytes(0, 128) == 0
 

@@ -16,6 +16,7 @@ from w8a8_int8_quantized_block_b200 import workloads as W
 from helpers import assert_close_bf16, assert_codes_match, bits, f32_of_bf16
 
 pytestmark = pytest.mark.gpu
+RING = 12  # panel slots of the one-kernel linear's codes ring (kFusedRingPanels)
 
 
 def _sample(M, N, rows, pairs, seed):
@@ -46,13 +47,30 @@ def test_proj_768p_full_size():
     y = C.linear_fused(xd, pw, bias.cuda(), workspace=ws)
     torch.cuda.synchronize()
     assert C.last_device_status() == (C.OK, 0)
-    qx = ws[:spec.M * spec.K].view(torch.int8).view(spec.M, spec.K).cpu().numpy()
-    # workspace layout: codes [M][K], then the scales, each region rounded up to 256 bytes
+    # workspace layout: the codes region ([M][K] bytes), then the scales, each
+    # rounded up to 256 bytes.  The one-kernel path keeps the codes of RING row
+    # panels of 256 at a time (panel p in slot p % RING), so after the call the
+    # slots hold the last RING panels; every row's scale is there.
     off = (spec.M * spec.K + 255) // 256 * 256
     sx = ws[off:off + spec.M * 4].view(torch.float32).cpu().numpy()
     xb = bits(x)
     qxr, sxr = O.quantize_act(xb, spec.block)
-    assert_codes_match(qx, sx, qxr, sxr, None, spec.block)
+    ring = ws[:RING * 256 * spec.K].view(torch.int8).view(RING * 256, spec.K).cpu().numpy()
+    panels = (spec.M + 255) // 256
+    qx = np.zeros_like(qxr)
+    held = np.zeros(spec.M, dtype=bool)
+    for p in range(panels - RING, panels):
+        r0, r1 = p * 256, min(spec.M, (p + 1) * 256)
+        qx[r0:r1] = ring[(p % RING) * 256:(p % RING) * 256 + (r1 - r0)]
+        held[r0:r1] = True
+    assert_codes_match(qx[held], sx[held], qxr[held], sxr[held], None, spec.block)
+    bad = np.nonzero(sx.view(np.uint32) != sxr.view(np.uint32))[0]
+    assert bad.size == 0, f"{bad.size} scales differ"
+    # every row's codes: the standalone quantiser (the same arithmetic; the
+    # fused and two-kernel outputs are compared bit for bit in test_gpu_parity)
+    q2, s2 = C.quantize_act(xd, spec.block)
+    torch.cuda.synchronize()
+    assert_codes_match(q2.cpu().numpy(), s2.cpu().numpy(), qxr, sxr, None, spec.block)
     qwr, swr = O.pack_weight(w.numpy(), spec.block)
     assert_codes_match(pw.q.cpu().numpy(), pw.s.cpu().numpy(), qwr, swr)
     rows, mi, ni = _sample(spec.M, spec.N, 48, 8192, 1)

@@ -168,6 +168,20 @@ def test_linear_fused_equals_two_step_bitwise():
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+@pytest.mark.parametrize("M,K,N", [(7937, 5376, 264), (16000, 256, 64)])
+def test_linear_fused_codes_ring_equals_two_step_bitwise(M, K, N):
+    # More than 12 row panels: the one-kernel path reuses its ring of code
+    # slots (7937 rows: 31 panels, the last of one row; 16000 rows: 63 panels
+    # of one column tile each, so every slot turns over five times).  The
+    # two-kernel path keeps every row's codes, so any slot overwritten too
+    # early or read stale changes outputs.
+    spec, (x, w, bias) = W.custom_linear(M, K, N, seed=M + 11, n_out=3, token_scale=True)
+    y1, _ = _run_linear((x, w, bias), fused=True)
+    y2, _ = _run_linear((x, w, bias), fused=False)
+    assert C.last_device_status() == (C.OK, 0)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
 @pytest.mark.parametrize("M,K,N", [(1, 128, 8), (127, 512, 384), (129, 640, 264), (257, 5376, 520),
                                    (1000, 1024, 2048)])
 def test_linear_ragged_shapes(M, K, N):

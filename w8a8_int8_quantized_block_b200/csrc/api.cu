@@ -243,8 +243,14 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
     if (!d->supported) return CONVROT_EUNSUPPORTED;
     const int64_t K = desc->K, N = desc->N;
     CUtensorMap amap, bmap, ymap;
-    if (!encode_3d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, static_cast<uint64_t>(K), static_cast<uint64_t>(M), 1,
-                   static_cast<uint64_t>(K), static_cast<uint64_t>(M * K), kGemmBK, kGemmBM, 1,
+    const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
+    // the codes ring: every panel its own slot when they fit (then rows past M
+    // read as zeros), else kFusedRingPanels full slots
+    const int64_t qrows = static_cast<int64_t>(fused_ring_slots(M)) < static_cast<int64_t>(panels)
+                              ? int64_t{fused_ring_slots(M)} * 2 * kGemmBM
+                              : M;
+    if (!encode_3d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, static_cast<uint64_t>(K), static_cast<uint64_t>(qrows),
+                   1, static_cast<uint64_t>(K), static_cast<uint64_t>(qrows * K), kGemmBK, kGemmBM, 1,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
     if (!encode_3d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, static_cast<uint64_t>(K), static_cast<uint64_t>(N), 1,
@@ -255,8 +261,7 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
                    static_cast<uint64_t>(ldy) * 2, static_cast<uint64_t>(M * ldy) * 2, kEpiColsBf16, kEpiRows, 1,
                    CU_TENSOR_MAP_SWIZZLE_64B))
         return CONVROT_ECUDA;
-    const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
-    if (cudaMemsetAsync(ready, 0, (panels + 1) * 4, stream) != cudaSuccess) return CONVROT_ECUDA;
+    if (cudaMemsetAsync(ready, 0, (2 * panels + 1) * 4, stream) != cudaSuccess) return CONVROT_ECUDA;
     GemmArgs a;
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(N);
@@ -369,7 +374,7 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
     const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
     return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) + round256(static_cast<size_t>(M) * 4) +
-           round256((panels + 1) * 4);
+           round256((2 * panels + 1) * 4);
 }
 
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,

@@ -97,11 +97,25 @@ constexpr int kEpiRows = 32;      // rows per epilogue store (one warp)
 // Largest K the one-kernel linear handles (one 96-thread group per row).
 constexpr int kFusedMaxK = 6144;
 
+// The one-kernel linear keeps the codes of at most this many 256-row panels
+// (a ring of slots, reused once every tile has loaded the panel in it), so
+// that they stay in L2 between the quantiser that writes them and the tensor
+// cores that read them, and are overwritten there instead of written back.
+constexpr int kFusedRingPanels = 12;
+
+// Slots of the ring for M rows: every panel its own slot when they fit.
+inline int fused_ring_slots(int64_t M) {
+    const int64_t panels = (M + 2 * kGemmBM - 1) / (2 * kGemmBM);
+    return static_cast<int>(panels < kFusedRingPanels ? panels : kFusedRingPanels);
+}
+
 // Rotate + quantise + GEMM + epilogue in one persistent CTA-pair kernel.
 // x: bf16 rows [M][ldx] (16-byte aligned rows); amap/bmap/ymap as for
-// launch_igemm with batch 1, amap over q.  q, s: the codes and scales it
-// writes; ready: ceil(M/256) + 1 zeroed counters (per-panel ready rows, then
-// the panels the GEMM has started).  kind: a RotKind.
+// launch_igemm with batch 1, amap over q's fused_ring_slots(M) * 256 rows
+// (M rows when the panels all fit).  q: the ring of codes; s: the scales
+// [M]; ready: 2 ceil(M/256) + 1 zeroed counters (per-panel ready rows, the
+// panels the GEMM has started, per-panel tiles whose codes are loaded).
+// kind: a RotKind.
 cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMap& amap, const CUtensorMap& bmap,
                                 const CUtensorMap& ymap, const GemmArgs& g, int8_t* q, float* s,
                                 unsigned int* ready, int kind, int epilogue, int num_sms, bool pdl,

@@ -24,6 +24,17 @@
 // and every CTA is resident (the grid is sized to what fits), so every wait
 // ends; each wait is bounded all the same.
 //
+// The codes live in a ring of kFusedRingPanels panel slots (16.5 MB at K =
+// 5376) rather than an [M][K] array: panel p goes to slot p % ring once every
+// tile has loaded the panel that held the slot before (the MMA issuer counts
+// a tile's panel as loaded when the last stage of its A has landed).  The
+// codes are stored and loaded with an L2 evict-last policy, so the ring stays
+// in L2 next to the weights while x and y stream past (evict-first), and a
+// slot is overwritten there rather than written back to HBM; with one slot
+// per panel the codes made a ~390 MB round trip through HBM per 768p step.  No wait forms a cycle: a
+// quantiser waits on a panel `ring` panels earlier, whose tiles only need
+// that panel's codes.
+//
 // Shared memory per CTA: the 6-stage GEMM ring (192 KB) and epilogue staging
 // and column scales (24 KB), as in the GEMM alone.  (A 4-stage ring, which
 // left room to stage input rows by TMA, ran the GEMM part 10% slower.)
@@ -53,7 +64,10 @@ constexpr int kPanelRows = 2 * kGemmBM;        // 256: the pair's tile height
 // Quantisers stay at most this many panels ahead of the first panel the GEMM
 // has not started, so the codes (1.4 MB per panel at K = 5376) are still in L2
 // when the tensor cores read them instead of making a round trip to HBM.
-constexpr int kPanelsAhead = 16;
+// (With the 12-slot ring below, 10 panels ahead measured best: DRAM traffic
+// per 768p step 846 MB, against 1025 MB for 20 slots / 16 ahead and 1210 MB
+// with one slot per panel.)
+constexpr int kPanelsAhead = 10;
 constexpr int kStagesF = 6;
 constexpr int kAStageF = kGemmBM * BK;
 constexpr int kBStageF = (BN / 2) * BK;
@@ -72,6 +86,8 @@ struct FusedArgs {
     float* s;               // [M] scales (workspace)
     unsigned int* ready;    // [ceil(M/256)] rows of each panel already quantised (zeroed)
     unsigned int* started;  // panels the GEMM has begun (a running max; zeroed)
+    unsigned int* loaded;   // [ceil(M/256)] tiles of each panel whose codes have landed (zeroed)
+    int ring;               // panel slots of the codes ring
     int tpr;                // K / 64: threads of a group holding data
     int kind;               // the rotation (a RotKind; the kernel is instantiated for it)
 };
@@ -143,6 +159,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         const int64_t stride = static_cast<int64_t>(gridDim.x) * kQGroups;
         const int64_t first = blockIdx.x + static_cast<int64_t>(gridDim.x) * qg;
         float* gred = red + qg * 2 * kQWarps;
+        const uint64_t keep_l2 = l2_policy_evict_last();  // the codes ring stays in L2 until it is reused
         uint32_t w[qcore::kRawWords];  // the next row's elements, loaded ahead
         if (holds && first < p.M) qcore::load_bf16_global(f.x + first * f.ldx, t, w);
         int it = 0;
@@ -156,6 +173,11 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                 !wait_count_bounded(f.started, static_cast<uint32_t>(panel - kPanelsAhead + 1), p.limit_ns,
                                     kErrTimeoutPanel, p.err))
                 break;  // the error word is set; the GEMM side times out the same way
+            // the ring slot is free once every tile of its previous panel has loaded it
+            if (panel >= f.ring && !wait_count_bounded(f.loaded + (panel - f.ring), static_cast<uint32_t>(tiles_n),
+                                                       p.limit_ns, kErrTimeoutPanel, p.err))
+                break;
+            const int64_t qrow = static_cast<int64_t>(panel % f.ring) * kPanelRows + (row - int64_t{panel} * kPanelRows);
             uint64_t P[kPairs];
             if (holds) {
                 qcore::unpack_bf16_pairs(w, P);
@@ -175,7 +197,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             for (int i = 1; i < kQWarps; ++i) amax = fmaxf(amax, gred[(it & 1) * kQWarps + i]);
             if (holds) {
                 const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-                qcore::quantize_store<true>(P, inv, f.q + row * p.K + static_cast<int64_t>(t) * kPerThread);
+                qcore::quantize_store<true, true>(P, inv, f.q + qrow * p.K + static_cast<int64_t>(t) * kPerThread,
+                                                  keep_l2);
                 if (t == 0) f.s[row] = __fdiv_rn(amax, 127.0f);
             }
             __threadfence();                    // this thread's codes are visible device-wide
@@ -188,6 +211,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     } else if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------- producer (both CTAs)
+            const uint64_t keep_l2 = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -205,7 +229,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     ready_panel = panel;
                     atomicMax(f.started, static_cast<unsigned int>(panel + 1));  // lets the quantisers move on
                 }
-                const int a_row = c.m0 + static_cast<int>(rank) * kGemmBM;
+                const int a_row = (panel % f.ring) * kPanelRows + static_cast<int>(rank) * kGemmBM;
                 const int b_row = c.n0 + static_cast<int>(rank) * (BN / 2);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, p.limit_ns, kErrTimeoutEmpty, p.err)) {
@@ -214,7 +238,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     }
                     if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (kAStageF + kBStageF));
                     const uint32_t leader_full = mapa_shared(smem_u32(&full_bar[stage]), 0);
-                    tma_load_3d_pair(sA + stage * kAStageF, &amap, leader_full, kb * BK, a_row, 0);
+                    tma_load_3d_pair_hint(sA + stage * kAStageF, &amap, leader_full, kb * BK, a_row, 0, keep_l2);
                     tma_load_3d_pair(sB + stage * kBStageF, &bmap, leader_full, kb * BK, b_row, 0);
                     if (++stage == kStagesF) {
                         stage = 0;
@@ -258,6 +282,11 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                         phase ^= 1u;
                     }
                 }
+                // Both CTAs' A stages of this tile have landed (each full barrier
+                // counts both halves), so its reads of the panel's ring slot are
+                // complete: the slot has one reader less.  (A plain reduction: the
+                // reads finished before the barrier wait returned.)
+                if (ok && f.ring < tiles_m) atomicAdd(f.loaded + t / tiles_n, 1u);
                 mma_commit_pair(&accf_bar[acc], 0x3);
                 if (++acc == kAccBufs) {
                     acc = 0;
@@ -375,6 +404,8 @@ cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMa
     f.s = s;
     f.ready = ready;
     f.started = ready + (g.M + kPanelRows - 1) / kPanelRows;
+    f.loaded = f.started + 1;
+    f.ring = fused_ring_slots(g.M);
     f.tpr = g.K / kPerThread;
     f.kind = kind;
     if (f.tpr > kQThreads || g.K % kPerThread != 0) return cudaErrorInvalidValue;

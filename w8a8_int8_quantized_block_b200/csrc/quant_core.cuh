@@ -222,8 +222,9 @@ __device__ __forceinline__ void fwht_across_lanes(uint64_t (&P)[kPairs], int sh,
 //     the packed multiply even with -fmad=false; as fma(v, 1, c) there is no
 //     multiply-add pair to fuse.  Crafted rows whose f32 product is exactly
 //     k + 1/2 while the exact product is not check this on the GPU.
-template <bool kMagicAdd>
-__device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], float inv, int8_t* dst) {
+template <bool kMagicAdd, bool kL2Hint = false>
+__device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], float inv, int8_t* dst,
+                                               uint64_t l2_policy = 0) {
     const uint64_t inv2 = pk(inv, inv);
     const uint64_t one2 = pk(1.0f, 1.0f);
     const uint64_t magic2 = pk(12582912.0f, 12582912.0f);  // 1.5 * 2^23
@@ -251,11 +252,20 @@ __device__ __forceinline__ void quantize_store(const uint64_t (&P)[kPairs], floa
         word[kPairs / 4 + i] = prmt(prmt(hi[0], hi[1], 0x0040u), prmt(hi[2], hi[3], 0x0040u), 0x5410u);
     }
 #pragma unroll
-    for (int i = 0; i < kPerThread / 32; ++i)
-        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 32 * i),
-                     "r"(word[8 * i]), "r"(word[8 * i + 1]), "r"(word[8 * i + 2]), "r"(word[8 * i + 3]),
-                     "r"(word[8 * i + 4]), "r"(word[8 * i + 5]), "r"(word[8 * i + 6]), "r"(word[8 * i + 7])
-                     : "memory");
+    for (int i = 0; i < kPerThread / 32; ++i) {
+        if constexpr (kL2Hint)
+            asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;" ::"l"(
+                             dst + 32 * i),
+                         "r"(word[8 * i]), "r"(word[8 * i + 1]), "r"(word[8 * i + 2]), "r"(word[8 * i + 3]),
+                         "r"(word[8 * i + 4]), "r"(word[8 * i + 5]), "r"(word[8 * i + 6]), "r"(word[8 * i + 7]),
+                         "l"(l2_policy)
+                         : "memory");
+        else
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 32 * i),
+                         "r"(word[8 * i]), "r"(word[8 * i + 1]), "r"(word[8 * i + 2]), "r"(word[8 * i + 3]),
+                         "r"(word[8 * i + 4]), "r"(word[8 * i + 5]), "r"(word[8 * i + 6]), "r"(word[8 * i + 7])
+                         : "memory");
+    }
 }
 
 // ---- regular H_4^(x)k stages
