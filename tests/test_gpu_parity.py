@@ -182,6 +182,17 @@ def test_linear_fused_codes_ring_equals_two_step_bitwise(M, K, N):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+def test_linear_fused_long_rows_match_oracle():
+    # K > 6144 (the MLP down projection's 21504): linear_fused runs the
+    # quantiser and the GEMM as two kernels
+    M, K, N = 257, 21504, 136
+    spec, (x, w, bias) = W.custom_linear(M, K, N, seed=23, n_out=30, token_scale=True)
+    y, pw = _run_linear((x, w, bias), fused=True)
+    assert C.last_device_status() == (C.OK, 0)
+    yr, *_ = O.linear(bits(x), w.numpy(), bias.numpy(), 128)
+    assert_close_bf16(f32_of_bf16(y), yr, "linear K=21504")
+
+
 @pytest.mark.parametrize("M,K,N", [(1, 128, 8), (127, 512, 384), (129, 640, 264), (257, 5376, 520),
                                    (1000, 1024, 2048)])
 def test_linear_ragged_shapes(M, K, N):

@@ -246,8 +246,8 @@ convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, cons
     const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
     // the codes ring: every panel its own slot when they fit (then rows past M
     // read as zeros), else kFusedRingPanels full slots
-    const int64_t qrows = static_cast<int64_t>(fused_ring_slots(M)) < static_cast<int64_t>(panels)
-                              ? int64_t{fused_ring_slots(M)} * 2 * kGemmBM
+    const int64_t qrows = static_cast<int64_t>(fused_ring_slots(M, K)) < static_cast<int64_t>(panels)
+                              ? int64_t{fused_ring_slots(M, K)} * 2 * kGemmBM
                               : M;
     if (!encode_3d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, static_cast<uint64_t>(K), static_cast<uint64_t>(qrows),
                    1, static_cast<uint64_t>(K), static_cast<uint64_t>(qrows * K), kGemmBK, kGemmBM, 1,

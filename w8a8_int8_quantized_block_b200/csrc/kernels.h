@@ -97,21 +97,30 @@ constexpr int kEpiRows = 32;      // rows per epilogue store (one warp)
 // Largest K the one-kernel linear handles (one 96-thread group per row).
 constexpr int kFusedMaxK = 6144;
 
-// The one-kernel linear keeps the codes of at most this many 256-row panels
-// (a ring of slots, reused once every tile has loaded the panel in it), so
-// that they stay in L2 between the quantiser that writes them and the tensor
-// cores that read them, and are overwritten there instead of written back.
+// The one-kernel linear keeps the codes of a few 256-row panels at a time (a
+// ring of slots, reused once every tile has loaded the panel in it), so that
+// they stay in L2 between the quantiser that writes them and the tensor cores
+// that read them, and are overwritten there instead of written back: about
+// 16.5 MB of slots (12 panels at K = 5376), at least 4 and at most 12.
 constexpr int kFusedRingPanels = 12;
+constexpr int64_t kFusedRingBytes = int64_t{12} * 256 * 5376;
 
-// Slots of the ring for M rows: every panel its own slot when they fit.
-inline int fused_ring_slots(int64_t M) {
+// Slots of the ring for M rows of K: every panel its own slot when they fit.
+inline int fused_ring_slots(int64_t M, int64_t K) {
     const int64_t panels = (M + 2 * kGemmBM - 1) / (2 * kGemmBM);
-    return static_cast<int>(panels < kFusedRingPanels ? panels : kFusedRingPanels);
+    int64_t slots = kFusedRingBytes / (2 * kGemmBM * K);
+    slots = slots < 4 ? 4 : (slots > kFusedRingPanels ? kFusedRingPanels : slots);
+    return static_cast<int>(panels < slots ? panels : slots);
 }
+
+// Whether the ring's lines are marked evict-last in L2: only while the weights
+// (N x K bytes, re-read for every panel) fit beside it with room to spare;
+// larger weights need the L2 more than the codes do.
+inline bool fused_codes_l2_hint(int64_t K, int64_t N) { return K * N <= (int64_t{48} << 20); }
 
 // Rotate + quantise + GEMM + epilogue in one persistent CTA-pair kernel.
 // x: bf16 rows [M][ldx] (16-byte aligned rows); amap/bmap/ymap as for
-// launch_igemm with batch 1, amap over q's fused_ring_slots(M) * 256 rows
+// launch_igemm with batch 1, amap over q's fused_ring_slots(M, K) * 256 rows
 // (M rows when the panels all fit).  q: the ring of codes; s: the scales
 // [M]; ready: 2 ceil(M/256) + 1 zeroed counters (per-panel ready rows, the
 // panels the GEMM has started, per-panel tiles whose codes are loaded).

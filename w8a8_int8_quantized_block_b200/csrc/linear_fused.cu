@@ -24,14 +24,17 @@
 // and every CTA is resident (the grid is sized to what fits), so every wait
 // ends; each wait is bounded all the same.
 //
-// The codes live in a ring of kFusedRingPanels panel slots (16.5 MB at K =
+// The codes live in a ring of panel slots (about 16.5 MB: 12 slots at K =
 // 5376) rather than an [M][K] array: panel p goes to slot p % ring once every
 // tile has loaded the panel that held the slot before (the MMA issuer counts
-// a tile's panel as loaded when the last stage of its A has landed).  The
+// a tile's panel as loaded when the last stage of its A has landed).  When
+// the weights are small enough to stay in L2 beside it (N K <= 48 MB), the
 // codes are stored and loaded with an L2 evict-last policy, so the ring stays
 // in L2 next to the weights while x and y stream past (evict-first), and a
 // slot is overwritten there rather than written back to HBM; with one slot
-// per panel the codes made a ~390 MB round trip through HBM per 768p step.  No wait forms a cycle: a
+// per panel the codes made a ~390 MB round trip through HBM per 768p step.
+// (Larger weights, as in a 4x MLP, need the L2 more; there the normal policy
+// is kept.)  No wait forms a cycle: a
 // quantiser waits on a panel `ring` panels earlier, whose tiles only need
 // that panel's codes.
 //
@@ -88,6 +91,7 @@ struct FusedArgs {
     unsigned int* started;  // panels the GEMM has begun (a running max; zeroed)
     unsigned int* loaded;   // [ceil(M/256)] tiles of each panel whose codes have landed (zeroed)
     int ring;               // panel slots of the codes ring
+    int l2_hint;            // mark the ring's lines evict-last in L2 (else the normal policy)
     int tpr;                // K / 64: threads of a group holding data
     int kind;               // the rotation (a RotKind; the kernel is instantiated for it)
 };
@@ -159,7 +163,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         const int64_t stride = static_cast<int64_t>(gridDim.x) * kQGroups;
         const int64_t first = blockIdx.x + static_cast<int64_t>(gridDim.x) * qg;
         float* gred = red + qg * 2 * kQWarps;
-        const uint64_t keep_l2 = l2_policy_evict_last();  // the codes ring stays in L2 until it is reused
+        // the codes ring stays in L2 until it is reused
+        const uint64_t keep_l2 = f.l2_hint ? l2_policy_evict_last() : l2_policy_evict_normal();
         uint32_t w[qcore::kRawWords];  // the next row's elements, loaded ahead
         if (holds && first < p.M) qcore::load_bf16_global(f.x + first * f.ldx, t, w);
         int it = 0;
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     } else if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------- producer (both CTAs)
-            const uint64_t keep_l2 = l2_policy_evict_last();
+            const uint64_t keep_l2 = f.l2_hint ? l2_policy_evict_last() : l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -405,7 +410,8 @@ cudaError_t launch_linear_fused(const uint16_t* x, int64_t ldx, const CUtensorMa
     f.ready = ready;
     f.started = ready + (g.M + kPanelRows - 1) / kPanelRows;
     f.loaded = f.started + 1;
-    f.ring = fused_ring_slots(g.M);
+    f.ring = fused_ring_slots(g.M, g.K);
+    f.l2_hint = fused_codes_l2_hint(g.K, g.N) ? 1 : 0;
     f.tpr = g.K / kPerThread;
     f.kind = kind;
     if (f.tpr > kQThreads || g.K % kPerThread != 0) return cudaErrorInvalidValue;
