@@ -111,14 +111,19 @@ int convrot_abi_version(void);
  * w: f32 [N][K] row-major.  block: a block value (see above).
  * Writes q: int8 [N][K] (K contiguous, "output-major") and s_w: f32 [N], and
  * fills *desc (HOST pointer) synchronously.  Requires K % 64 == 0,
- * K % b == 0, K <= 32768, N <= 2^31-1, 16-byte aligned pointers. */
+ * K % b == 0, K <= 32768, N <= 2^31-1, 16-byte aligned pointers.  Weights
+ * must be finite: a row holding inf or NaN is outside the contract (its codes
+ * and scale are unspecified; nothing checks them on the device). */
 convrot_status convrot_pack_weight(const float* w, int64_t N, int64_t K, int32_t block, int8_t* q,
                                    float* s_w, convrot_wdesc* desc, void* stream);
 
 /* Steps 1-2: x: bf16 [M][K] with row stride ldx (elements) ->
  * q: int8 [M][K] (contiguous) and s_x: f32 [M].  block: a block value.
  * Requires K % 64 == 0, K % b == 0, K <= 32768, ldx >= K, ldx % 8 == 0,
- * 0 < M <= 2^31-1.  A row of zeros gives s_x = 0 and zero codes. */
+ * 0 < M <= 2^31-1.  A row of zeros gives s_x = 0 and zero codes.  Inputs
+ * must be finite: a row holding inf or NaN is outside the contract (its codes
+ * and scale are unspecified; nothing checks them on the device).  The same
+ * holds for every entry point that quantises activations. */
 convrot_status convrot_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int32_t block,
                                     int8_t* q, float* s_x, void* stream);
 

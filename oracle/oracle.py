@@ -188,9 +188,17 @@ def quantize_rows(z: np.ndarray):
     return q, s
 
 
+def _require_finite_bf16(bits: np.ndarray, what: str) -> None:
+    """Non-finite inputs are outside the method's contract (the pages quantise
+    finite activations and weights only): refuse them rather than compute."""
+    if bool(((bits & 0x7F80) == 0x7F80).any()):
+        raise ValueError(f"{what}: non-finite bf16 input (inf or NaN) is outside the contract")
+
+
 def quantize_act(x_bits: np.ndarray, b: int, regular: bool = False):
     """bf16 activations (uint16 bits [M, K]) -> rotate (block b) -> (q, s_x)."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    _require_finite_bf16(x_bits, "quantize_act")
     M, K = x_bits.shape
     q = np.empty((M, K), dtype=np.int8)
     s = np.empty((M,), dtype=np.float32)
@@ -224,6 +232,7 @@ def act_quantize(h_bits: np.ndarray, act: int, b: int, regular: bool = False):
     """Activation prologue + rotation + rowwise int8: the down projection's
     (q, s_x) from the up projection's bf16 output h ([M, K] or [M, 2K])."""
     h_bits = np.ascontiguousarray(h_bits, dtype=np.uint16)
+    _require_finite_bf16(h_bits, "act_quantize")
     M = h_bits.shape[0]
     K = _act_width(h_bits, act)
     q = np.empty((M, K), dtype=np.int8)
@@ -235,6 +244,8 @@ def act_quantize(h_bits: np.ndarray, act: int, b: int, regular: bool = False):
 def pack_weight(w: np.ndarray, b: int, regular: bool = False):
     """f32 weights [N, K] -> rotate along K -> per-output-channel (q_w, s_w)."""
     w = np.ascontiguousarray(w, dtype=np.float32)
+    if not bool(np.isfinite(w).all()):
+        raise ValueError("pack_weight: non-finite weights (inf or NaN) are outside the contract")
     N, K = w.shape
     q = np.empty((N, K), dtype=np.int8)
     s = np.empty((N,), dtype=np.float32)
@@ -330,6 +341,7 @@ def attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, scale:
     1/sqrt(d) unless given; returns O fp64 [H, Lq, d] and the codes and
     scales (qx, sq, kx, sk)."""
     H, Lq, d = q_bits.shape
+    _require_finite_bf16(np.asarray(v_bits, dtype=np.uint16), "attention (v)")  # q, k: checked by the quantiser
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     qx, sq = quantize_act(q_bits.reshape(H * Lq, d), 0)
     kx, sk = quantize_act(k_bits.reshape(-1, d), 0)

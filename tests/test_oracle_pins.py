@@ -550,3 +550,27 @@ def test_attention_scores_are_the_dequantised_qk_product():
     S = O.dequant(O.igemm(qx[0], kx[0]), sq[0], sk[0], None, 0) * 0.5
     P = np.exp(S - S.max(1, keepdims=True)); P /= P.sum(1, keepdims=True)
     assert np.allclose(a1[0], P @ O.bf16_bits_to_f32(v[0]).astype(np.float64), rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------------ inputs outside the contract
+
+@pytest.mark.parametrize("bad", [0x7F80, 0xFF80, 0x7FC0, 0x7F81])  # +inf, -inf, quiet and signalling NaN
+def test_oracle_refuses_non_finite_bf16_inputs(bad):
+    x = np.full((3, 256), 0x3F80, dtype=np.uint16)  # 1.0
+    x[1, 77] = bad
+    with pytest.raises(ValueError):
+        O.quantize_act(x, 128)
+    with pytest.raises(ValueError):
+        O.act_quantize(x, O.ACT_GELU, 128)
+    # the largest finite bf16 magnitudes are inside the contract
+    x[1, 77] = 0x7F7F
+    q, s = O.quantize_act(x, 128)
+    assert np.isfinite(s).all() and np.abs(q).max() == 127
+
+
+@pytest.mark.parametrize("bad", [np.inf, -np.inf, np.nan])
+def test_oracle_refuses_non_finite_weights(bad):
+    w = np.ones((4, 128), dtype=np.float32)
+    w[2, 5] = bad
+    with pytest.raises(ValueError):
+        O.pack_weight(w, 128)
