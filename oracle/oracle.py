@@ -26,7 +26,7 @@ Every function cites the passage it follows (page title and section):
   matrix H_256 = H_4^(x)4") -- MiniMax-H3-Rung-Omega README, "Technical
   Architecture Overview", item 1.
 
-Readings where the pages are silent (all listed in the design doc): Sylvester
+Readings where the pages are silent: Sylvester
 order H[i][j] = (-1)^popcount(i & j); unnormalised transform with the 1/b
 folded into the dequantisation; fp32 butterflies in ascending stage order;
 s = amax/127 and q = rne(z * (127/amax)) in f32; a zero row has s = 0;
