@@ -77,6 +77,23 @@ def test_proj_768p_full_size():
     _check_outputs(y, qxr, sxr, qwr, swr, bias.numpy(), spec.block, rows, mi, ni, what="768p")
 
 
+def test_proj_768p_one_kernel_equals_two_kernels_bitwise():
+    # At 768p the one-kernel path's codes ring (12 panel slots for 151 panels)
+    # turns over 12 times; its output must equal the two-kernel path's
+    # (standalone quantiser into a full [M][K] array, then the GEMM) bit for bit.
+    spec = W.PROJ_768P
+    x, w, bias = W.linear_inputs(spec)
+    pw = C.pack_weight(w.cuda(), spec.block)
+    xd, bd = x.cuda(), bias.cuda()
+    y1 = C.linear_fused(xd, pw, bd)
+    q, s = C.quantize_act(xd, spec.block)
+    y2 = C.w8a8_linear(q, s, pw, bd)
+    torch.cuda.synchronize()
+    assert C.last_device_status() == (C.OK, 0)
+    differ = (y1.view(torch.int16) != y2.view(torch.int16)).sum().item()
+    assert differ == 0, f"{differ} of {y1.numel()} outputs differ"
+
+
 def test_proj_4k_full_size():
     spec = W.PROJ_4K
     x, w, bias = W.linear_inputs(spec)

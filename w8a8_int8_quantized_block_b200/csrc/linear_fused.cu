@@ -76,7 +76,7 @@ constexpr int kAStageF = kGemmBM * BK;
 constexpr int kBStageF = (BN / 2) * BK;
 constexpr int kSmemRingF = kStagesF * (kAStageF + kBStageF);
 constexpr int kSmemBarsF = 8 * (2 * kStagesF + 2 * kAccBufs) + 16;
-constexpr int kSmemRedF = kQGroups * 2 * kQWarps * 4;
+constexpr int kSmemRedF = kQGroups * 2 * kQWarps * 4 + kQGroups * 4;  // warp maxima, then one abort flag per group
 constexpr int kSmemTotalF = kSmemRingF + epi_smem(kEpiWarpsF, kEpiBufsF) + kSmemBarsF + kSmemRedF + 1024;
 static_assert(kSmemTotalF <= 227 * 1024, "shared memory budget");
 static_assert(kQThreads * kPerThread >= kFusedMaxK, "a group must cover a row");
@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     uint64_t* acce_bar = accf_bar + kAccBufs;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + kAccBufs);
     float* red = reinterpret_cast<float*>(tmem_slot + 4);  // [group][2][warp]
+    int* qabort = reinterpret_cast<int*>(red + kQGroups * 2 * kQWarps);  // [group]: a wait of the group gave up
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -141,6 +142,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             mbar_init(&accf_bar[a], 1);
             mbar_init(&acce_bar[a], 2 * kEpiWarpsF);
         }
+        for (int gq = 0; gq < kQGroups; ++gq) qabort[gq] = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -169,19 +171,28 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         if (holds && first < p.M) qcore::load_bf16_global(f.x + first * f.ldx, t, w);
         int it = 0;
         for (int64_t row = first; row < p.M; row += stride, ++it) {
-            // Keep within kPanelsAhead panels of the GEMM (every thread of the
-            // group waits, so the group stays in step).  The GEMM starts panels
-            // in order and each group quantises its rows in order, so every
-            // panel inside the window gets finished and the window moves on.
+            // Two waits before the row's codes may be written, both taken by
+            // thread 0 of the group alone; the group barrier below hands the
+            // outcome (and, through the barrier, the acquired counts) to all
+            // 96 threads, which then go on or leave together.  A thread that
+            // timed out on its own could otherwise leave the others stuck at
+            // that barrier.
+            //  - Keep within kPanelsAhead panels of the GEMM.  The GEMM starts
+            //    panels in order and each group quantises its rows in order, so
+            //    every panel inside the window gets finished and the window
+            //    moves on.
+            //  - The ring slot is free once every tile of its previous panel
+            //    has loaded it.
             const int panel = static_cast<int>(row / kPanelRows);
-            if (panel >= kPanelsAhead &&
-                !wait_count_bounded(f.started, static_cast<uint32_t>(panel - kPanelsAhead + 1), p.limit_ns,
-                                    kErrTimeoutPanel, p.err))
-                break;  // the error word is set; the GEMM side times out the same way
-            // the ring slot is free once every tile of its previous panel has loaded it
-            if (panel >= f.ring && !wait_count_bounded(f.loaded + (panel - f.ring), static_cast<uint32_t>(tiles_n),
-                                                       p.limit_ns, kErrTimeoutPanel, p.err))
-                break;
+            if (t == 0) {
+                bool ok = panel < kPanelsAhead ||
+                          wait_count_bounded(f.started, static_cast<uint32_t>(panel - kPanelsAhead + 1),
+                                             p.limit_ns, kErrTimeoutPanel, p.err);
+                ok = ok && (panel < f.ring || wait_count_bounded(f.loaded + (panel - f.ring),
+                                                                 static_cast<uint32_t>(tiles_n), p.limit_ns,
+                                                                 kErrTimeoutPanel, p.err));
+                if (!ok) qabort[qg] = 1;  // the error word is set; the GEMM side times out the same way
+            }
             const int64_t qrow = static_cast<int64_t>(panel % f.ring) * kPanelRows + (row - int64_t{panel} * kPanelRows);
             uint64_t P[kPairs];
             if (holds) {
@@ -197,7 +208,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             // so its bits order like the values.
             float amax = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(qcore::piece_absmax(P))));
             if (lane == 0) gred[(it & 1) * kQWarps + qw] = amax;
-            named_bar_sync(1 + qg, kQThreads);  // warp maxima published
+            named_bar_sync(1 + qg, kQThreads);  // warp maxima and thread 0's wait outcome published
+            if (qabort[qg]) break;              // the same value for every thread of the group
             amax = gred[(it & 1) * kQWarps];
             for (int i = 1; i < kQWarps; ++i) amax = fmaxf(amax, gred[(it & 1) * kQWarps + i]);
             if (holds) {

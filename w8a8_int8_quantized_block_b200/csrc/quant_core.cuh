@@ -124,13 +124,33 @@ __device__ __forceinline__ void load_pairs(const uint8_t* slot, int R0, int t, u
 }
 
 // ---- the activation prologue of the down projection
+//
+// The activation is evaluated in double precision and rounded once to f32,
+// operation by operation as the plain definition reads: the input (a bf16
+// value) is exact in double, the double erfc / exp are within a few units in
+// the 53-bit last place of the true value, so the f32 result is the correctly
+// rounded activation unless the exact value lies within about 2^-28 of an f32
+// rounding boundary.  (An f32 evaluation with erfcf / expf is off by several
+// f32 ulp, and in GELU's negative tail by far more, because rounding the
+// argument of erfc is amplified there; those errors moved codes across
+// rounding ties.)
 
 // gelu(x) = x Phi(x) = 0.5 x erfc(-x / sqrt 2) (the erfc form has no
-// cancellation for negative x).
-__device__ __forceinline__ float gelu_prologue(float x) { return 0.5f * x * erfcf(-0.70710678118654752f * x); }
+// cancellation for negative x).  0.5 x is exact; the quotient by the double
+// nearest sqrt 2 and the product are IEEE-rounded double operations.
+__device__ __forceinline__ float gelu_prologue(float x) {
+    const double v = static_cast<double>(x);
+    const double t = __ddiv_rn(-v, 1.4142135623730951);  // the double nearest sqrt(2)
+    return __double2float_rn(__dmul_rn(0.5 * v, erfc(t)));
+}
 
-// silu(g) = g / (1 + e^-g), IEEE division.
-__device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, 1.0f + expf(-g)); }
+// silu(g) * u = g / (1 + e^-g) * u in double (IEEE division and product),
+// rounded once to f32.
+__device__ __forceinline__ float swiglu_value(float g, float u) {
+    const double gd = static_cast<double>(g);
+    const double sg = __ddiv_rn(gd, __dadd_rn(1.0, exp(-gd)));
+    return __double2float_rn(__dmul_rn(sg, static_cast<double>(u)));
+}
 
 __device__ __forceinline__ void gelu_pairs(uint64_t (&P)[kPairs]) {
 #pragma unroll
@@ -157,8 +177,8 @@ __device__ __forceinline__ void swiglu_pairs(uint64_t (&P)[kPairs], const uint8_
             const int j = e & (kPairs - 1);
             float a, b;
             upk(P[j], a, b);
-            if (e < kPairs) a = silu(a) * u;
-            else b = silu(b) * u;
+            if (e < kPairs) a = swiglu_value(a, u);
+            else b = swiglu_value(b, u);
             P[j] = pk(a, b);
         }
     }
