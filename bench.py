@@ -2,10 +2,19 @@
 
 One step = one whole pass of the hot path over one batch: rotate + quantise
 the bf16 activations, int8 GEMM, dequantise with bias to bf16 (the weights
-are packed once, offline, as the pages' checkpoints are).  The workload is
-the full 768p projection, M = 38656 tokens, K = N = 5376, Hadamard block 128.
+are packed once, offline, as the pages' checkpoints are).  The headline
+workload is the full 768p projection, M = 38656 tokens, K = N = 5376,
+Hadamard block 128.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+The default run prints one JSON line: the headline (K back-to-back steps),
+each kernel of the step timed in its own back-to-back loop, a sustained leg
+(the same step for at least two seconds, under the power cap), the end-to-end
+leg through host buffers, the oracle's CPU baseline, and -- on one GPU -- a
+`configs` object with the other workloads (the tiny and 4096-token
+projections, the 768p MLP pair, the 42-head Q K^T GEMM and int8 attention),
+each with its roofline fraction and its own CPU baseline.
 
 Multi-GPU (torchrun): every rank runs its own full batch (token rows are
 independent; no collective on the data path), value = all ranks' work / the
@@ -34,7 +43,8 @@ GEMM_PROFILE = os.path.join(ROOT, "profiles", "linear_fused_proj_m38656_k5376_n5
 KERNEL_SOURCES = [os.path.join(ROOT, "w8a8_int8_quantized_block_b200", "csrc", f)
                   for f in ("linear_fused.cu", "gemm_core.cuh", "quant_core.cuh", "ptx.cuh", "kernels.h")]
 INT8_PER_BF16 = 2.0  # nominal dense ratio of 8-bit to bf16 tensor throughput (4.5 vs 2.25 PFLOP/s)
-FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_SUSTAINED = 6650.0, 1590.0, 1400.0
+L2_FLUSH_BYTES = 256 << 20  # written between timed calls of workloads that fit in the 126 MB L2
 
 
 REGULAR = 0x10000  # the C ABI's CONVROT_HADAMARD_REGULAR flag on a block value
@@ -86,18 +96,28 @@ def parse():
     ap.add_argument("--rows", type=int, default=None,
                     help="with --kernel-only: only the first ROWS token rows of the projection (a smaller case "
                          "of the same workload, for detailed profiler captures)")
-    ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm"], default=None,
+    ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm", "bmm", "mlp-down", "act"], default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
-                         "(for profiler captures; prints no result line)")
+                         "(for profiler captures; prints no result line).  bmm: the 42-head Q K^T GEMM "
+                         "(--heads for fewer); mlp-down: the MLP's down projection GEMM (K = 21504) on "
+                         "--rows rows; act: the GELU prologue quantiser of that projection")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' legs (the configs object of the default line)")
+    ap.add_argument("--sustained-seconds", type=float, default=2.0,
+                    help="length of the sustained leg (the headline step repeated under the power cap)")
+    ap.add_argument("--quant-launches", type=int, default=1000,
+                    help="back-to-back launches of the standalone quantiser in its own timed loop")
     return ap.parse_args()
 
 
 def peaks():
+    """(hbm GB/s, bf16 burst TFLOP/s, bf16 sustained TFLOP/s, source)."""
     try:
         p = json.load(open(PEAKS_FILE))
-        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+        bf16 = float(p["bf16_tflops"])
+        return float(p["hbm_gbs"]), bf16, float(p.get("bf16_tflops_sustained", bf16)), "measured"
     except (OSError, KeyError, ValueError):
-        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_SUSTAINED, "fallback"
 
 
 def kernel_hash() -> str:
@@ -292,18 +312,341 @@ def config_dict(spec, n, context_parallel=False):
                   "stay L2-resident across steps as they do when one layer serves many batches"}
 
 
-# ---------------------------------------------------------------------------- GPU path
+# ---------------------------------------------------------------------------- timing helpers
+
+
+IDLE_GAP_S = 1.0  # the GPU idles this long before each timed leg, so no leg inherits the power cap of the last
+
+
+def loop_time(fn, n: int, stream, world: int, clocks: bool = True, gap_s: float = IDLE_GAP_S):
+    """n back-to-back calls between two CUDA events on `stream` (a barrier and
+    a synchronize on both sides, after `gap_s` seconds of idle GPU); returns
+    (slowest rank's seconds per call, NVML clock summary of the region or None)."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    time.sleep(gap_s)
+    clk = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if clk:
+        clk.__enter__()
+    try:
+        barrier()
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        barrier()
+    finally:
+        if clk:
+            clk.__exit__()
+    return max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / n, (clk.summary() if clk else None)
+
+
+def graph_time(fn, calls: int, reps: int):
+    """Device time of one call when `calls` calls are replayed from one CUDA
+    graph (no host launch cost between them): fn(stream) enqueues one call."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(calls):
+            fn(s)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(reps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / (reps * calls)
+    del g
+    return t
+
+
+def cold_time(fn, n: int, stream, flush):
+    """Mean device time of one call with the L2 flushed before each (the flush
+    is outside the events): for workloads small enough to sit in L2."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / n / 1e3
+
+
+def check_status(C, where: str):
+    st, code = C.last_device_status()
+    if st != C.OK:
+        raise RuntimeError(f"device status {st} (code {code}) {where}")
+
+
+def grow_sample(run, start: int, limit: int, target_s: float):
+    """Grow a row sample until one timed oracle pass takes about target_s;
+    returns (rows, seconds)."""
+    rows = start
+    t = run(rows)
+    while t < 0.5 * target_s and rows < limit:
+        rows = int(min(limit, max(2 * rows, round(rows * target_s / max(t, 1e-3)))))
+        t = run(rows)
+    return rows, t
+
+
+# ---------------------------------------------------------------------------- other workloads
+
+
+def measure_tiny(args, world, stream, flush, peak_i8):
+    """The tiny projection (M = 256, K = N = 512): one fused call, latency-bound."""
+    import numpy as np
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+    spec = W.TINY
+    x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
+    x, bias = x_cpu.cuda(), b_cpu.cuda()
+    pw = C.pack_weight(w_cpu.cuda(), spec.block)
+    ws = C.alloc_workspace(spec.M, spec.K)
+    import torch
+    y = torch.empty(spec.M, spec.N, dtype=torch.bfloat16, device="cuda")
+    call = lambda st: C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=st)
+    step = lambda: call(stream)
+    for _ in range(5):
+        step()
+    t_cold = cold_time(step, 50, stream, flush)
+    t_warm, clk = loop_time(step, 500, stream, world)
+    t_graph = graph_time(call, 100, 20)
+    check_status(C, "after the tiny projection")
+    out = {"workload": spec.name, "us": t_graph * 1e6, "TOPS": spec.ops / t_graph / 1e12,
+           "frac_of_int8_peak": spec.ops / t_graph / 1e12 / peak_i8,
+           "us_direct_calls": t_warm * 1e6, "us_cold": t_cold * 1e6,
+           "bound": "latency: 0.13 GOP is one 256-row panel of two column tiles, so 2 of 74 CTA pairs work and "
+                    "the call is the one-kernel path's fill and drain plus the launch",
+           "timing": "us: device time per call with 100 calls replayed from one CUDA graph (20 replays); "
+                     "us_direct_calls: 500 calls from the host in a row (host launch cost included); "
+                     "us_cold: mean of 50 direct calls with the L2 flushed before each",
+           "clocks": clk}
+    if not args.no_cpu_baseline:
+        from oracle import oracle as O
+        xb, qw_sw = O.bf16_bits(x_cpu), oracle_pack(w_cpu.numpy(), spec.block)
+        b = b_cpu.numpy().astype(np.float32)
+        reps, t = 0, 0.0
+        while t < 1.0:
+            t += oracle_sample(xb, qw_sw[0], qw_sw[1], b, spec.M, spec.block)
+            reps += 1
+        out["cpu_baseline"] = {"value": reps * spec.ops / t / 1e12, "unit": UNIT, "cores": O.num_threads(),
+                               "kind": "oracle", "sample": f"the whole workload ({spec.M} rows), {reps} passes"}
+    return out
+
+
+def measure_proj4k(args, world, stream, flush, peak_i8):
+    """The 4096-token projection (K = N = 5376): tensor-bound, fits in L2."""
+    import numpy as np
+    import torch
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+    spec = W.PROJ_4K
+    x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
+    x, bias = x_cpu.cuda(), b_cpu.cuda()
+    pw = C.pack_weight(w_cpu.cuda(), spec.block)
+    ws = C.alloc_workspace(spec.M, spec.K)
+    y = torch.empty(spec.M, spec.N, dtype=torch.bfloat16, device="cuda")
+    step = lambda: C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream)
+    for _ in range(5):
+        step()
+    t_cold = cold_time(step, 50, stream, flush)
+    t_warm, clk = loop_time(step, 300, stream, world)
+    check_status(C, "after the 4096-token projection")
+    out = {"workload": spec.name, "us": t_cold * 1e6, "TOPS": spec.ops / t_cold / 1e12,
+           "frac_of_int8_peak": spec.ops / t_cold / 1e12 / peak_i8,
+           "us_back_to_back": t_warm * 1e6, "TOPS_back_to_back": spec.ops / t_warm / 1e12,
+           "bound": "tensor (2 M N K = 236.8 GOP; 16 x 21 tiles of 256 x 256 over 74 CTA pairs)",
+           "timing": "us: mean of 50 calls with the L2 flushed before each (x, y and the weights, 117 MB, "
+                     "would otherwise stay in the 126 MB L2); back_to_back: 300 calls in a row",
+           "clocks": clk}
+    if not args.no_cpu_baseline:
+        from oracle import oracle as O
+        xb = O.bf16_bits(x_cpu)
+        qw, sw = oracle_pack(w_cpu.numpy(), spec.block)
+        b = b_cpu.numpy().astype(np.float32)
+        rows, t = grow_sample(lambda r: oracle_sample(xb, qw, sw, b, r, spec.block), 16, spec.M, 5.0)
+        out["cpu_baseline"] = {"value": 2.0 * rows * spec.N * spec.K / t / 1e12, "unit": UNIT,
+                               "cores": O.num_threads(), "kind": "oracle",
+                               "sample": f"{rows} of {spec.M} token rows through the whole path in {t:.1f} s"}
+    return out
+
+
+MLP_METRIC = "ConvRot W8A8 MLP TOPS at M=38656, K=5376, H=21504 (up + GELU + down)"
+
+
+def measure_mlp(args, world, stream, peak_i8, steps: int, route_for_clocks: str = "epilogue"):
+    """The 768p MLP pair by both routes of its GELU: in the up projection's
+    epilogue (then the plain quantiser on the down projection's input), or as
+    the down projection's prologue (convrot_linear_act on the plain up
+    projection's output)."""
+    import numpy as np
+    import torch
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+
+    spec = W.MLP_768P
+    x_cpu, w1_cpu, w2_cpu = W.mlp_inputs(spec)
+    x = x_cpu.cuda()
+    p1 = C.pack_weight(w1_cpu.cuda(), spec.block)
+    p2 = C.pack_weight(w2_cpu.cuda(), spec.block)
+    ws1 = C.alloc_workspace(spec.M, spec.K)
+    ws2 = C.alloc_workspace(spec.M, spec.H)
+    h = torch.empty(spec.M, spec.H, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(spec.M, spec.K, dtype=torch.bfloat16, device="cuda")
+
+    def up(gelu):
+        C.linear_fused(x, p1, None, gelu=gelu, workspace=ws1, out=h, stream=stream)
+
+    def down(prologue):
+        if prologue:
+            C.linear_act(h, C.ACT_GELU, p2, None, workspace=ws2, out=y, stream=stream)
+        else:
+            C.linear_fused(h, p2, None, workspace=ws2, out=y, stream=stream)
+
+    routes = {"epilogue": (lambda: (up(True), down(False))), "prologue": (lambda: (up(False), down(True)))}
+    for r in routes.values():
+        for _ in range(2):
+            r()
+    times, kern, clocks = {}, {}, {}
+    for name, fn in routes.items():
+        times[name], clocks[name] = loop_time(fn, steps, stream, world)
+        nk = min(steps, 20)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nk)]
+        torch.cuda.synchronize()
+        for i in range(nk):
+            ev[i][0].record(stream)
+            up(name == "epilogue")
+            ev[i][1].record(stream)
+            down(name == "prologue")
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        kern[name] = {"up_us": sum(e[0].elapsed_time(e[1]) for e in ev) / nk * 1e3,
+                      "down_us": sum(e[1].elapsed_time(e[2]) for e in ev) / nk * 1e3}
+    check_status(C, "after the MLP")
+    t = times["epilogue"]
+    out = {"workload": spec.name, "route": "epilogue (GELU in the up projection's epilogue)",
+           "ms_per_step": t * 1e3, "TOPS": spec.ops / t / 1e12, "frac_of_int8_peak": spec.ops / t / 1e12 / peak_i8,
+           "bound": "tensor (17.9 TOP per step)",
+           "routes": {n: {"TOPS": spec.ops / times[n] / 1e12, "ms_per_step": times[n] * 1e3, **kern[n],
+                          "clocks": clocks[n]} for n in times},
+           "timing": f"{steps} steps back to back per route (inputs larger than L2: h is 1.66 GB)",
+           "clocks": clocks[route_for_clocks]}
+    del x, h, y, ws1, ws2, p1, p2
+    if not args.no_cpu_baseline:
+        from oracle import oracle as O
+        xb = O.bf16_bits(x_cpu)
+        q1, s1 = O.pack_weight(w1_cpu.numpy(), spec.block)
+        q2, s2 = O.pack_weight(w2_cpu.numpy(), spec.block)
+
+        def run(r):
+            t0 = time.perf_counter()
+            qx, sx = O.quantize_act(xb[:r], spec.block)
+            hh = O.dequant(O.igemm(qx, q1), sx, s1, None, spec.block, True)
+            hb = O.bf16_bits(torch.from_numpy(hh).to(torch.bfloat16))
+            qh, sh = O.quantize_act(hb, spec.block)
+            O.dequant(O.igemm(qh, q2), sh, s2, None, spec.block)
+            return time.perf_counter() - t0
+
+        rows, t = grow_sample(run, 4, spec.M, 5.0)
+        out["cpu_baseline"] = {"value": 4.0 * rows * spec.H * spec.K / t / 1e12, "unit": UNIT,
+                               "cores": O.num_threads(), "kind": "oracle",
+                               "sample": f"{rows} of {spec.M} token rows through both projections (GELU in "
+                                         f"fp64, bf16 between them) in {t:.1f} s"}
+    return out
+
+
+def measure_bmm(args, world, stream, hbm, peak_i8, steps: int):
+    """The skinny-K batched GEMM (42 heads, M = N = 8192, K = 128): quantise Q
+    and K per row (no rotation), then the GEMM writing 5.64 GB of bf16."""
+    import numpy as np
+    import torch
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+    spec = W.QK_BMM
+    q_cpu, k_cpu = W.bmm_inputs(spec)
+    B, M, N, K = spec.batch, spec.M, spec.N, spec.K
+    q, k = q_cpu.cuda().view(B * M, K), k_cpu.cuda().view(B * N, K)
+    qa = torch.empty(B * M, K, dtype=torch.int8, device="cuda")
+    qb = torch.empty(B * N, K, dtype=torch.int8, device="cuda")
+    sa = torch.empty(B * M, device="cuda")
+    sb = torch.empty(B * N, device="cuda")
+    y = torch.empty(B, M, N, dtype=torch.bfloat16, device="cuda")
+
+    def gemm():
+        C.w8a8_bmm(qa.view(B, M, K), sa, qb.view(B, N, K), sb, out=y, stream=stream)
+
+    def step():
+        C.quantize_act(q, 0, qa, sa, stream=stream)
+        C.quantize_act(k, 0, qb, sb, stream=stream)
+        gemm()
+
+    for _ in range(3):
+        step()
+    t_step, clk = loop_time(step, steps, stream, world)
+    t_gemm, clk_g = loop_time(gemm, steps, stream, world)
+    t_fill, _ = loop_time(lambda: y.fill_(1.0), steps, stream, world, clocks=False)
+    check_status(C, "after the Q K^T GEMM")
+    out_bytes = B * M * N * 2
+    gemm_bytes = out_bytes + (B * M + B * N) * (K + 4)
+    out = {"workload": spec.name, "us": t_step * 1e6, "TOPS": spec.ops / t_step / 1e12,
+           "gemm_us": t_gemm * 1e6, "gemm_TOPS": spec.ops / t_gemm / 1e12,
+           "gemm_GB/s": gemm_bytes / t_gemm / 1e9, "frac_of_hbm": gemm_bytes / t_gemm / 1e9 / hbm,
+           "hbm_peak_gbs": hbm, "algorithmic_bytes_per_launch": gemm_bytes,
+           "write_only_ceiling_gbs": out_bytes / t_fill / 1e9,
+           "frac_of_write_ceiling": (gemm_bytes / t_gemm) / (out_bytes / t_fill),
+           "bound": "HBM store (5.64 GB of bf16 out per step, 2 bytes per 256 ops)",
+           "timing": f"{steps} steps back to back (quantise Q, quantise K, GEMM); the GEMM alone likewise; "
+                     "write_only_ceiling: torch fill_ of the same 5.64 GB output, back to back",
+           "clocks": clk, "clocks_gemm": clk_g}
+    del q, k, qa, qb, sa, sb, y
+    if not args.no_cpu_baseline:
+        from oracle import oracle as O
+        qbits = O.bf16_bits(q_cpu[0])
+        kbits = O.bf16_bits(k_cpu[0])
+
+        def run(r):
+            t0 = time.perf_counter()
+            qx, sx = O.quantize_act(qbits[:r], 0)
+            kx, sk = O.quantize_act(kbits, 0)
+            O.dequant(O.igemm(qx, kx), sx, sk, None, 0)
+            return time.perf_counter() - t0
+
+        rows, t = grow_sample(run, 64, M, 5.0)
+        out["cpu_baseline"] = {"value": 2.0 * rows * N * K / t / 1e12, "unit": UNIT, "cores": O.num_threads(),
+                               "kind": "oracle",
+                               "sample": f"{rows} query rows of head 0 against its {N} keys (quantise, int64 "
+                                         f"GEMM, fp64 dequant) in {t:.1f} s"}
+    return out
 
 
 ATTN_METRIC = "int8 attention TFLOP/s at 42 heads x 8192 tokens, d=128 (Q K^T int8 + P V bf16)"
 
 
-def run_attention(args, rank: int, world: int):
+def measure_attention(args, world, stream, bf16, steps: int, heads=None):
     """int8 attention on the 42-head, 8192-token workload: the whole entry
     (quantise Q and K, transpose V, attend) and the attention kernel alone.
     Work = 2 H L^2 d int8 ops (Q K^T) + 2 H L^2 d bf16 flops (P V)."""
+    import numpy as np
     import torch
-    import torch.distributed as dist
     from w8a8_int8_quantized_block_b200 import convrot as C
     from w8a8_int8_quantized_block_b200 import workloads as W
 
@@ -311,16 +654,15 @@ def run_attention(args, rank: int, world: int):
     H, L, d = spec.batch, spec.M, spec.K
     q_cpu, k_cpu = W.bmm_inputs(spec)
     v_cpu = torch.randn(H, L, d, generator=torch.Generator().manual_seed(44)).to(torch.bfloat16)
-    if args.heads is not None:  # a smaller case of the same workload: its first heads
-        if not 1 <= args.heads <= H:
+    if heads is not None:  # a smaller case of the same workload: its first heads
+        if not 1 <= heads <= H:
             raise SystemExit(f"--heads must be in [1, {H}]")
-        H = args.heads
+        H = heads
         q_cpu, k_cpu, v_cpu = q_cpu[:H].contiguous(), k_cpu[:H].contiguous(), v_cpu[:H].contiguous()
     q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
     Lib = C.load()
     ws = torch.empty((Lib.convrot_attention_workspace_bytes(H, L, L),), dtype=torch.uint8, device="cuda")
     o = torch.empty(H, L, d, dtype=torch.bfloat16, device="cuda")
-    stream = torch.cuda.current_stream()
     r256 = lambda n: (n + 255) // 256 * 256
     off_sq = r256(H * L * d)
     off_kx = off_sq + r256(H * L * 4)
@@ -340,172 +682,154 @@ def run_attention(args, rank: int, world: int):
     main_units = units - units % sms if part_bytes else units
     attn_launches = (1 if main_units > 0 else 0) + (2 if part_bytes else 0)
 
-    def full():
-        C.attention(q, k, v, workspace=ws, out=o, stream=stream)
-
-    def kernel():
-        C.attention_int8(qx, sq, kx, sk, vt, out=o, stream=stream, split_ws=part)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    for _ in range(max(3, args.warmup)):
+    full = lambda: C.attention(q, k, v, workspace=ws, out=o, stream=stream)
+    kernel = lambda: C.attention_int8(qx, sq, kx, sk, vt, out=o, stream=stream, split_ws=part)
+    for _ in range(3):
         full()
-    barrier()
-    times = {}
-    clk_summary = None
-    for name, fn in (("kernel", kernel), ("full", full)):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(torch.cuda.current_device()) as clk:
-            barrier()
-            e0.record(stream)
-            for _ in range(args.steps):
-                fn()
-            e1.record(stream)
-            barrier()
-        times[name] = max_over_ranks(e0.elapsed_time(e1) / 1e3, world) / args.steps
-        if name == "kernel":
-            clk_summary = clk.summary()
-    st, code = C.last_device_status()
-    if st != C.OK:
-        raise RuntimeError(f"device status {st} (code {code})")
+    t_kernel, clk = loop_time(kernel, steps, stream, world)
+    t_full, clk_full = loop_time(full, steps, stream, world)
+    check_status(C, "after attention")
+    int8_peak = bf16 * INT8_PER_BF16
+    half = 2.0 * H * L * L * d          # each of the two products
+    ops = 2 * half
+    t_tensor = half / (int8_peak * 1e12) + half / (bf16 * 1e12)   # both products at their peaks
+    mufu = 16 * sms * 1.965e9                                      # 2^x per second (SFU, nominal)
+    t_exp = H * L * L / mufu
+    out = {"workload": f"attention_h{H}_l{L}_d{d}", "heads": H, "L": L, "d": d,
+           "ms": t_full * 1e3, "TFLOP/s": ops / t_full / 1e12,
+           "kernel_ms": t_kernel * 1e3, "kernel_TFLOP/s": ops / t_kernel / 1e12,
+           "frac_of_tensor_bound": t_tensor / t_kernel, "tensor_bound_ms": t_tensor * 1e3,
+           "exp2_bound_ms": t_exp * 1e3, "attn_launches": attn_launches,
+           "bound": f"tensor: Q K^T at bf16 burst x {INT8_PER_BF16}, P V at the bf16 burst {bf16} TFLOP/s; the "
+                    f"2^x of the softmax alone would take {t_exp * 1e3:.3f} ms on the special-function units "
+                    f"(nominal 16/clk/SM at 1965 MHz)",
+           "timing": f"{steps} calls back to back (the kernel on quantised inputs; the whole entry)",
+           "clocks": clk, "clocks_full": clk_full}
+    del q, k, v, ws, o
+    if not args.no_cpu_baseline:
+        from oracle import oracle as O
+        qx0, sq0 = O.quantize_act(O.bf16_bits(q_cpu[0]), 0)
+        kx0, sk0 = O.quantize_act(O.bf16_bits(k_cpu[0]), 0)
+        vb = O.bf16_bits(v_cpu[:1])
+
+        def run(r):
+            t0 = time.perf_counter()
+            O.attention_rows(qx0[None], sq0[None], kx0[None], sk0[None], vb, np.zeros(r, dtype=np.int64),
+                             np.arange(r), d ** -0.5)
+            return time.perf_counter() - t0
+
+        rows, t = grow_sample(run, 4, L, 4.0)
+        out["cpu_baseline"] = {"value": 4.0 * rows * L * d / t / 1e12, "unit": "TFLOP/s", "cores": O.num_threads(),
+                               "kind": "oracle",
+                               "sample": f"{rows} query rows of head 0 over all {L} keys (int64 scores, fp64 "
+                                         f"softmax and P V), in {t:.1f} s"}
+    return out, ops
+
+
+def run_attention(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+    stream = torch.cuda.current_stream()
+    hbm, bf16, bf16_sus, kind = peaks()
+    r, ops = measure_attention(args, world, stream, bf16, args.steps, args.heads)
     if rank == 0:
-        hbm, bf16, kind = peaks()
-        int8_peak = bf16 * INT8_PER_BF16
-        half = 2.0 * H * L * L * d          # each of the two products
-        ops = 2 * half
-        t_tensor = half / (int8_peak * 1e12) + half / (bf16 * 1e12)   # both products at their peaks
-        mufu = 16 * 148 * 1.965e9                                      # 2^x per second (SFU, nominal)
-        t_exp = H * L * L / mufu
-        value = world * ops / times["full"] / 1e12
+        value = world * ops / (r["ms"] / 1e3) / 1e12
         line = {
             "metric": ATTN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": times["full"] * 1e3, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
-            "config": {"workload": f"attention_h{H}_l{L}_d{d}", "heads": H, "Lq": L, "Lk": L, "d": d,
+            "config": {"workload": r["workload"], "heads": r["heads"], "Lq": r["L"], "Lk": r["L"], "d": r["d"],
                        "parallelism": f"dp{world} (independent heads and sequences per GPU)",
-                       "l2": f"Q, K, V are {H * L * d * 2 / 1e6:.0f} MB each (bf16), O the same"
-                             f"{'' if 4 * H * L * d * 2 > 126e6 else ' (together below L2: a small profiling case)'}; the score "
-                             f"matrix ({H * L * L * 2 / 1e9:.1f} GB as bf16) is never stored"},
-            "roofline": {"bound": "tensor",
-                         "kernel": f"attention_kernel (Q K^T, softmax, P V; {attn_launches} launch"
-                                   f"{'es: whole units, split units, combine' if attn_launches > 1 else ''})",
-                         "achieved": ops / times["kernel"] / 1e12, "peak": ops / t_tensor / 1e12,
-                         "unit": "TFLOP/s", "frac": t_tensor / times["kernel"], "traffic": None,
-                         "peak_source": f"{kind}: Q K^T at bf16 burst x {INT8_PER_BF16}, P V at the bf16 burst "
-                                        f"{bf16} TFLOP/s; the 2^x of the softmax alone would take "
-                                        f"{t_exp * 1e3:.3f} ms on the special-function units (nominal 16/clk/SM)"},
-            "kernels": {"attention_kernel_us": times["kernel"] * 1e6,
-                        "quantise_transpose_us": (times["full"] - times["kernel"]) * 1e6},
-            "clocks": clk_summary,
-            "gpu_launches": (3 + attn_launches) * args.steps,
+                       "l2": "Q, K, V and O are 88 MB each at 42 heads (bf16); the score matrix is never stored"},
+            "roofline": {"bound": "tensor", "kernel": f"attention_kernel ({r['attn_launches']} launch(es))",
+                         "achieved": r["kernel_TFLOP/s"], "peak": ops / (r["tensor_bound_ms"] / 1e3) / 1e12,
+                         "unit": "TFLOP/s", "frac": r["frac_of_tensor_bound"], "traffic": None,
+                         "peak_source": f"{kind}: {r['bound']}"},
+            "kernels": {"attention_kernel_us": r["kernel_ms"] * 1e3,
+                        "quantise_transpose_us": (r["ms"] - r["kernel_ms"]) * 1e3},
+            "clocks": r["clocks_full"],
+            "gpu_launches": (3 + r["attn_launches"]) * args.steps,
         }
+        if "cpu_baseline" in r:
+            line["cpu_baseline"] = r["cpu_baseline"]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
-MLP_METRIC = "ConvRot W8A8 MLP TOPS at M=38656, K=5376, H=21504 (up + GELU + down)"
-
-
 def run_mlp(args, rank: int, world: int):
-    """The 768p MLP step by both routes of its GELU: in the up projection's
-    epilogue (then the plain quantiser on the down projection's input), or as
-    the down projection's prologue (convrot_linear_act on the plain up
-    projection's output).  The line's value is for --mlp-route."""
+    """The MLP line; its value is for --mlp-route."""
     import torch
     import torch.distributed as dist
-    from w8a8_int8_quantized_block_b200 import convrot as C
     from w8a8_int8_quantized_block_b200 import workloads as W
-
-    spec = W.MLP_768P
-    x_cpu, w1_cpu, w2_cpu = W.mlp_inputs(spec)
-    x = x_cpu.cuda()
-    p1 = C.pack_weight(w1_cpu.cuda(), spec.block)
-    p2 = C.pack_weight(w2_cpu.cuda(), spec.block)
-    del w1_cpu, w2_cpu
-    ws1 = C.alloc_workspace(spec.M, spec.K)
-    ws2 = C.alloc_workspace(spec.M, spec.H)
-    h = torch.empty(spec.M, spec.H, dtype=torch.bfloat16, device="cuda")
-    y = torch.empty(spec.M, spec.K, dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
-
-    def up(gelu):
-        C.linear_fused(x, p1, None, gelu=gelu, workspace=ws1, out=h, stream=stream)
-
-    def down(prologue):
-        if prologue:
-            C.linear_act(h, C.ACT_GELU, p2, None, workspace=ws2, out=y, stream=stream)
-        else:
-            C.linear_fused(h, p2, None, workspace=ws2, out=y, stream=stream)
-
-    routes = {"epilogue": (lambda: (up(True), down(False))), "prologue": (lambda: (up(False), down(True)))}
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    for r in routes.values():
-        for _ in range(max(3, args.warmup)):
-            r()
-    barrier()
-    times, kern = {}, {}
-    clk_summary = None
-    for name in ("epilogue", "prologue"):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(torch.cuda.current_device()) as clk:
-            barrier()
-            e0.record(stream)
-            for _ in range(args.steps):
-                routes[name]()
-            e1.record(stream)
-            barrier()
-        times[name] = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-        if name == args.mlp_route:
-            clk_summary = clk.summary()
-        # per launch: up projection, then the down projection's two kernels
-        nk = min(args.steps, 50)
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nk)]
-        barrier()
-        for i in range(nk):
-            ev[i][0].record(stream)
-            up(name == "epilogue")
-            ev[i][1].record(stream)
-            down(name == "prologue")
-            ev[i][2].record(stream)
-        barrier()
-        kern[name] = {"up_us": sum(e[0].elapsed_time(e[1]) for e in ev) / nk * 1e3,
-                      "down_us": sum(e[1].elapsed_time(e[2]) for e in ev) / nk * 1e3}
-    st, code = C.last_device_status()
-    if st != C.OK:
-        raise RuntimeError(f"device status {st} (code {code})")
+    hbm, bf16, bf16_sus, kind = peaks()
+    int8_peak = bf16 * INT8_PER_BF16
+    r = measure_mlp(args, world, stream, int8_peak, args.steps, args.mlp_route)
     if rank == 0:
-        hbm, bf16, kind = peaks()
-        int8_peak = bf16 * INT8_PER_BF16
-        t = times[args.mlp_route]
-        value = job_tops(spec.ops, args.steps, world, t)
+        spec = W.MLP_768P
+        t = r["routes"][args.mlp_route]["ms_per_step"] / 1e3
+        value = job_tops(spec.ops, 1, world, t)
         line = {
             "metric": MLP_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "H": spec.H, "block": spec.block,
                        "activation": "gelu", "route": args.mlp_route,
                        "parallelism": f"dp{world} (independent token batches per GPU)",
                        "l2": "inputs larger than L2: h is 1.66 GB per step"},
             "pct_of_int8_peak": round(100.0 * value / world / int8_peak, 2),
-            "routes": {n: {"TOPS": job_tops(spec.ops, args.steps, world, times[n]),
-                           "ms_per_step": times[n] / args.steps * 1e3, **kern[n]} for n in times},
-            "clocks": clk_summary,
-            "gpu_launches": 3 * args.steps,  # up (one kernel), down (prologue quantiser + GEMM)
+            "routes": r["routes"],
+            "clocks": r["clocks"],
+            "gpu_launches": 3 * args.steps,  # up (one kernel), down (quantiser + GEMM)
         }
+        if "cpu_baseline" in r:
+            line["cpu_baseline"] = r["cpu_baseline"]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def kernel_only(args, spec, x, x_cpu, pw, bias, ws, y, stream):
+    """`--kernel-only`: launch one kernel warmup + steps times (profiler captures)."""
+    import torch
+    from w8a8_int8_quantized_block_b200 import convrot as C
+    from w8a8_int8_quantized_block_b200 import workloads as W
+    which = args.kernel_only
+    if which in ("fused", "quant", "gemm"):
+        q, s = ws[:spec.M * spec.K].view(torch.int8).view(spec.M, spec.K), torch.empty(spec.M, device="cuda")
+        C.quantize_act(x, spec.block, q, s, stream=stream)
+        one = {"fused": lambda: C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream),
+               "quant": lambda: C.quantize_act(x, spec.block, q, s, stream=stream),
+               "gemm": lambda: C.w8a8_linear(q, s, pw, bias, out=y, stream=stream)}[which]
+    elif which == "bmm":
+        bs = W.QK_BMM
+        B = bs.batch if args.heads is None else args.heads
+        qa = torch.randint(-127, 128, (B, bs.M, bs.K), dtype=torch.int8, device="cuda")
+        qb = torch.randint(-127, 128, (B, bs.N, bs.K), dtype=torch.int8, device="cuda")
+        sa, sb = torch.rand(B * bs.M, device="cuda"), torch.rand(B * bs.N, device="cuda")
+        yb = torch.empty(B, bs.M, bs.N, dtype=torch.bfloat16, device="cuda")
+        one = lambda: C.w8a8_bmm(qa, sa, qb, sb, out=yb, stream=stream)
+    else:  # the MLP's down projection (K = 21504) on the first --rows rows of its workload
+        ms = W.MLP_768P
+        rows = ms.M if args.rows is None else args.rows
+        g = torch.Generator(device="cuda").manual_seed(ms.seed)
+        h = (torch.randn(rows, ms.H, device="cuda", generator=g) * 2.0).to(torch.bfloat16)
+        w2 = torch.randn(ms.K, ms.H, device="cuda", generator=g) * ms.w_std
+        p2 = C.pack_weight(w2, ms.block)
+        del w2
+        q2 = torch.empty(rows, ms.H, dtype=torch.int8, device="cuda")
+        s2 = torch.empty(rows, device="cuda")
+        y2 = torch.empty(rows, ms.K, dtype=torch.bfloat16, device="cuda")
+        C.act_quantize(h, C.ACT_GELU, ms.block, q2, s2, stream=stream)
+        one = (lambda: C.w8a8_linear(q2, s2, p2, None, out=y2, stream=stream)) if which == "mlp-down" else \
+            (lambda: C.act_quantize(h, C.ACT_GELU, ms.block, q2, s2, stream=stream))
+    for _ in range(args.warmup + args.steps):
+        one()
+    torch.cuda.synchronize()
+    check_status(C, "after the kernel-only loop")
 
 
 def main():
@@ -532,10 +856,12 @@ def main():
         return run_mlp(args, rank, world)
     spec = workload(args)
     x_cpu, w_cpu, b_cpu = W.linear_inputs(spec)
-    if args.rows is not None:
+    if args.rows is not None and not args.kernel_only:
+        raise SystemExit("--rows needs --kernel-only")
+    if args.rows is not None and args.kernel_only in ("fused", "quant", "gemm"):
         import dataclasses
-        if not args.kernel_only or not 1 <= args.rows <= spec.M:
-            raise SystemExit(f"--rows needs --kernel-only and 1 <= ROWS <= {spec.M}")
+        if not 1 <= args.rows <= spec.M:
+            raise SystemExit(f"--rows must be in [1, {spec.M}]")
         spec = dataclasses.replace(spec, M=args.rows, name=f"{spec.name}_rows{args.rows}")
         x_cpu = x_cpu[:args.rows].contiguous()
     job = spec  # the whole job's tokens
@@ -550,8 +876,10 @@ def main():
     pw = C.pack_weight(w_cpu.cuda(), spec.block)
     ws = C.alloc_workspace(spec.M, spec.K)
     y = torch.empty(spec.M, spec.N, dtype=torch.bfloat16, device="cuda")
-    q, s = ws[:spec.M * spec.K].view(torch.int8).view(spec.M, spec.K), torch.empty(spec.M, device="cuda")
     stream = torch.cuda.current_stream()
+
+    if args.kernel_only:
+        return kernel_only(args, spec, x, x_cpu, pw, bias, ws, y, stream)
 
     def barrier():
         if world > 1:
@@ -570,83 +898,72 @@ def main():
         def step():
             C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream)
 
-    if args.kernel_only:
-        C.quantize_act(x, spec.block, q, s, stream=stream)
-        one = {"fused": step,
-               "quant": lambda: C.quantize_act(x, spec.block, q, s, stream=stream),
-               "gemm": lambda: C.w8a8_linear(q, s, pw, bias, out=y, stream=stream)}[args.kernel_only]
-        for _ in range(args.warmup + args.steps):
-            one()
-        torch.cuda.synchronize()
-        st, code = C.last_device_status()
-        if st != C.OK:
-            raise RuntimeError(f"device status {st} (code {code})")
-        return
-
     for _ in range(max(3, args.warmup)):
         step()
     barrier()
-    st, code = C.last_device_status()
-    if st != C.OK:
-        raise RuntimeError(f"device status {st} (code {code}) after warm-up")
+    check_status(C, "after warm-up")
 
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        barrier()
-    elapsed_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-    st, code = C.last_device_status()
-    if st != C.OK:
-        raise RuntimeError(f"device status {st} (code {code}) after the timed region")
+    # ---- the headline: K steps back to back
+    per_step, clk_head = loop_time(step, args.steps, stream, world)
+    elapsed_s = per_step * args.steps
+    check_status(C, "after the timed region")
     if args.context_parallel:
         value = job.ops * args.steps / elapsed_s / 1e12  # strong scaling: the ranks share one job
     else:
         value = job_tops(spec.ops, args.steps, world, elapsed_s)
 
-    # Per-kernel durations, same stream, CUDA events around each launch: the
-    # one-kernel step (its ready-counter memset included), then the two
-    # kernels of the split path for comparison.
-    nk = min(args.steps, 200)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nk)]
-    barrier()
-    for i in range(nk):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-        C.quantize_act(x, spec.block, q, s, stream=stream)
-        ev[i][2].record(stream)
-        C.w8a8_linear(q, s, pw, bias, out=y, stream=stream)
-        ev[i][3].record(stream)
-    barrier()
-    t_fused = sum(e[0].elapsed_time(e[1]) for e in ev) / nk / 1e3
-    t_quant = sum(e[1].elapsed_time(e[2]) for e in ev) / nk / 1e3
-    t_gemm = sum(e[2].elapsed_time(e[3]) for e in ev) / nk / 1e3
+    # ---- each kernel of the step in its own back-to-back loop (CUDA events on
+    # the launching stream around the loop; x and y are larger than L2)
+    q, s = ws[:spec.M * spec.K].view(torch.int8).view(spec.M, spec.K), torch.empty(spec.M, device="cuda")
+    fused = lambda: C.linear_fused(x, pw, bias, workspace=ws, out=y, stream=stream)
+    quant = lambda: C.quantize_act(x, spec.block, q, s, stream=stream)
+    gemm = lambda: C.w8a8_linear(q, s, pw, bias, out=y, stream=stream)
+    nk = max(args.steps, 100)
+    t_fused, clk_fused = loop_time(fused, nk, stream, world)
+    for _ in range(3):
+        quant()
+    t_quant, clk_quant = loop_time(quant, args.quant_launches, stream, world)
+    t_gemm, clk_gemm = loop_time(gemm, nk, stream, world)
+    check_status(C, "after the per-kernel loops")
 
-    # End to end through the C ABI with host buffers (copies inside the timed region).
+    # ---- sustained: the same step for at least --sustained-seconds, under the power cap
+    n_sus = max(args.steps, int(args.sustained_seconds / max(per_step, 1e-6)) + 1)
+    t_sus, clk_sus = loop_time(step, n_sus, stream, world)
+    check_status(C, "after the sustained leg")
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     x_host = x_cpu.pin_memory()
     y_host = torch.empty(spec.M, spec.N, dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty_like(x)
+    e2e = lambda: C.linear_fused_host(x_host, pw, bias, False, x_dev, ws, y, y_host, stream=stream)
     for _ in range(2):
-        C.linear_fused_host(x_host, pw, bias, False, x_dev, ws, y, y_host, stream=stream)
-    barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        C.linear_fused_host(x_host, pw, bias, False, x_dev, ws, y, y_host, stream=stream)
-    e1.record(stream)
-    barrier()
-    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-    e2e_value = job_tops(spec.ops, args.e2e_steps, world, e2e_s)
-    st, code = C.last_device_status()
-    if st != C.OK:
-        raise RuntimeError(f"device status {st} (code {code}) after the end-to-end leg")
+        e2e()
+    e2e_per, _ = loop_time(e2e, args.e2e_steps, stream, world, clocks=False)
+    e2e_value = job_tops(spec.ops, 1, world, e2e_per)
+    check_status(C, "after the end-to-end leg")
+    del x_host, y_host, x_dev
+
+    hbm, bf16, bf16_sus, kind = peaks()
+    int8_peak = bf16 * INT8_PER_BF16
+    int8_sus = bf16_sus * INT8_PER_BF16
+
+    # ---- the other workloads (one GPU)
+    configs = None
+    if world == 1 and not args.no_configs and not args.context_parallel:
+        del q, s
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        configs = {}
+        configs["tiny"] = measure_tiny(args, world, stream, flush, int8_peak)
+        configs["proj_4k"] = measure_proj4k(args, world, stream, flush, int8_peak)
+        del flush
+        configs["mlp"] = measure_mlp(args, world, stream, int8_peak, max(5, min(args.steps, 20)))
+        torch.cuda.empty_cache()
+        configs["qk_bmm"] = measure_bmm(args, world, stream, hbm, int8_peak, max(5, min(args.steps, 20)))
+        torch.cuda.empty_cache()
+        configs["attention"], _ = measure_attention(args, world, stream, bf16, max(5, min(args.steps, 20)))
+        torch.cuda.empty_cache()
 
     if rank == 0:
-        hbm, bf16, kind = peaks()
-        int8_peak = bf16 * INT8_PER_BF16
         achieved = spec.ops / t_fused / 1e12
         quant_bytes = spec.M * spec.K * 3 + spec.M * 4
         line = {
@@ -662,19 +979,30 @@ def main():
                          "peak_source": f"{kind} bf16 burst {bf16} TFLOP/s x {INT8_PER_BF16} (nominal int8:bf16)",
                          "algorithmic_ops_per_launch": spec.ops},
             "kernels": {
-                "linear_fused_kernel": {"us": t_fused * 1e6, "TOPS": achieved, "frac_of_int8_peak": achieved / int8_peak},
+                "linear_fused_kernel": {"us": t_fused * 1e6, "TOPS": achieved, "frac_of_int8_peak": achieved / int8_peak,
+                                        "launches": nk, "clocks": clk_fused},
                 "igemm_pair_kernel (split path)": {"us": t_gemm * 1e6, "TOPS": spec.ops / t_gemm / 1e12,
-                                                   "frac_of_int8_peak": spec.ops / t_gemm / 1e12 / int8_peak},
-                "rotate_quant_kernel (split path)": {"us": t_quant * 1e6, "GB/s": quant_bytes / t_quant / 1e9,
-                                 "frac_of_hbm": quant_bytes / t_quant / 1e9 / hbm, "hbm_peak_gbs": hbm,
-                                 "algorithmic_bytes_per_launch": quant_bytes},
+                                                   "frac_of_int8_peak": spec.ops / t_gemm / 1e12 / int8_peak,
+                                                   "launches": nk, "clocks": clk_gemm},
+                "rotate_quant_kernel": {"us": t_quant * 1e6, "GB/s": quant_bytes / t_quant / 1e9,
+                                        "frac_of_hbm": quant_bytes / t_quant / 1e9 / hbm, "hbm_peak_gbs": hbm,
+                                        "algorithmic_bytes_per_launch": quant_bytes,
+                                        "launches": args.quant_launches, "clocks": clk_quant,
+                                        "timing": "back-to-back launches between two CUDA events"},
             },
-            "clocks": clk.summary(),
+            "sustained": {"ms_per_step": t_sus * 1e3, "steps": n_sus, "seconds": t_sus * n_sus,
+                          "TOPS": job_tops(spec.ops, 1, world, t_sus),
+                          "frac": spec.ops / t_sus / 1e12 / int8_sus, "peak": int8_sus,
+                          "peak_source": f"{kind} bf16 sustained {bf16_sus} TFLOP/s x {INT8_PER_BF16}",
+                          "clocks": clk_sus},
+            "clocks": clk_head,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": spec.M * spec.K * 2,
                     "d2h_bytes_per_step": spec.M * spec.N * 2, "steps": args.e2e_steps,
                     "path": "convrot_linear_fused_host (pinned host x -> device -> linear -> pinned host y)"},
-            "gpu_launches": args.steps,  # one linear_fused_kernel per step (plus a 604-byte memset node)
+            "gpu_launches": args.steps,  # one linear_fused_kernel per step (plus a memset node of its counters)
         }
+        if configs is not None:
+            line["configs"] = configs
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(spec)
         print(json.dumps(line), flush=True)

@@ -135,20 +135,33 @@ convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int
                                    const convrot_wdesc* desc, const float* bias, int32_t epilogue, int64_t M,
                                    uint16_t* y, int64_t ldy, void* stream);
 
-/* Bytes of device workspace convrot_linear_fused needs: the int8 codes
- * (M*K, rounded up to 256), the scales (4*M, rounded up to 256) and the
- * one-kernel path's counters (4 * (2 * ceil(M/256) + 1), rounded up to 256). */
+/* Workspace of the linear entry points (convrot_linear_fused, _act, _host).
+ * Layout, each region starting on a 256-byte boundary:
+ *   scales    f32 [M]                                        at byte 0
+ *   counters  uint32 [2 ceil(M/256) + 1] (one-kernel path)   after the scales
+ *   codes     int8, last: the whole [M][K] array on the two-kernel path, or
+ *             a ring of min(M, R * 256) rows on the one-kernel path (R = 12
+ *             panel slots at K = 5376; R * 256 * K is about 16.5 MB, 4 <= R
+ *             <= 12), reused as the tensor cores finish each panel.
+ * convrot_workspace_bytes: enough for either path (the whole codes array).
+ * convrot_fused_workspace_bytes: enough for the one-kernel path alone, which
+ * convrot_linear_fused takes when K % 128 == 0, 128 <= K <= 6144, x is
+ * 32-byte aligned and ldx % 16 == 0 (about 17 MB instead of 208 MB at
+ * M = 38656, K = 5376); for other K it equals convrot_workspace_bytes.
+ * Both return 0 for M <= 0 or K <= 0. */
 size_t convrot_workspace_bytes(int64_t M, int64_t K);
+size_t convrot_fused_workspace_bytes(int64_t M, int64_t K);
 
 /* The whole linear, steps 1-4, on `stream`: one kernel (quantiser warps run
  * ahead of the tensor cores in the same CTAs) when K % 128 == 0, 128 <= K <=
  * 6144, x is 32-byte aligned and ldx % 16 == 0; otherwise two kernels (the
  * GEMM starts while the quantiser drains).  x: bf16 [M][K] (row stride ldx);
- * the codes and scales go to `workspace` (>= convrot_workspace_bytes(M, K)
- * bytes, 256-byte aligned, caller-owned, must not be shared by calls that
- * overlap).  The one-kernel path keeps the codes of at most 12 row panels of
- * 256 rows at a time (a ring, reused as the tensor cores finish each panel),
- * so after the call the workspace holds the scales of every row but not every
+ * the codes and scales go to `workspace` (256-byte aligned, caller-owned,
+ * must not be shared by calls that overlap) of at least the size of the path
+ * taken: convrot_fused_workspace_bytes(M, K) on the one-kernel path,
+ * convrot_workspace_bytes(M, K) on the two-kernel path (CONVROT_EINVAL with
+ * less).  The one-kernel path keeps only a ring of row panels' codes, so
+ * after the call the workspace holds the scales of every row but not every
  * row's codes. */
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw,
                                     const float* s_w, const convrot_wdesc* desc, const float* bias,
@@ -174,9 +187,10 @@ convrot_status convrot_act_quantize(const uint16_t* h, int64_t M, int64_t K, int
                                     int32_t block, int8_t* q, float* s_x, void* stream);
 
 /* The down projection with the activation prologue: convrot_act_quantize of
- * h into `workspace` (as convrot_linear_fused lays it out), then steps 3-4
- * with the packed weights (K = desc->K).  Two kernels on `stream`; the GEMM
- * starts while the prologue drains. */
+ * h into `workspace` (laid out as above, the whole codes array: at least
+ * convrot_workspace_bytes(M, desc->K) bytes), then steps 3-4 with the packed
+ * weights (K = desc->K).  Two kernels on `stream`; the GEMM starts while the
+ * prologue drains. */
 convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int32_t act, const int8_t* qw,
                                   const float* s_w, const convrot_wdesc* desc, const float* bias, int32_t epilogue,
                                   void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy, void* stream);
@@ -223,7 +237,8 @@ convrot_status convrot_attention_int8(const int8_t* qx, const float* s_q, const 
  * in host memory: copies x_host (bf16 [M][K], contiguous; pinned for overlap)
  * into the caller's device buffer x_dev, runs the fused linear into y_dev
  * (bf16 [M][N], contiguous) and copies it back to y_host.  The workspace is
- * that of convrot_linear_fused (>= convrot_workspace_bytes(M, K)).  Rows of
+ * that of convrot_linear_fused for the largest chunk of rows it is called on
+ * (convrot_workspace_bytes(M, K) is always enough).  Rows of
  * more than ~32 MiB of input run in chunks whose copy in, compute and copy
  * out overlap: the copies go on two streams the library owns (one per
  * direction and device), ordered by events, and `stream` waits for the last
@@ -243,9 +258,12 @@ convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, cons
  * The caller still passes x and y exactly as for convrot_linear_fused; the
  * int8 codes and scales go to a scratch array built into the library instead
  * of a caller workspace.  That array is 32 MiB per device, held by every GPU
- * that loads the library until the process exits: the call accepts
- * convrot_workspace_bytes(M, desc->K) <= 33554432 (M <= 6236 at K = 5376) and
- * returns CONVROT_ETOOLARGE, launching nothing, beyond that.
+ * that loads the library until the process exits: the call accepts problems
+ * whose workspace on the path convrot_linear_fused would take fits in
+ * 33554432 bytes (convrot_fused_workspace_bytes on the one-kernel path: M up
+ * to about 4.2 million rows at K = 5376; convrot_workspace_bytes on the
+ * two-kernel path: M <= 6236 at K = 5376, M <= 1560 at K = 21504) and returns
+ * CONVROT_ETOOLARGE, launching nothing, beyond that.
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
  * All calls share the one array and it keeps the previous call's contents

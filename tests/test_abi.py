@@ -38,11 +38,30 @@ def test_abi_version_and_status_strings():
 
 def test_workspace_bytes():
     L = C.load()
-    # codes, scales, and two counters per 256-row panel plus one, each rounded to 256 bytes
+    # scales, two counters per 256-row panel plus one, then the codes, each
+    # rounded to 256 bytes; the codes are the whole [M][K] array (either path)
+    # or the one-kernel path's ring of min(M, slots * 256) rows
     r = lambda v: (v + 255) // 256 * 256
-    assert L.convrot_workspace_bytes(38656, 5376) == 38656 * 5376 + r(38656 * 4) + r((2 * 151 + 1) * 4)
+    head = r(38656 * 4) + r((2 * 151 + 1) * 4)
+    assert L.convrot_workspace_bytes(38656, 5376) == head + 38656 * 5376
+    assert L.convrot_fused_workspace_bytes(38656, 5376) == head + 12 * 256 * 5376   # 12 slots, ~17 MB
+    assert L.convrot_fused_workspace_bytes(38656, 6144) == r(38656 * 4) + r(303 * 4) + 10 * 256 * 6144
+    assert L.convrot_fused_workspace_bytes(38656, 512) == r(38656 * 4) + r(303 * 4) + 12 * 256 * 512
+    assert L.convrot_fused_workspace_bytes(38656, 21504) == L.convrot_workspace_bytes(38656, 21504)  # two kernels
+    assert L.convrot_fused_workspace_bytes(1000, 5376) == L.convrot_workspace_bytes(1000, 5376)  # 4 panels fit
+    assert L.convrot_fused_workspace_bytes(3073, 5376) == r(3073 * 4) + r(27 * 4) + 12 * 256 * 5376
     assert L.convrot_workspace_bytes(1, 128) == 256 + 256 + 256
-    assert L.convrot_workspace_bytes(0, 128) == 0
+    assert L.convrot_workspace_bytes(0, 128) == 0 and L.convrot_fused_workspace_bytes(0, 128) == 0
+
+
+def test_noalloc_limits_follow_the_path():
+    # the allocation-free entry point's 32 MiB scratch holds the workspace of
+    # the path taken: the whole codes array on the two-kernel path, the ring on
+    # the one-kernel path
+    L, lim = C.load(), 32 << 20
+    assert L.convrot_workspace_bytes(6236, 5376) <= lim < L.convrot_workspace_bytes(6237, 5376)
+    assert L.convrot_workspace_bytes(1560, 21504) <= lim < L.convrot_workspace_bytes(1561, 21504)
+    assert L.convrot_fused_workspace_bytes(4_000_000, 5376) <= lim < L.convrot_fused_workspace_bytes(4_300_000, 5376)
 
 
 FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: validation fails first

@@ -101,9 +101,8 @@ def test_down_projection_with_prologue_matches_oracle(act):
     qw, sw = O.pack_weight(w.numpy(), 64)
     yr = O.dequant(O.igemm(qr, qw), sr, sw, bias.numpy(), 64)
     assert_close_bf16(f32_of_bf16(y), yr, "down projection with prologue")
-    qx = ws[:M * K].view(torch.int8).view(M, K).cpu().numpy()
-    off = (M * K + 255) // 256 * 256
-    sx = ws[off:off + 4 * M].view(torch.float32).cpu().numpy()
+    qx = C.workspace_codes(ws, M, K).cpu().numpy()
+    sx = C.workspace_scales(ws, M).cpu().numpy()
     assert_prologue_codes(qx, sx, h, act, 64)
 
 
@@ -155,9 +154,8 @@ def test_mlp_down_prologue_full_size():
     y = C.linear_act(h, C.ACT_GELU, pw2, None, workspace=ws)
     torch.cuda.synchronize()
     assert C.last_device_status() == (C.OK, 0)
-    q = ws[:spec.M * spec.H].view(torch.int8).view(spec.M, spec.H)
-    off = (spec.M * spec.H + 255) // 256 * 256
-    s = ws[off:off + 4 * spec.M].view(torch.float32)
+    q = C.workspace_codes(ws, spec.M, spec.H)
+    s = C.workspace_scales(ws, spec.M)
     h_cpu = h.cpu()
     del h
     differ = _check_rows_in_chunks(q, s, h_cpu, C.ACT_GELU, spec.block)

@@ -87,9 +87,8 @@ def test_linear_every_rotation_matches_oracle(block, fused):
     assert_close_bf16(f32_of_bf16(y), yr, f"linear {_ids(block)}")
     if fused:
         # the one-kernel path leaves its codes in the workspace: exact too
-        qx = ws[:M * K].view(torch.int8).view(M, K).cpu().numpy()
-        off = (M * K + 255) // 256 * 256
-        sx = ws[off:off + 4 * M].view(torch.float32).cpu().numpy()
+        qx = C.workspace_codes(ws, M, K).cpu().numpy()
+        sx = C.workspace_scales(ws, M).cpu().numpy()
         assert np.array_equal(qx, qxr)
         assert np.array_equal(sx.view(np.uint32), sxr.view(np.uint32))
 

@@ -42,9 +42,12 @@ def _padding_intact(body: torch.Tensor, M: int, N: int, ldy: int, what: str):
     assert (rows[:, 2 * N:] == SENT).all(), f"{what}: bytes written into a row's padding"
 
 
-@pytest.mark.parametrize("M,K,N,ldx_pad", [(300, 640, 264, 0), (300, 640, 264, 8), (7000, 512, 72, 0)])
+@pytest.mark.parametrize("M,K,N,ldx_pad", [(300, 640, 264, 0), (300, 640, 264, 8), (7000, 512, 72, 0),
+                                            (3500, 5376, 264, 0)])
 def test_linear_fused_writes_stay_inside(M, K, N, ldx_pad):
-    # ldx_pad 0: the one-kernel path (7000 rows: its codes ring wraps); 8: the two-kernel path
+    # ldx_pad 0: the one-kernel path, in a workspace of exactly its own size
+    # (7000 and 3500 rows: its codes ring wraps, and the workspace is shorter
+    # than a whole codes array); 8: the two-kernel path in the full size
     spec, (x, w, bias) = W.custom_linear(M, K, N, seed=M + ldx_pad, n_out=2)
     xp = torch.zeros(M, K + ldx_pad, dtype=torch.bfloat16)
     xp[:, :K] = x
@@ -52,7 +55,7 @@ def test_linear_fused_writes_stay_inside(M, K, N, ldx_pad):
     pw = C.pack_weight(w.to(DEV), 128)
     ldy = N + 24
     ybuf, ybody, y = _strided_bf16(M, N, ldy)
-    nws = C.workspace_bytes(M, K)
+    nws = C.fused_workspace_bytes(M, K) if ldx_pad == 0 else C.workspace_bytes(M, K)
     wbuf, ws = _guarded(nws)
     C.linear_fused(xd, pw, bias.to(DEV), workspace=ws, out=y)
     torch.cuda.synchronize()

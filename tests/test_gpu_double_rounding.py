@@ -56,7 +56,7 @@ def test_pack_weight_double_rounding_exact():
 
 def test_one_kernel_linear_codes_double_rounding_exact():
     # The quantiser warps inside the one-kernel linear write the same codes to
-    # the workspace (codes [M][K] first).
+    # the workspace (every row's codes while the panels fit the ring).
     xr = rotated_rows()
     M, K = xr.shape
     x = torch.from_numpy(xr).to(torch.bfloat16)
@@ -67,8 +67,7 @@ def test_one_kernel_linear_codes_double_rounding_exact():
     torch.cuda.synchronize()
     assert C.last_device_status() == (C.OK, 0)
     qr, sr = O.quantize_act(bits(x), 128)
-    q = ws[:M * K].view(torch.int8).view(M, K).cpu().numpy()
-    off = (M * K + 255) // 256 * 256
-    s = ws[off:off + 4 * M].view(torch.float32).cpu().numpy()
+    q = C.workspace_codes(ws, M, K).cpu().numpy()
+    s = C.workspace_scales(ws, M).cpu().numpy()
     assert np.array_equal(q, qr)
     assert np.array_equal(s.view(np.uint32), sr.view(np.uint32))

@@ -43,19 +43,20 @@ def test_proj_768p_full_size():
     x, w, bias = W.linear_inputs(spec)
     pw = C.pack_weight(w.cuda(), spec.block)
     xd = x.cuda()
-    ws = C.alloc_workspace(spec.M, spec.K)
+    # the one-kernel path's own workspace size: scales, counters, then the
+    # codes ring (about 17 MB, not the 208 MB of a whole codes array)
+    ws = C.alloc_workspace(spec.M, spec.K, one_kernel_only=True)
+    assert ws.numel() < 20 << 20
     y = C.linear_fused(xd, pw, bias.cuda(), workspace=ws)
     torch.cuda.synchronize()
     assert C.last_device_status() == (C.OK, 0)
-    # workspace layout: the codes region ([M][K] bytes), then the scales, each
-    # rounded up to 256 bytes.  The one-kernel path keeps the codes of RING row
-    # panels of 256 at a time (panel p in slot p % RING), so after the call the
-    # slots hold the last RING panels; every row's scale is there.
-    off = (spec.M * spec.K + 255) // 256 * 256
-    sx = ws[off:off + spec.M * 4].view(torch.float32).cpu().numpy()
+    # The one-kernel path keeps the codes of RING row panels of 256 at a time
+    # (panel p in slot p % RING), so after the call the slots hold the last
+    # RING panels; every row's scale is there.
+    sx = C.workspace_scales(ws, spec.M).cpu().numpy()
     xb = bits(x)
     qxr, sxr = O.quantize_act(xb, spec.block)
-    ring = ws[:RING * 256 * spec.K].view(torch.int8).view(RING * 256, spec.K).cpu().numpy()
+    ring = C.workspace_codes(ws, spec.M, spec.K, rows=RING * 256).cpu().numpy()
     panels = (spec.M + 255) // 256
     qx = np.zeros_like(qxr)
     held = np.zeros(spec.M, dtype=bool)

@@ -16,7 +16,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libconvrot.so")
-SOURCES = ["api.cu", "rotate_quant.cu", "igemm_tcgen05.cu", "linear_fused.cu", "attention.cu"]
+SOURCES = ["api.cu", "rotate_quant.cu", "rotate_quant_block.cu", "igemm_tcgen05.cu", "linear_fused.cu",
+           "attention.cu"]
 HEADERS = ["ptx.cuh", "ptx_attn.cuh", "kernels.h", "attention.h", "quant_core.cuh", "gemm_core.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",

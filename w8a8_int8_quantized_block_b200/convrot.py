@@ -41,7 +41,7 @@ EXPORTS = (
     "convrot_w8a8_bmm", "convrot_igemm_s32", "convrot_last_device_status", "convrot_set_wait_limit_ns",
     "convrot_selftest_wait_timeout", "convrot_linear_fused_noalloc", "convrot_act_quantize", "convrot_linear_act",
     "convrot_attention_workspace_bytes", "convrot_attention", "convrot_attention_split_bytes",
-    "convrot_attention_int8",
+    "convrot_attention_int8", "convrot_fused_workspace_bytes",
 )
 
 
@@ -83,6 +83,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "convrot_quantize_act": ([P, I64, I64, I64, I32, P, P, P], ctypes.c_int),
         "convrot_w8a8_linear": ([P, P, P, P, ctypes.POINTER(WDesc), P, I32, I64, P, I64, P], ctypes.c_int),
         "convrot_workspace_bytes": ([I64, I64], ctypes.c_size_t),
+        "convrot_fused_workspace_bytes": ([I64, I64], ctypes.c_size_t),
         "convrot_linear_fused": ([P, I64, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, ctypes.c_size_t, P, I64, P],
                                  ctypes.c_int),
         "convrot_linear_fused_host": ([P, I64, P, P, ctypes.POINTER(WDesc), P, I32, P, P, ctypes.c_size_t, P, P, P],
@@ -272,12 +273,39 @@ def w8a8_linear(qx: torch.Tensor, sx: torch.Tensor, pw: PackedWeight, bias: torc
 
 
 def workspace_bytes(M: int, K: int) -> int:
+    """Workspace bytes for either path of linear_fused (the whole codes array)."""
     return int(load().convrot_workspace_bytes(M, K))
 
 
-def alloc_workspace(M: int, K: int, device=None) -> torch.Tensor:
-    """Caller-owned workspace for linear_fused (torch allocations are 512-byte aligned)."""
-    return torch.empty((workspace_bytes(M, K),), dtype=torch.uint8, device=device or "cuda")
+def fused_workspace_bytes(M: int, K: int) -> int:
+    """Workspace bytes for linear_fused's one-kernel path (its codes ring)."""
+    return int(load().convrot_fused_workspace_bytes(M, K))
+
+
+def alloc_workspace(M: int, K: int, device=None, one_kernel_only: bool = False) -> torch.Tensor:
+    """Caller-owned workspace for linear_fused (torch allocations are 512-byte
+    aligned); one_kernel_only: just the one-kernel path's size."""
+    n = fused_workspace_bytes(M, K) if one_kernel_only else workspace_bytes(M, K)
+    return torch.empty((n,), dtype=torch.uint8, device=device or "cuda")
+
+
+def _r256(n: int) -> int:
+    return (n + 255) // 256 * 256
+
+
+def workspace_scales(ws: torch.Tensor, M: int) -> torch.Tensor:
+    """The f32 [M] scales region of a linear workspace (it comes first)."""
+    return ws[:4 * M].view(torch.float32)
+
+
+def workspace_codes(ws: torch.Tensor, M: int, K: int, rows: int | None = None) -> torch.Tensor:
+    """The int8 codes region of a linear workspace as [rows, K] (default M
+    rows: the two-kernel path's whole array; the one-kernel path's ring holds
+    fewer).  It follows the scales and the one-kernel path's counters."""
+    panels = (M + 255) // 256
+    off = _r256(4 * M) + _r256(4 * (2 * panels + 1))
+    rows = M if rows is None else rows
+    return ws[off:off + rows * K].view(torch.int8).view(rows, K)
 
 
 def linear_fused(x: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None, gelu: bool = False,

@@ -35,6 +35,18 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
+struct LaunchFigure {
+    const void* kernel;
+    int dev;
+    int threads;
+    size_t smem;
+    int figure;
+};
+constexpr int kMaxLaunchFigures = 1024;
+LaunchFigure g_figures[kMaxLaunchFigures];
+int g_num_figures = 0;
+std::mutex g_figure_mutex;
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -85,6 +97,22 @@ bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint6
     return r == CUDA_SUCCESS;
 }
 
+// 4D tiled tensor map: dims {d0 (contiguous), d1, d2, d3}, byte strides of
+// dims 1-3 (any order: a view may visit memory out of its natural order), box
+// {b0, b1, b2, b3}.
+bool encode_4d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, const uint64_t (&dims)[4],
+               const uint64_t (&strides)[3], const uint32_t (&box)[4], CUtensorMapSwizzle sw) {
+    if (!encoder_ready()) return false;
+    cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+    cuuint64_t st[3] = {strides[0], strides[1], strides[2]};
+    cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    std::memset(map, 0, sizeof(*map));
+    CUresult r = g_encode(map, dt, 4, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 constexpr int64_t kMaxI32 = 2147483647;
@@ -132,6 +160,23 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
     const DeviceInfo* d = device_info();
     if (!d) return CONVROT_ECUDA;
     if (!d->supported) return CONVROT_EUNSUPPORTED;
+    // bf16 rows with the 128-point Sylvester rotation (or none) and K % 128 == 0:
+    // one whole Hadamard block per thread (fewer instructions per element).
+    RqbGeometry gb;
+    if (in_elem_bytes == 2 && act == CONVROT_ACT_NONE && (kind == kRotSyl128 || kind == kRotNone) &&
+        rqb_geometry(K, &gb)) {
+        CUtensorMap xmap4;
+        const uint64_t nb = static_cast<uint64_t>(K / 128);
+        // {64 elements, K/128 blocks, 2 halves, M rows}: the first halves of a
+        // row's blocks land in consecutive shared rows, then the second halves
+        if (!encode_4d(&xmap4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, {64, nb, 2, static_cast<uint64_t>(M)},
+                       {256, 128, static_cast<uint64_t>(ldx) * 2},
+                       {64, static_cast<uint32_t>(nb), 2, static_cast<uint32_t>(gb.rows_per_cta)},
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return CONVROT_ECUDA;
+        return cuda_status(launch_rotate_quant_block(xmap4, kind, M, gb, q, K, s, g_limit_ns.load(), d->err,
+                                                     d->num_sms, stream));
+    }
     RqGeometry g;
     if (!rq_geometry(K, row_elems, in_elem_bytes, &g)) return CONVROT_EINVAL;
     CUtensorMap xmap;
@@ -235,6 +280,42 @@ bool fused_eligible(int64_t K, int32_t block) {
     return decode_block(block, &b, &kind) && K % 128 == 0 && K >= 128 && K <= kFusedMaxK;
 }
 
+// Workspace of the linear entry points.  Every region starts on a 256-byte
+// boundary:
+//   scales    f32 [M]                                         at 0
+//   counters  u32 [2 ceil(M/256) + 1] of the one-kernel path  after the scales
+//   codes     int8: the whole [M][K] array (two-kernel path), or the ring of
+//             min(M, fused_ring_slots(M, K) * 256) rows (one-kernel path)
+// The codes come last, so the two paths differ only in the workspace's length.
+struct WsLayout {
+    size_t counters;  // byte offset of the counters
+    size_t codes;     // byte offset of the codes
+    size_t full;      // bytes with the whole [M][K] codes array
+    size_t ring;      // bytes with the one-kernel path's ring of codes
+};
+
+WsLayout ws_layout(int64_t M, int64_t K) {
+    WsLayout l;
+    const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
+    l.counters = round256(static_cast<size_t>(M) * 4);
+    l.codes = l.counters + round256((2 * panels + 1) * 4);
+    l.full = l.codes + round256(static_cast<size_t>(M) * static_cast<size_t>(K));
+    const int64_t ring_rows = std::min<int64_t>(M, int64_t{fused_ring_slots(M, K)} * 2 * kGemmBM);
+    l.ring = l.codes + round256(static_cast<size_t>(ring_rows) * static_cast<size_t>(K));
+    return l;
+}
+
+// Whether convrot_linear_fused takes the one-kernel path for these rows.
+bool takes_one_kernel(const void* x, int64_t ldx, const convrot_wdesc* desc) {
+    return fused_eligible(desc->K, desc->block) && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && ldx % 16 == 0;
+}
+
+// Workspace bytes convrot_linear_fused needs on the path it takes.
+size_t linear_ws_needed(const void* x, int64_t M, int64_t ldx, const convrot_wdesc* desc) {
+    const WsLayout l = ws_layout(M, desc->K);
+    return takes_one_kernel(x, ldx, desc) ? l.ring : l.full;
+}
+
 convrot_status linear_one_kernel(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
                                  const convrot_wdesc* desc, const float* bias, int epi, int8_t* qx, float* sx,
                                  unsigned int* ready, uint16_t* y, int64_t ldy, cudaStream_t stream) {
@@ -317,6 +398,28 @@ HostPipe* host_pipe() {
 }
 
 }  // namespace
+
+bool launch_figure_get(const void* kernel, int threads, size_t smem, int* figure) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(g_figure_mutex);
+    for (int i = 0; i < g_num_figures; ++i) {
+        const LaunchFigure& f = g_figures[i];
+        if (f.kernel == kernel && f.dev == dev && f.threads == threads && f.smem == smem) {
+            *figure = f.figure;
+            return true;
+        }
+    }
+    return false;
+}
+
+void launch_figure_put(const void* kernel, int threads, size_t smem, int figure) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return;
+    std::lock_guard<std::mutex> lock(g_figure_mutex);
+    if (g_num_figures < kMaxLaunchFigures) g_figures[g_num_figures++] = LaunchFigure{kernel, dev, threads, smem, figure};
+}
+
 }  // namespace convrot
 
 using namespace convrot;
@@ -372,9 +475,13 @@ convrot_status convrot_w8a8_linear(const int8_t* qx, const float* s_x, const int
 
 size_t convrot_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
-    const size_t panels = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM));
-    return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) + round256(static_cast<size_t>(M) * 4) +
-           round256((2 * panels + 1) * 4);
+    return ws_layout(M, K).full;
+}
+
+size_t convrot_fused_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    const WsLayout l = ws_layout(M, K);
+    return (K % 128 == 0 && K >= 128 && K <= kFusedMaxK) ? l.ring : l.full;
 }
 
 convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, const int8_t* qw, const float* s_w,
@@ -382,19 +489,19 @@ convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, c
                                     void* workspace, size_t ws_bytes, uint16_t* y, int64_t ldy, void* stream) {
     convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y, ldy, bias);
     if (st != CONVROT_OK) return st;
+    if (!x || !aligned16(x) || ldx < desc->K || ldx % 8 != 0) return CONVROT_EINVAL;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CONVROT_EINVAL;
-    if (ws_bytes < convrot_workspace_bytes(M, desc->K)) return CONVROT_EINVAL;
-    int8_t* qx = static_cast<int8_t*>(workspace);
-    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                         round256(static_cast<size_t>(M) * static_cast<size_t>(desc->K)));
-    unsigned int* ready = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(sx) +
-                                                          round256(static_cast<size_t>(M) * 4));
+    if (ws_bytes < linear_ws_needed(x, M, ldx, desc)) return CONVROT_EINVAL;
+    const WsLayout l = ws_layout(M, desc->K);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    float* sx = reinterpret_cast<float*>(w);
+    unsigned int* ready = reinterpret_cast<unsigned int*>(w + l.counters);
+    int8_t* qx = reinterpret_cast<int8_t*>(w + l.codes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int epi = epilogue == CONVROT_EPI_GELU ? kEpiBf16Gelu : kEpiBf16;
-    if (!x || !aligned16(x) || ldx < desc->K || ldx % 8 != 0) return CONVROT_EINVAL;
     // One kernel (the quantiser warps run ahead of the tensor cores) when the
     // rows suit its 32-byte loads; otherwise the two-kernel path below.
-    if (fused_eligible(desc->K, desc->block) && (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && ldx % 16 == 0)
+    if (takes_one_kernel(x, ldx, desc))
         return linear_one_kernel(x, M, ldx, qw, s_w, desc, bias, epi, qx, sx, ready, y, ldy, s);
     st = rotate_quant(x, 2, M, desc->K, ldx, desc->block, qx, sx, s);
     if (st != CONVROT_OK) return st;
@@ -414,10 +521,10 @@ convrot_status convrot_linear_act(const uint16_t* h, int64_t M, int64_t ldh, int
     if (st != CONVROT_OK) return st;
     if (act != CONVROT_ACT_GELU && act != CONVROT_ACT_SWIGLU) return CONVROT_EINVAL;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CONVROT_EINVAL;
-    if (ws_bytes < convrot_workspace_bytes(M, desc->K)) return CONVROT_EINVAL;
-    int8_t* qx = static_cast<int8_t*>(workspace);
-    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                         round256(static_cast<size_t>(M) * static_cast<size_t>(desc->K)));
+    const WsLayout l = ws_layout(M, desc->K);
+    if (ws_bytes < l.full) return CONVROT_EINVAL;
+    float* sx = static_cast<float*>(workspace);
+    int8_t* qx = reinterpret_cast<int8_t*>(static_cast<uint8_t*>(workspace) + l.codes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     st = rotate_quant(h, 2, M, desc->K, ldh, desc->block, qx, sx, s, act);
     if (st != CONVROT_OK) return st;
@@ -524,11 +631,13 @@ convrot_status convrot_linear_fused_host(const uint16_t* x_host, int64_t M, cons
     if (!x_host || !y_host || !x_dev || !aligned16(x_dev)) return CONVROT_EINVAL;
     if (desc->N % 8 != 0) return CONVROT_EINVAL;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CONVROT_EINVAL;
-    if (ws_bytes < convrot_workspace_bytes(M, desc->K)) return CONVROT_EINVAL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t K = desc->K, N = desc->N;
     const int64_t chunk = host_chunk_rows(M, K);
+    // every chunk's call runs on the first (largest) chunk's workspace
+    if (ws_bytes < linear_ws_needed(x_dev, chunk, K, desc)) return CONVROT_EINVAL;
     HostPipe* hp = chunk < M ? host_pipe() : nullptr;
+    if (hp == nullptr && ws_bytes < linear_ws_needed(x_dev, M, K, desc)) return CONVROT_EINVAL;
     if (hp == nullptr) {  // one piece: copy in, compute, copy out, all on the caller's stream
         if (cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(M * K) * 2, cudaMemcpyHostToDevice, s) !=
             cudaSuccess)
@@ -612,7 +721,8 @@ convrot_status convrot_linear_fused_noalloc(const uint16_t* x, int64_t M, int64_
                                             int32_t epilogue, uint16_t* y, int64_t ldy, void* stream) {
     convrot_status st = linear_checks(qw, s_w, desc, epilogue, M, y, ldy, bias);
     if (st != CONVROT_OK) return st;
-    if (convrot_workspace_bytes(M, desc->K) > kNoAllocScratchBytes) return CONVROT_ETOOLARGE;
+    if (!x || !aligned16(x) || ldx < desc->K || ldx % 8 != 0) return CONVROT_EINVAL;
+    if (linear_ws_needed(x, M, ldx, desc) > kNoAllocScratchBytes) return CONVROT_ETOOLARGE;
     void* scratch = noalloc_scratch();
     if (scratch == nullptr) return CONVROT_ECUDA;
     return convrot_linear_fused(x, M, ldx, qw, s_w, desc, bias, epilogue, scratch, kNoAllocScratchBytes, y, ldy,

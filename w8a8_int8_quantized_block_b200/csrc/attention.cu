@@ -583,8 +583,13 @@ cudaError_t launch_attention(const CUtensorMap& qmap, const CUtensorMap& kmap, c
                              int Lq, int Lk, const float* s_q, const float* s_k, float scale_log2, uint16_t* o,
                              uint64_t limit_ns, unsigned int* err, bool pdl, cudaStream_t stream,
                              const AttnSplit& sp, void* part) {
-    cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    int set = 0;
+    if (!launch_figure_get(reinterpret_cast<const void*>(attention_kernel), kThreadsA, kSmemA, &set)) {
+        e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA);
+        if (e != cudaSuccess) return e;
+        launch_figure_put(reinterpret_cast<const void*>(attention_kernel), kThreadsA, kSmemA, 1);
+    }
     AttnArgs a;
     a.H = H;
     a.Lq = Lq;

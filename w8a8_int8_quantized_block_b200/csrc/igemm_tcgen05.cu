@@ -420,8 +420,13 @@ template <int EPI>
 cudaError_t launch_single(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
                           const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
     auto kern = igemm_kernel<EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal1);
-    if (e != cudaSuccess) return e;
+    int set = 0;
+    cudaError_t e;
+    if (!launch_figure_get(reinterpret_cast<const void*>(kern), kThreads1, kSmemTotal1, &set)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal1);
+        if (e != cudaSuccess) return e;
+        launch_figure_put(reinterpret_cast<const void*>(kern), kThreads1, kSmemTotal1, 1);
+    }
     const int64_t tiles = static_cast<int64_t>((a.M + BM1 - 1) / BM1) * ((a.N + BN - 1) / BN) * a.batch;
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaLaunchConfig_t cfg = {};
@@ -443,8 +448,7 @@ template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
                         const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
     auto kern = igemm_pair_kernel<EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalP);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     const int64_t tiles = static_cast<int64_t>((a.M + BMP - 1) / BMP) * ((a.N + BN - 1) / BN) * a.batch;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreadsP);
@@ -460,10 +464,15 @@ cudaError_t launch_pair(const CUtensorMap& amap, const CUtensorMap& bmap, const 
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
     int max_clusters = 0;
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
-    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
-    if (e != cudaSuccess) return e;
-    if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+    if (!launch_figure_get(reinterpret_cast<const void*>(kern), kThreadsP, kSmemTotalP, &max_clusters)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalP);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
+        e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+        launch_figure_put(reinterpret_cast<const void*>(kern), kThreadsP, kSmemTotalP, max_clusters);
+    }
     const int64_t pairs = tiles < max_clusters ? tiles : max_clusters;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     e = cudaLaunchKernelEx(&cfg, kern, amap, bmap, ymap, a);

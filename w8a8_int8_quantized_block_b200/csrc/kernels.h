@@ -8,6 +8,18 @@
 
 namespace convrot {
 
+// ---------------------------------------------------------------- launch set-up cache
+//
+// A kernel's launch set-up depends only on the kernel and the device: its
+// dynamic shared-memory opt-in and how many CTAs (or CTA clusters) of a given
+// block size and shared memory fit.  Asking the runtime for them costs tens of
+// microseconds of host time per call, which a small problem would spend
+// waiting, so each figure is found on its first use on a device and kept.
+// Key: the kernel's address, the current device, block size, dynamic shared
+// memory.  Thread-safe.
+bool launch_figure_get(const void* kernel, int threads, size_t smem, int* figure);
+void launch_figure_put(const void* kernel, int threads, size_t smem, int figure);
+
 // ---------------------------------------------------------------- rotate + quantise
 
 // Launch geometry of the rotate+quantise kernel for one row length.
@@ -50,6 +62,30 @@ enum ActKind : int { kActNone = 0, kActGelu = 1, kActSwiglu = 2 };
 cudaError_t launch_rotate_quant(const CUtensorMap& xmap, int in_elem_bytes, int kind, int act, int64_t M, int64_t K,
                                 const RqGeometry& g, int8_t* q, int64_t ldq, float* s, uint64_t limit_ns,
                                 unsigned int* err, int num_sms, cudaStream_t stream);
+
+// Launch geometry of the one-block-per-thread quantiser (rotate_quant_block.cu).
+struct RqbGeometry {
+    int tpr;           // threads holding data in one row (K / 128, one Hadamard block each)
+    int tpr_pad;       // threads per row including idle ones (long rows: = tpr, packed back to back)
+    int rows_per_cta;  // rows one CTA handles per group
+    int threads;       // CTA size
+    int nb;            // Hadamard blocks per row (the 4-D view's block extent)
+    int nstage;        // shared-memory ring slots
+    size_t smem_bytes; // dynamic shared memory requested
+};
+
+// Geometry for bf16 rows of K elements (K % 128 == 0, K <= 32768); false when
+// the rows do not fit this kernel.
+bool rqb_geometry(int64_t K, RqbGeometry* g);
+
+// The quantiser with one whole 128-element block per thread, for bf16 rows
+// rotated by the Sylvester H_128 (kind kRotSyl128) or not at all (kRotNone).
+// `xmap`: 4-D view {64 elements, K/128 blocks, 2 halves, M rows} with byte
+// strides {256, 128, row stride}, box {64, K/128, 2, rows_per_cta}, 128-byte
+// swizzle.  Same codes and scales as launch_rotate_quant.
+cudaError_t launch_rotate_quant_block(const CUtensorMap& xmap, int kind, int64_t M, const RqbGeometry& g, int8_t* q,
+                                      int64_t ldq, float* s, uint64_t limit_ns, unsigned int* err, int num_sms,
+                                      cudaStream_t stream);
 
 // One CTA waits on an mbarrier that nothing arrives on, so its bounded wait
 // must give up after `limit_ns` and record kErrTimeoutSelfTest.

@@ -362,8 +362,7 @@ template <int EPI, int KIND>
 cudaError_t launch_fused_epi(const CUtensorMap& amap, const CUtensorMap& bmap, const CUtensorMap& ymap,
                              const FusedArgs& f, int num_sms, bool pdl, cudaStream_t stream) {
     auto kern = linear_fused_kernel<EPI, KIND>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalF);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreadsF);
     cfg.dynamicSmemBytes = kSmemTotalF;
@@ -378,15 +377,21 @@ cudaError_t launch_fused_epi(const CUtensorMap& amap, const CUtensorMap& bmap, c
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
     int max_clusters = 0;
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
-    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
-    if (e != cudaSuccess) return e;
-    if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+    if (!launch_figure_get(reinterpret_cast<const void*>(kern), kThreadsF, kSmemTotalF, &max_clusters)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalF);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
+        e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+        launch_figure_put(reinterpret_cast<const void*>(kern), kThreadsF, kSmemTotalF, max_clusters);
+    }
     // Every CTA quantises rows other CTAs wait for, so all of them must be
-    // resident at once: never launch more clusters than fit.
-    const int64_t tiles = static_cast<int64_t>((f.g.M + kPanelRows - 1) / kPanelRows) * ((f.g.N + BN - 1) / BN);
-    const int64_t pairs = tiles < max_clusters ? tiles : max_clusters;
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    // resident at once: never launch more clusters than fit.  Launch all that
+    // fit even when there are fewer tiles: the quantiser groups of CTAs without
+    // a tile still share the rows (a 256-row problem of two tiles would
+    // otherwise quantise its rows 32 at a time in each of 8 groups).
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * max_clusters));
     e = cudaLaunchKernelEx(&cfg, kern, amap, bmap, ymap, f);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -68,6 +68,7 @@ constexpr int kMaxThreads = 512;
 #define CONVROT_RQ_MAX_IDLE_PCT 2  // pack long rows until at most this share of threads is idle
 #endif
 constexpr int kMaxStages = 3;
+constexpr int kRqSmemBudget = 200 * 1024;  // the largest dynamic shared memory a geometry may ask for
 constexpr int kMaxLongRows = 8;  // rows per group when rows span several warps
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -192,13 +193,17 @@ template <typename Tin, int KIND, int ACT>
 cudaError_t launch_typed(const CUtensorMap& xmap, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
                          float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
     auto kern = rotate_quant_kernel<Tin, KIND, ACT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(g.smem_bytes));
-    if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem_bytes);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (!launch_figure_get(reinterpret_cast<const void*>(kern), g.threads, g.smem_bytes, &per_sm)) {
+        // The opt-in is the largest slot ring any geometry asks for, so that it
+        // never shrinks below what an earlier launch of this kernel needed.
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRqSmemBudget);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem_bytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        launch_figure_put(reinterpret_cast<const void*>(kern), g.threads, g.smem_bytes, per_sm);
+    }
     const int64_t groups = (M + g.rows_per_cta - 1) / g.rows_per_cta;
     const int64_t cap = static_cast<int64_t>(per_sm) * num_sms;
     const int64_t grid = groups < cap ? groups : cap;
@@ -262,7 +267,7 @@ bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g)
     }
     const size_t slot = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
     if (slot % 1024 != 0) return false;  // slots must stay 1024-byte aligned for the swizzle
-    const size_t budget = 200 * 1024;
+    const size_t budget = kRqSmemBudget;
     g->nstage = CONVROT_RQ_STAGES;
     while (g->nstage > 1 && slot * g->nstage + 1024 > budget) --g->nstage;
     if (g->nstage > 2 && slot * g->nstage > 96 * 1024) g->nstage = 2;  // leave room for a second CTA
