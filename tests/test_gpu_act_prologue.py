@@ -32,6 +32,12 @@ def _h(M, K, act, seed):
     h[:, 3] *= 6  # an outlier channel
     h[0] = 0.0    # a zero row: s = 0, codes 0
     h[1, :] = -9.0  # deep in GELU's tail
+    if M > 2:
+        # inputs outside the kernel's tables of common values (tiny, huge, the
+        # edges of each range, zero), which it evaluates directly
+        odd = torch.tensor([1e-9, -3e-7, 9.5e-7, -9.6e-7, 1.5e-5, -1.6e-5, 255.0, -257.0, 4095.0, -4097.0,
+                            5000.0, -7000.0, 300.0, -1e4, 0.0, 2.0e-38])
+        h[2] = odd.repeat(cols // odd.numel() + 1)[:cols]
     return h.to(torch.bfloat16)
 
 

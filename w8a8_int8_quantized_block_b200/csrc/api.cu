@@ -177,8 +177,9 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
         return cuda_status(launch_rotate_quant_block(xmap4, kind, M, gb, q, K, s, g_limit_ns.load(), d->err,
                                                      d->num_sms, stream));
     }
+    const int ak = act == CONVROT_ACT_GELU ? kActGelu : act == CONVROT_ACT_SWIGLU ? kActSwiglu : kActNone;
     RqGeometry g;
-    if (!rq_geometry(K, row_elems, in_elem_bytes, &g)) return CONVROT_EINVAL;
+    if (!rq_geometry(K, row_elems, in_elem_bytes, &g, ak)) return CONVROT_EINVAL;
     CUtensorMap xmap;
     const uint32_t inner = 128u / static_cast<uint32_t>(in_elem_bytes);
     const CUtensorMapDataType dt =
@@ -187,7 +188,6 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
                    static_cast<uint64_t>(ldx) * in_elem_bytes, inner, static_cast<uint32_t>(g.box1),
                    static_cast<uint32_t>(g.rows_per_cta), CU_TENSOR_MAP_SWIZZLE_128B))
         return CONVROT_ECUDA;
-    const int ak = act == CONVROT_ACT_GELU ? kActGelu : act == CONVROT_ACT_SWIGLU ? kActSwiglu : kActNone;
     return cuda_status(launch_rotate_quant(xmap, in_elem_bytes, kind, ak, M, K, g, q, K, s, g_limit_ns.load(),
                                            d->err, d->num_sms, stream));
 }

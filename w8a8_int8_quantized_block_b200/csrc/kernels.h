@@ -38,7 +38,8 @@ struct RqGeometry {
 // K: elements quantised per row; row_elems: elements loaded per row (K, or
 // 2K for the SwiGLU prologue); in_elem_bytes: 2 for bf16 activations, 4 for
 // f32 weights.
-bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g);
+// act: the ActKind the kernel applies first (its table takes shared memory).
+bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g, int act = 0);
 
 // The rotations a row can get: none, Sylvester H_b (b = 64, 128, 256) or the
 // regular H_4^(x)k (b = 16, 64, 256).

@@ -144,28 +144,91 @@ __device__ __forceinline__ float gelu_prologue(float x) {
     return __double2float_rn(__dmul_rn(0.5 * v, erfc(t)));
 }
 
-// silu(g) * u = g / (1 + e^-g) * u in double (IEEE division and product),
-// rounded once to f32.
-__device__ __forceinline__ float swiglu_value(float g, float u) {
+
+// silu(g) = g / (1 + e^-g) in double (IEEE sum and division).
+__device__ __forceinline__ double silu_double(float g) {
     const double gd = static_cast<double>(g);
-    const double sg = __ddiv_rn(gd, __dadd_rn(1.0, exp(-gd)));
-    return __double2float_rn(__dmul_rn(sg, static_cast<double>(u)));
+    return __ddiv_rn(gd, __dadd_rn(1.0, exp(-gd)));
 }
 
-__device__ __forceinline__ void gelu_pairs(uint64_t (&P)[kPairs]) {
+// Tables of the activation for the common inputs.  The input h (or the gate
+// g) is a bf16 value, so its double-precision activation depends on 16 bits
+// only: a CTA evaluates it once for every bf16 value of a range of binades,
+// with the same double operations as above, into shared memory, and each
+// element then costs one shared-memory read.  Inputs outside the range (zero,
+// tiny or huge values, a few per million in activations) take the direct
+// evaluation, so every element gets the value the direct evaluation gives
+// it.  Entry of a bf16 bit pattern b: sign, then the binade
+// e - E0 (e the biased exponent), then the 7 mantissa bits.
+template <int E0, int BINADES>
+struct ActTable {
+    static constexpr int kEntries = 2 * BINADES * 128;
+    // The entry of bf16 bit pattern b, or -1 outside [2^(E0-127), 2^(E0-127+BINADES)).
+    __device__ static __forceinline__ int index(uint32_t b) {
+        const uint32_t d = ((b >> 7) & 0xFFu) - static_cast<uint32_t>(E0);
+        return d < static_cast<uint32_t>(BINADES)
+                   ? static_cast<int>((b >> 15) * (BINADES * 128) + d * 128 + (b & 0x7Fu))
+                   : -1;
+    }
+    // The bf16 value of entry i, widened to f32.
+    __device__ static __forceinline__ float value(int i) {
+        const int sgn = i / (BINADES * 128), r = i - sgn * (BINADES * 128);
+        return __uint_as_float(static_cast<uint32_t>((sgn << 15) | ((E0 + (r >> 7)) << 7) | (r & 127)) << 16);
+    }
+};
+using GeluTable = ActTable<107, 32>;  // |h| in [2^-20, 2^12): f32 entries, 32 KB
+using SiluTable = ActTable<111, 24>;  // |g| in [2^-16, 2^8): double entries (silu(g) before the product), 48 KB
+
+// Shared-memory bytes of the table an activation kernel keeps (0: none).
+constexpr int act_table_bytes(int act) {
+    return act == kActGelu ? GeluTable::kEntries * 4 : act == kActSwiglu ? SiluTable::kEntries * 8 : 0;
+}
+
+// Fill the table (all threads of the CTA; the caller synchronises after).
+template <int ACT>
+__device__ __forceinline__ void act_table_fill(void* tab, int tid, int nthreads) {
+    if constexpr (ACT == kActGelu) {
+        float* t = static_cast<float*>(tab);
+        for (int i = tid; i < GeluTable::kEntries; i += nthreads) t[i] = gelu_prologue(GeluTable::value(i));
+    } else if constexpr (ACT == kActSwiglu) {
+        double* t = static_cast<double*>(tab);
+        for (int i = tid; i < SiluTable::kEntries; i += nthreads) t[i] = silu_double(SiluTable::value(i));
+    }
+}
+
+// The direct evaluations for inputs outside a table's range, kept out of
+// line: inlined at every element they would make the loop many times longer
+// than the instruction cache, for a path almost never taken.
+__device__ __noinline__ float gelu_direct(float h) { return gelu_prologue(h); }
+__device__ __noinline__ double silu_direct(float g) { return silu_double(g); }
+
+__device__ __forceinline__ float gelu_lookup(float h, const float* tab) {
+    const int i = GeluTable::index(__float_as_uint(h) >> 16);
+    return i >= 0 ? tab[i] : gelu_direct(h);
+}
+
+__device__ __forceinline__ void gelu_pairs(uint64_t (&P)[kPairs], const float* tab) {
 #pragma unroll
     for (int j = 0; j < kPairs; ++j) {
         float a, b;
         upk(P[j], a, b);
-        P[j] = pk(gelu_prologue(a), gelu_prologue(b));
+        P[j] = pk(gelu_lookup(a, tab), gelu_lookup(b, tab));
     }
+}
+
+// silu(g) * u = g / (1 + e^-g) * u: the product in double (IEEE), rounded
+// once to f32; silu(g) from the table when g is in its range.
+__device__ __forceinline__ float swiglu_lookup(float g, float u, const double* tab) {
+    const int i = SiluTable::index(__float_as_uint(g) >> 16);
+    const double sg = i >= 0 ? tab[i] : silu_direct(g);
+    return __double2float_rn(__dmul_rn(sg, static_cast<double>(u)));
 }
 
 // x = silu(g) * u for this thread's 64 elements: P holds g; the matching u
 // are the thread's 64 bf16 of the row's second half, one 128-byte shared row
 // at 128-byte row `Ru` of the swizzled slot, read one 16-byte chunk (eight
 // elements) at a time.
-__device__ __forceinline__ void swiglu_pairs(uint64_t (&P)[kPairs], const uint8_t* slot, int Ru) {
+__device__ __forceinline__ void swiglu_pairs(uint64_t (&P)[kPairs], const uint8_t* slot, int Ru, const double* tab) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const uint4 v = *reinterpret_cast<const uint4*>(slot + Ru * 128 + ((c ^ (Ru & 7)) << 4));
@@ -177,8 +240,8 @@ __device__ __forceinline__ void swiglu_pairs(uint64_t (&P)[kPairs], const uint8_
             const int j = e & (kPairs - 1);
             float a, b;
             upk(P[j], a, b);
-            if (e < kPairs) a = swiglu_value(a, u);
-            else b = swiglu_value(b, u);
+            if (e < kPairs) a = swiglu_lookup(a, u, tab);
+            else b = swiglu_lookup(b, u, tab);
             P[j] = pk(a, b);
         }
     }

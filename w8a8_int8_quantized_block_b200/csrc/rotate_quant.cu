@@ -39,6 +39,8 @@
 // operations as the plain definition, in the same order.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "kernels.h"
 #include "ptx.cuh"
 #include "quant_core.cuh"
@@ -68,7 +70,8 @@ constexpr int kMaxThreads = 512;
 #define CONVROT_RQ_MAX_IDLE_PCT 2  // pack long rows until at most this share of threads is idle
 #endif
 constexpr int kMaxStages = 3;
-constexpr int kRqSmemBudget = 200 * 1024;  // the largest dynamic shared memory a geometry may ask for
+constexpr int kRqSmemBudget = 200 * 1024;  // the largest ring of row slots a geometry may ask for
+constexpr int kRqSmemOptIn = 226 * 1024;   // ring + an activation's table: the most any launch asks for
 constexpr int kMaxLongRows = 8;  // rows per group when rows span several warps
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -120,6 +123,9 @@ __global__ void __maxnreg__(ACT == kActNone ? CONVROT_RQ_MAXREG : CONVROT_RQ_MAX
                              static_cast<int>(g * rows_per_cta), policy);
     };
 
+    // The activation's table follows the ring (act_table_bytes(ACT) bytes).
+    void* act_tab = ring + static_cast<size_t>(nstage) * slot_bytes;
+    if constexpr (ACT != kActNone) act_table_fill<ACT>(act_tab, tid, blockDim.x);
     if (tid < 2 * kMaxLongRows) rowmax[tid / kMaxLongRows][tid % kMaxLongRows] = 0ull;
     if (tid == 0) {
         abort_flag = 0;
@@ -144,8 +150,9 @@ __global__ void __maxnreg__(ACT == kActNone ? CONVROT_RQ_MAXREG : CONVROT_RQ_MAX
         if (active) {
             const uint8_t* sl = ring + static_cast<size_t>(slot) * slot_bytes;
             load_pairs<Tin>(sl, rloc * row_pitch, t, P);
-            if constexpr (ACT == kActGelu) gelu_pairs(P);
-            if constexpr (ACT == kActSwiglu) swiglu_pairs(P, sl, rloc * row_pitch + tpr + t);  // u: second half
+            if constexpr (ACT == kActGelu) gelu_pairs(P, static_cast<const float*>(act_tab));
+            if constexpr (ACT == kActSwiglu)  // u: the row's second half
+                swiglu_pairs(P, sl, rloc * row_pitch + tpr + t, static_cast<const double*>(act_tab));
         } else {
 #pragma unroll
             for (int j = 0; j < kPairs; ++j) P[j] = 0ull;
@@ -193,21 +200,23 @@ template <typename Tin, int KIND, int ACT>
 cudaError_t launch_typed(const CUtensorMap& xmap, int64_t M, const RqGeometry& g, int8_t* q, int64_t ldq,
                          float* s, uint64_t limit_ns, unsigned int* err, int num_sms, cudaStream_t stream) {
     auto kern = rotate_quant_kernel<Tin, KIND, ACT>;
+    const size_t smem = g.smem_bytes + static_cast<size_t>(act_table_bytes(ACT));  // ring (+ the activation's table)
+    if (smem > static_cast<size_t>(kRqSmemOptIn)) return cudaErrorInvalidValue;
     int per_sm = 0;
-    if (!launch_figure_get(reinterpret_cast<const void*>(kern), g.threads, g.smem_bytes, &per_sm)) {
-        // The opt-in is the largest slot ring any geometry asks for, so that it
-        // never shrinks below what an earlier launch of this kernel needed.
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRqSmemBudget);
+    if (!launch_figure_get(reinterpret_cast<const void*>(kern), g.threads, smem, &per_sm)) {
+        // The opt-in is the most any geometry may ask for, so that it never
+        // shrinks below what an earlier launch of this kernel needed.
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRqSmemOptIn);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem_bytes);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, smem);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) return cudaErrorInvalidConfiguration;
-        launch_figure_put(reinterpret_cast<const void*>(kern), g.threads, g.smem_bytes, per_sm);
+        launch_figure_put(reinterpret_cast<const void*>(kern), g.threads, smem, per_sm);
     }
     const int64_t groups = (M + g.rows_per_cta - 1) / g.rows_per_cta;
     const int64_t cap = static_cast<int64_t>(per_sm) * num_sms;
     const int64_t grid = groups < cap ? groups : cap;
-    kern<<<static_cast<unsigned>(grid), g.threads, g.smem_bytes, stream>>>(
+    kern<<<static_cast<unsigned>(grid), g.threads, smem, stream>>>(
         xmap, M, g.tpr, g.tpr_pad, g.rows_per_cta, g.rows128, g.box1, g.nbox, g.nstage, groups, q, ldq, s, limit_ns,
         err);
     return cudaGetLastError();
@@ -221,7 +230,7 @@ int next_pow2(int v) {
 
 }  // namespace
 
-bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g) {
+bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g, int act) {
     if (K <= 0 || K % 64 != 0 || K > 32768) return false;
     if (row_elems != K && row_elems != 2 * K) return false;
     g->tpr = static_cast<int>(K / kPerThread);
@@ -267,7 +276,8 @@ bool rq_geometry(int64_t K, int64_t row_elems, int in_elem_bytes, RqGeometry* g)
     }
     const size_t slot = static_cast<size_t>(g->nbox) * g->box1 * 128 * g->rows_per_cta;
     if (slot % 1024 != 0) return false;  // slots must stay 1024-byte aligned for the swizzle
-    const size_t budget = kRqSmemBudget;
+    // the ring's share: an activation kernel also keeps its table in shared memory
+    const size_t budget = std::min<size_t>(kRqSmemBudget, kRqSmemOptIn - act_table_bytes(act));
     g->nstage = CONVROT_RQ_STAGES;
     while (g->nstage > 1 && slot * g->nstage + 1024 > budget) --g->nstage;
     if (g->nstage > 2 && slot * g->nstage > 96 * 1024) g->nstage = 2;  // leave room for a second CTA
