@@ -27,6 +27,14 @@ def test_library_builds_and_exports_every_declared_symbol():
     assert sorted(C.EXPORTS) == declared
 
 
+def test_library_matches_its_sources():
+    # the library that loads is the one built from the sources in this tree
+    # (a compile or link failure raises instead of leaving an older library)
+    from w8a8_int8_quantized_block_b200 import build as B
+    C.load()
+    assert B.is_current()
+
+
 def test_abi_version_and_status_strings():
     L = C.load()
     assert L.convrot_abi_version() == 1

@@ -5,6 +5,7 @@
 from __future__ import annotations
 
 import argparse
+import hashlib
 import os
 import shutil
 import subprocess
@@ -29,16 +30,35 @@ def _nvcc() -> str:
     return cand if os.path.exists(cand) else (shutil.which("nvcc") or "nvcc")
 
 
-def _newest_input() -> float:
+DIGEST = LIB + ".inputs"  # sha256 of the sources, headers and flags the library was built from
+
+
+def _inputs_digest() -> str:
+    """Digest of everything the library is built from (file contents, not
+    times: a copied tree keeps the digest whatever its files' times)."""
+    h = hashlib.sha256()
     paths = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     paths.append(os.path.join(ROOT, "include", "convrot.h"))
     paths.append(os.path.abspath(__file__))
-    return max(os.path.getmtime(p) for p in paths)
+    for p in paths:
+        h.update(p.encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def is_current() -> bool:
+    """Whether the built library matches the current sources."""
+    try:
+        with open(DIGEST) as f:
+            return os.path.exists(LIB) and f.read().strip() == _inputs_digest()
+    except OSError:
+        return False
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     """Compile every CUDA source for sm_100a and link the shared library."""
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
+    if not force and is_current():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     nvcc = _nvcc()
@@ -62,6 +82,8 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(DIGEST, "w") as f:
+        f.write(_inputs_digest() + "\n")
     return LIB
 
 

@@ -69,9 +69,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
         from . import build as _build
         try:
             _build.build()
-        except (OSError, RuntimeError) as e:  # no nvcc: only an existing library will do
+        except OSError as e:  # no nvcc here: only an existing library will do
             if not os.path.exists(p):
                 raise RuntimeError(f"libconvrot.so is missing and could not be built: {e}") from e
+        # (a failed compile or link raises: a library older than its sources is never used)
     if not os.path.exists(p):
         raise RuntimeError(f"libconvrot.so not found at {p}; run `python -m w8a8_int8_quantized_block_b200.build`")
     L = ctypes.CDLL(p)

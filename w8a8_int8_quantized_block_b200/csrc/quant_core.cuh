@@ -196,15 +196,9 @@ __device__ __forceinline__ void act_table_fill(void* tab, int tid, int nthreads)
     }
 }
 
-// The direct evaluations for inputs outside a table's range, kept out of
-// line: inlined at every element they would make the loop many times longer
-// than the instruction cache, for a path almost never taken.
-__device__ __noinline__ float gelu_direct(float h) { return gelu_prologue(h); }
-__device__ __noinline__ double silu_direct(float g) { return silu_double(g); }
-
 __device__ __forceinline__ float gelu_lookup(float h, const float* tab) {
     const int i = GeluTable::index(__float_as_uint(h) >> 16);
-    return i >= 0 ? tab[i] : gelu_direct(h);
+    return i >= 0 ? tab[i] : gelu_prologue(h);
 }
 
 __device__ __forceinline__ void gelu_pairs(uint64_t (&P)[kPairs], const float* tab) {
@@ -220,7 +214,7 @@ __device__ __forceinline__ void gelu_pairs(uint64_t (&P)[kPairs], const float* t
 // once to f32; silu(g) from the table when g is in its range.
 __device__ __forceinline__ float swiglu_lookup(float g, float u, const double* tab) {
     const int i = SiluTable::index(__float_as_uint(g) >> 16);
-    const double sg = i >= 0 ? tab[i] : silu_direct(g);
+    const double sg = i >= 0 ? tab[i] : silu_double(g);
     return __double2float_rn(__dmul_rn(sg, static_cast<double>(u)));
 }
 
