@@ -41,7 +41,7 @@ def _inputs_digest() -> str:
     paths.append(os.path.join(ROOT, "include", "convrot.h"))
     paths.append(os.path.abspath(__file__))
     for p in paths:
-        h.update(p.encode())
+        h.update(os.path.relpath(p, ROOT).encode())  # where the tree sits does not matter
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()
