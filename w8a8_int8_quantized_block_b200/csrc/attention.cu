@@ -34,11 +34,12 @@
 //   warps 2-9  softmax, four warps per query tile, one thread per query row
 //              (TMEM lane quadrant = warp % 4).  One sweep over the scores in
 //              TMEM (16-column loads, each overlapped with the arithmetic on
-//              the previous 16) gives the row maximum and,
-//              against the running maximum m, p = 2^(x - m) on the
-//              special-function unit, rounded to bf16 (kept in registers) and
-//              summed; a second sweep runs only when a row's maximum moved
-//              (see below).  p goes to the tile's P buffer (128-byte swizzle,
+//              the previous 16) gives, against the running maximum m,
+//              p = 2^(x - m) on the special-function unit, rounded to bf16
+//              (kept in registers) and summed.  The tile's row maximum is
+//              only taken when some row's sum of p exceeds 2^8 (else every
+//              p <= 2^8 and m stays), and the exponentials are redone only
+//              when a row's maximum moved (see below).  p goes to the tile's P buffer (128-byte swizzle,
 //              the A operand's canonical K-major layout).  Then O *=
 //              2^(m_old - m_new) in TMEM (the reference maximum moves only
 //              when a row's scores exceed it by more than 8 in log2 units, and
@@ -49,6 +50,8 @@
 // unwinds).  V arrives as V^T [h][d][key] (K-major for the P V product),
 // written by transpose_kernel below.
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "attention.h"
 #include "gemm_core.cuh"
@@ -333,22 +336,25 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 if (!ok) break;
                 tc_fence_after_sync();
                 const float4* cs4 = reinterpret_cast<const float4*>(sSk + st * kTile);
-                // One sweep over the tile's scores from TMEM: x = float(q . k) * s_k[c]
-                // (the score in log2 units is x * rs, rs = s_q * scale * log2(e) >= 0),
-                // the tile's row maximum, and p = 2^(x rs - mref) as packed bf16 in
-                // registers with their sum.
+                // Passes over the tile's scores from TMEM: x = float(q . k) * s_k[c]
+                // (the score in log2 units is x * rs, rs = s_q * scale * log2(e) >= 0)
+                // and p = 2^(x rs - mref) as packed bf16 in registers with their sum.
                 // The softmax is exact for any reference m (O / l cancels it); m
                 // only has to keep 2^(x - m) in range.  So the exponentials are
                 // taken against the running m right away, and m moves only when a
                 // row's maximum exceeds it by more than 8 (p <= 2^8 otherwise, fine
-                // in bf16 and f32): then, and on the first tile (m = -inf), a second
-                // sweep redoes the warp's rows against the new references (rows that
-                // did not move recompute the same values).
-                float mx = -INFINITY, m_new = m, mref = m;
+                // in bf16 and f32).  A row whose p sum to at most 2^8 has every
+                // p <= 2^8, so the maximum is taken (a second pass) only when some
+                // row's sum exceeds that, and a third pass redoes the exponentials
+                // only when some row's maximum moved.  The first tile (m = -inf)
+                // takes its maximum first, then the exponentials.
+                float m_new = m;
                 uint64_t sum2 = pk2(0.0f, 0.0f);
                 uint32_t pw[kTile / 2];
-#pragma unroll 1
-                for (int sweep = 0; sweep < 2; ++sweep) {
+                // One pass: with do_exp, p = 2^(x rs - mref) into pw and sum2; with
+                // do_max, the row maximum of x (returned, in log2 units).
+                auto pass = [&](auto do_max, auto do_exp, float mref) -> float {
+                    constexpr bool kMax = decltype(do_max)::value, kExp = decltype(do_exp)::value;
                     const uint64_t nm2 = pk2(-mref, -mref);
                     float mxa = -INFINITY, mxb = -INFINITY;
                     float4 cq;
@@ -369,23 +375,45 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                             const uint64_t x2 = mul2(pk2(__int2float_rn(static_cast<int>(r[2 * q])),
                                                          __int2float_rn(static_cast<int>(r[2 * q + 1]))),
                                                      c2);
-                            float x0, x1, y0, y1;
-                            upk2(x2, x0, x1);
-                            if (q & 1)
-                                mxb = max3(mxb, x0, x1);
-                            else
-                                mxa = max3(mxa, x0, x1);
-                            upk2(fma2(x2, rs2, nm2), y0, y1);
-                            const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-                            sum2 = add2(sum2, pk2(p0, p1));
-                            pw[pi] = pack2_bf16(p0, p1);
+                            if constexpr (kMax) {
+                                float x0, x1;
+                                upk2(x2, x0, x1);
+                                if (q & 1)
+                                    mxb = max3(mxb, x0, x1);
+                                else
+                                    mxa = max3(mxa, x0, x1);
+                            }
+                            if constexpr (kExp) {
+                                float y0, y1;
+                                upk2(fma2(x2, rs2, nm2), y0, y1);
+                                const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+                                sum2 = add2(sum2, pk2(p0, p1));
+                                pw[pi] = pack2_bf16(p0, p1);
+                            }
                         }
                         if (c + 1 < kTile / 16) tmem_ld_wait_regs(rb[(c + 1) & 1]);
                     }
-                    mx = fmaxf(mxa, mxb) * rs;  // the tile's row maximum in log2 units
-                    m_new = (mx > m + kRescaleLog2) ? mx : m;
-                    if (sweep == 1 || !__any_sync(0xFFFFFFFFu, m_new != mref)) break;
-                    mref = m_new;
+                    return fmaxf(mxa, mxb) * rs;
+                };
+                using T_ = std::true_type;
+                using F_ = std::false_type;
+                if (m == -INFINITY) {
+                    // the first key tile: the maximum first, then the exponentials against it
+                    m_new = pass(T_{}, F_{}, 0.0f);
+                    pass(F_{}, T_{}, m_new);
+                } else {
+                    // Against the running maximum m.  Every p <= 2^8 whenever the
+                    // tile's sum of p is at most 2^8, and then m need not move; only
+                    // a larger sum asks for the tile's maximum, and the exponentials
+                    // are redone when some row's maximum exceeds m by more than 8.
+                    pass(F_{}, T_{}, m);
+                    float s0, s1;
+                    upk2(sum2, s0, s1);
+                    if (__any_sync(0xFFFFFFFFu, !(s0 + s1 <= 256.0f))) {
+                        const float mx = pass(T_{}, F_{}, 0.0f);
+                        m_new = (mx > m + kRescaleLog2) ? mx : m;
+                        if (__any_sync(0xFFFFFFFFu, m_new != m)) pass(F_{}, T_{}, m_new);
+                    }
                 }
                 __syncwarp();  // the warp is done with the stage's key scales
                 if (lane == 0) mbar_arrive(&k_empty[st]);
