@@ -96,11 +96,13 @@ def parse():
     ap.add_argument("--rows", type=int, default=None,
                     help="with --kernel-only: only the first ROWS token rows of the projection (a smaller case "
                          "of the same workload, for detailed profiler captures)")
-    ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm", "bmm", "mlp-down", "act"], default=None,
+    ap.add_argument("--kernel-only", choices=["fused", "quant", "gemm", "bmm", "mlp-up", "mlp-down", "act"],
+                    default=None,
                     help="set up, then launch only this kernel --warmup + --steps times and exit "
                          "(for profiler captures; prints no result line).  bmm: the 42-head Q K^T GEMM "
-                         "(--heads for fewer); mlp-down: the MLP's down projection GEMM (K = 21504) on "
-                         "--rows rows; act: the GELU prologue quantiser of that projection")
+                         "(--heads for fewer); mlp-up: the MLP's up projection (one kernel, 5376 -> 21504, GELU "
+                         "epilogue) on --rows rows; mlp-down: its down projection GEMM (K = 21504); act: the "
+                         "GELU prologue quantiser of that projection")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads' legs (the configs object of the default line)")
     ap.add_argument("--sustained-seconds", type=float, default=2.0,
@@ -812,6 +814,17 @@ def kernel_only(args, spec, x, x_cpu, pw, bias, ws, y, stream):
         sa, sb = torch.rand(B * bs.M, device="cuda"), torch.rand(B * bs.N, device="cuda")
         yb = torch.empty(B, bs.M, bs.N, dtype=torch.bfloat16, device="cuda")
         one = lambda: C.w8a8_bmm(qa, sa, qb, sb, out=yb, stream=stream)
+    elif which == "mlp-up":  # the MLP's up projection on the first --rows rows of its workload
+        ms = W.MLP_768P
+        rows = ms.M if args.rows is None else args.rows
+        g = torch.Generator(device="cuda").manual_seed(ms.seed)
+        xu = (torch.randn(rows, ms.K, device="cuda", generator=g) * 2.0).to(torch.bfloat16)
+        w1 = torch.randn(ms.H, ms.K, device="cuda", generator=g) * ms.w_std
+        p1 = C.pack_weight(w1, ms.block)
+        del w1
+        wsu = C.alloc_workspace(rows, ms.K)
+        hu = torch.empty(rows, ms.H, dtype=torch.bfloat16, device="cuda")
+        one = lambda: C.linear_fused(xu, p1, None, gelu=True, workspace=wsu, out=hu, stream=stream)
     else:  # the MLP's down projection (K = 21504) on the first --rows rows of its workload
         ms = W.MLP_768P
         rows = ms.M if args.rows is None else args.rows

@@ -182,6 +182,35 @@ def test_linear_fused_codes_ring_equals_two_step_bitwise(M, K, N):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+@pytest.mark.parametrize("M,K,N", [(5000, 5376, 9488), (600, 6144, 8208)])
+def test_grouped_tile_order_one_kernel_equals_two_kernels(M, K, N):
+    # Weights over 48 MiB (N K = 51.0 / 50.4 MB): the two-kernel GEMM walks
+    # the row panels in groups of 8 per column tile, the one-kernel path in
+    # groups of half its codes ring.  5000 rows: 20 panels; two-kernel groups
+    # 8, 8, 4; one-kernel groups 6, 6, 6, 2 with a ring of 12 slots that wraps.
+    # 600 rows: 3 panels, one short group.  N ends in a part-filled column tile.
+    spec, (x, w, bias) = W.custom_linear(M, K, N, seed=M + 17, n_out=3, token_scale=True)
+    y1, pw = _run_linear((x, w, bias), fused=True)
+    y2, _ = _run_linear((x, w, bias), fused=False)
+    assert C.last_device_status() == (C.OK, 0)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    rows = np.unique(np.random.default_rng(M).choice(M, 24, replace=False))
+    yr, *_ = O.linear(bits(x[torch.from_numpy(rows)]), w.numpy(), bias.numpy(), 128)
+    assert_close_bf16(f32_of_bf16(y1[torch.from_numpy(rows).to(DEV)]), yr, "grouped tile order")
+
+
+def test_igemm_s32_grouped_tile_order_bitexact():
+    # N K = 8208 x 6144 = 50.4 MB: the accumulators of a grouped tile order
+    # (3 row panels of 256 in one short group, 33 column tiles, the last
+    # part-filled), every element against the exact int64 product
+    M, N, K = 700, 8208, 6144
+    qa = _codes((1, M, K), 31)
+    qb = _codes((1, N, K), 32)
+    acc = C.igemm_s32(qa.to(DEV), qb.to(DEV)).cpu().numpy().astype(np.int64)
+    assert C.last_device_status() == (C.OK, 0)
+    assert (acc[0] == O.igemm(qa[0].numpy(), qb[0].numpy())).all()
+
+
 def test_linear_fused_long_rows_match_oracle():
     # K > 6144 (the MLP down projection's 21504): linear_fused runs the
     # quantiser and the GEMM as two kernels

@@ -40,13 +40,23 @@ struct TileCoord {
     int m0, n0, b;
 };
 
-// Tile t of a [batch][tiles_m][tiles_n] grid of bm x BN tiles, n fastest.
-__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bm) {
+// Tile t of a [batch][tiles_m][tiles_n] grid of bm x BN tiles.  Within a
+// batch the row tiles go in groups of `group` (the last group may be
+// shorter); inside a group the column tile changes slowest and the row tile
+// fastest, so consecutive tiles (run at the same time by neighbouring CTA
+// pairs) share their column tile.  group = 1: n fastest, one row tile after
+// another.
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bm, int group = 1) {
     const int per_batch = tiles_m * tiles_n;
     const int b = t / per_batch;
     const int r = t - b * per_batch;
-    const int mb = r / tiles_n;
-    return {mb * bm, (r - mb * tiles_n) * BN, b};
+    const int per_group = group * tiles_n;
+    const int g = r / per_group;
+    const int rows = min(group, tiles_m - g * group);  // row tiles in this group
+    const int w = r - g * per_group;
+    const int n = w / rows;
+    const int mb = g * group + (w - n * rows);
+    return {mb * bm, n * BN, b};
 }
 
 // Column scale (s_b * alpha) and bias of one tile's BN columns into this

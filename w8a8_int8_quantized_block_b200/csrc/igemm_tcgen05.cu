@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1);
+                const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1, p.group_m);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, p.limit_ns, kErrTimeoutEmpty, p.err)) {
                         ok = false;
@@ -205,15 +205,15 @@ __global__ void __launch_bounds__(kThreads1, 1)
         int nbuf = 0;
         TileScales next{};
         if (blockIdx.x < num_tiles) {
-            const TileCoord c = tile_coord(blockIdx.x, tiles_m, tiles_n, BM1);
+            const TileCoord c = tile_coord(blockIdx.x, tiles_m, tiles_n, BM1, p.group_m);
             fetch_tile_scales<EPI>(p, c, c.m0 + quad * 32 + lane, lane, next);
         }
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1);
+            const TileCoord c = tile_coord(t, tiles_m, tiles_n, BM1, p.group_m);
             store_tile_columns<EPI>(next, p.alpha, sColScale, sColBias, lane);
             const float sa = next.row_scale;
             if (t + static_cast<int>(gridDim.x) < num_tiles) {
-                const TileCoord cn = tile_coord(t + gridDim.x, tiles_m, tiles_n, BM1);
+                const TileCoord cn = tile_coord(t + gridDim.x, tiles_m, tiles_n, BM1, p.group_m);
                 fetch_tile_scales<EPI>(p, cn, cn.m0 + quad * 32 + lane, lane, next);
             }
             const bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-                const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP);
+                const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP, p.group_m);
                 const int a_row = c.m0 + static_cast<int>(rank) * kGemmBM;
                 const int b_row = c.n0 + static_cast<int>(rank) * (BN / 2);
                 for (int kb = 0; kb < k_blocks; ++kb) {
@@ -378,15 +378,15 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         const int row_off = static_cast<int>(rank) * kGemmBM + quad * 32;  // this warp's rows within the tile
         TileScales next{};
         if (pair < num_tiles) {
-            const TileCoord c = tile_coord(pair, tiles_m, tiles_n, BMP);
+            const TileCoord c = tile_coord(pair, tiles_m, tiles_n, BMP, p.group_m);
             fetch_tile_scales<EPI>(p, c, c.m0 + row_off + lane, lane, next);
         }
         for (int t = pair; t < num_tiles; t += num_pairs) {
-            const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP);
+            const TileCoord c = tile_coord(t, tiles_m, tiles_n, BMP, p.group_m);
             store_tile_columns<EPI>(next, p.alpha, sColScale, sColBias, lane);
             const float sa = next.row_scale;
             if (t + num_pairs < num_tiles) {
-                const TileCoord cn = tile_coord(t + num_pairs, tiles_m, tiles_n, BMP);
+                const TileCoord cn = tile_coord(t + num_pairs, tiles_m, tiles_n, BMP, p.group_m);
                 fetch_tile_scales<EPI>(p, cn, cn.m0 + row_off + lane, lane, next);
             }
             const bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);

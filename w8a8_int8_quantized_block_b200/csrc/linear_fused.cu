@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             bool ok = true;
             int ready_panel = -1;
             for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-                const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows);
+                const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows, p.group_m);
                 const int panel = c.m0 / kPanelRows;
                 if (panel != ready_panel) {
                     if (!wait_count_bounded(f.ready + panel, panel_rows(panel, p.M), p.limit_ns, kErrTimeoutPanel,
@@ -303,7 +303,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                 // counts both halves), so its reads of the panel's ring slot are
                 // complete: the slot has one reader less.  (A plain reduction: the
                 // reads finished before the barrier wait returned.)
-                if (ok && f.ring < tiles_m) atomicAdd(f.loaded + t / tiles_n, 1u);
+                if (ok && f.ring < tiles_m)
+                    atomicAdd(f.loaded + tile_coord(t, tiles_m, tiles_n, kPanelRows, p.group_m).m0 / kPanelRows, 1u);
                 mma_commit_pair(&accf_bar[acc], 0x3);
                 if (++acc == kAccBufs) {
                     acc = 0;
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         uint32_t acc_phase = 0;
         int nbuf = 0;
         for (int t = pair; t < num_tiles; t += num_pairs) {
-            const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows);
+            const TileCoord c = tile_coord(t, tiles_m, tiles_n, kPanelRows, p.group_m);
             load_tile_columns<EPI>(p, c, sColScale, sColBias, lane);
             bool ok = mbar_wait_bounded(&accf_bar[acc], acc_phase, p.limit_ns, kErrTimeoutAccFull, p.err);
             tc_fence_after_sync();
