@@ -50,6 +50,10 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n,
     const int per_batch = tiles_m * tiles_n;
     const int b = t / per_batch;
     const int r = t - b * per_batch;
+    if (group == 1) {  // the plain order (the same tiles; two divisions fewer)
+        const int mb = r / tiles_n;
+        return {mb * bm, (r - mb * tiles_n) * BN, b};
+    }
     const int per_group = group * tiles_n;
     const int g = r / per_group;
     const int rows = min(group, tiles_m - g * group);  // row tiles in this group

@@ -274,6 +274,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                // the tile's row panel (its codes' ring slot gets one reader less below)
+                const int tile_panel = tile_coord(t, tiles_m, tiles_n, kPanelRows, p.group_m).m0 / kPanelRows;
                 if (!mbar_wait_bounded(&acce_bar[acc], acc_phase ^ 1u, p.limit_ns, kErrTimeoutAccEmpty, p.err)) {
                     ok = false;
                     break;
@@ -303,8 +305,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                 // counts both halves), so its reads of the panel's ring slot are
                 // complete: the slot has one reader less.  (A plain reduction: the
                 // reads finished before the barrier wait returned.)
-                if (ok && f.ring < tiles_m)
-                    atomicAdd(f.loaded + tile_coord(t, tiles_m, tiles_n, kPanelRows, p.group_m).m0 / kPanelRows, 1u);
+                if (ok && f.ring < tiles_m) atomicAdd(f.loaded + tile_panel, 1u);
                 mma_commit_pair(&accf_bar[acc], 0x3);
                 if (++acc == kAccBufs) {
                     acc = 0;
