@@ -160,11 +160,15 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
     const DeviceInfo* d = device_info();
     if (!d) return CONVROT_ECUDA;
     if (!d->supported) return CONVROT_EUNSUPPORTED;
-    // bf16 rows with the 128-point Sylvester rotation (or none) and K % 128 == 0:
-    // one whole Hadamard block per thread (fewer instructions per element).
+    // bf16 rows with the 128-point Sylvester rotation (or none), 256 <= K <= 8192
+    // and K % 128 == 0: one whole Hadamard block per thread (fewer instructions
+    // per element).  Measured against the 64-element kernel, back to back on
+    // 38656 rows: K = 5376 117 vs 123 us, K = 2048 equal; longer rows (K =
+    // 21504: 526 vs 508 us, one 352-thread CTA per SM) and K = 128 (24.6 vs
+    // 23.5 us on 344064 rows) keep the 64-element kernel.
     RqbGeometry gb;
     if (in_elem_bytes == 2 && act == CONVROT_ACT_NONE && (kind == kRotSyl128 || kind == kRotNone) &&
-        rqb_geometry(K, &gb)) {
+        K >= 256 && K <= 8192 && rqb_geometry(K, &gb)) {
         CUtensorMap xmap4;
         const uint64_t nb = static_cast<uint64_t>(K / 128);
         // {64 elements, K/128 blocks, 2 halves, M rows}: the first halves of a
