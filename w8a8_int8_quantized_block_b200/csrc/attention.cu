@@ -23,14 +23,16 @@
 //              still holds its values, so no load waits on the P V chain.
 //   warp 1     TMEM owner and MMA issuer (one thread), per key tile j and
 //              query tile t = A, B in turn:
-//                S_t = Q_t K_{j+1}^T  kind::i8, M = N = 128, 4 MMAs of K = 32
 //                O_t += P_t V_j       kind::f16 (bf16 in, f32 accumulate), 8
-//                                     MMAs of K = 16
-//              TMEM holds S_A, O_A, S_B, O_B (128 columns each).  The next
-//              scores of a tile are issued before its P V, and the tensor
-//              cores work on one query tile while the softmax works on the
-//              other.  (One issuer serving both tiles in turn measured faster
-//              than one issuer per tile: 1.90 vs 2.01 ms on 42 heads of 8192.)
+//                                     MMAs of K = 16, A (P_t) read from TMEM
+//                S_t = Q_t K_{j+1}^T  kind::i8, M = N = 128, 4 MMAs of K = 32
+//              TMEM holds S_A, O_A, S_B, O_B (128 columns each); P_t sits in
+//              the first 64 columns of S_t (bf16 pairs).  The tensor pipe runs
+//              one thread's MMAs in issue order, so the next scores overwrite
+//              P_t only after P V has read it; the tensor cores work on one
+//              query tile while the softmax works on the other.  (One issuer
+//              serving both tiles in turn measured faster than one issuer per
+//              tile: 1.90 vs 2.01 ms on 42 heads of 8192.)
 //   warps 2-9  softmax, four warps per query tile, one thread per query row
 //              (TMEM lane quadrant = warp % 4).  One sweep over the scores in
 //              TMEM (16-column loads, each overlapped with the arithmetic on
@@ -39,8 +41,10 @@
 //              (kept in registers) and summed.  The tile's row maximum is
 //              only taken when some row's sum of p exceeds 2^8 (else every
 //              p <= 2^8 and m stays), and the exponentials are redone only
-//              when a row's maximum moved (see below).  p goes to the tile's P buffer (128-byte swizzle,
-//              the A operand's canonical K-major layout).  Then O *=
+//              when a row's maximum moved (see below).  p goes back into TMEM
+//              over the scores just read (two 32-column stores), where P V
+//              takes it as its A operand, so P never passes through shared
+//              memory (which the MMAs' operand reads keep busy).  Then O *=
 //              2^(m_old - m_new) in TMEM (the reference maximum moves only
 //              when a row's scores exceed it by more than 8 in log2 units, and
 //              the rescale is skipped when no row of the warp moved); finally
@@ -71,17 +75,15 @@ constexpr int kQBytes = kTile * kD;           // int8 Q tile: 16 KB
 constexpr int kKBytes = kTile * kD;           // int8 K tile: 16 KB
 constexpr int kAtomBytes = 128 * 128;         // one 128-row x 128-byte swizzle column: 16 KB
 constexpr int kVBytes = 2 * kAtomBytes;       // V^T tile (128 d x 128 keys bf16): 32 KB
-constexpr int kPBytes = 2 * kAtomBytes;       // P tile (128 queries x 128 keys bf16): 32 KB
 constexpr int kSkBytes = kTile * 4;           // the tile's key scales
 constexpr int kKStages = 3;                   // K codes + key scales
 constexpr int kVStages = 2;                   // V^T
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQTiles * kQBytes;
 constexpr int kOffV = kOffK + kKStages * kKBytes;
-constexpr int kOffP = kOffV + kVStages * kVBytes;
-constexpr int kOffSk = kOffP + kQTiles * kPBytes;
+constexpr int kOffSk = kOffV + kVStages * kVBytes;
 constexpr int kOffBar = kOffSk + kKStages * kSkBytes;
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * kQTiles;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 3 * kQTiles;
 constexpr int kSmemA = kOffBar + kNumBars * 8 + 16 + 1024;  // + TMEM slot, + 1024-byte alignment slack
 static_assert(kSmemA <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kTmemColsA = 512;          // per query tile: S (128 columns), O (128 columns)
@@ -159,7 +161,6 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     uint8_t* sQ = smem + kOffQ;
     uint8_t* sK = smem + kOffK;
     uint8_t* sV = smem + kOffV;
-    uint8_t* sP = smem + kOffP;
     float* sSk = reinterpret_cast<float*>(smem + kOffSk);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* q_full = bars;
@@ -168,8 +169,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     uint64_t* v_full = k_empty + kKStages;    // [value stage]
     uint64_t* v_empty = v_full + kVStages;    // [value stage]
     uint64_t* s_full = v_empty + kVStages;    // [query tile]
-    uint64_t* s_free = s_full + kQTiles;      // [query tile]
-    uint64_t* p_ready = s_free + kQTiles;     // [query tile]
+    uint64_t* p_ready = s_full + kQTiles;     // [query tile]
     uint64_t* pv_done = p_ready + kQTiles;    // [query tile]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
@@ -200,8 +200,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         }
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&s_free[t], 4);   // one arrival per softmax warp of the tile
-            mbar_init(&p_ready[t], 4);
+            mbar_init(&p_ready[t], 4);  // one arrival per softmax warp of the tile
             mbar_init(&pv_done[t], 1);
         }
         fence_mbar_init();
@@ -256,53 +255,44 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             constexpr uint32_t idesc_qk = umma_idesc_i8(kTile, kTile);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kTile, kD);
             auto issue_qk = [&](int t, int j) {
-                const uint32_t q_addr = smem_u32(sQ + t * kQBytes);
-                const uint32_t k_addr = smem_u32(sK + (j % kKStages) * kKBytes);
+                const uint64_t qd = umma_desc_sw128_kmajor(smem_u32(sQ + t * kQBytes));
+                const uint64_t kd = umma_desc_sw128_kmajor(smem_u32(sK + (j % kKStages) * kKBytes));
 #pragma unroll
-                for (int k = 0; k < kD / 32; ++k)
-                    mma_i8(tmem + col_s(t), umma_desc_sw128_kmajor(q_addr + k * 32),
-                           umma_desc_sw128_kmajor(k_addr + k * 32), idesc_qk, k > 0 ? 1u : 0u);
+                for (int k = 0; k < kD / 32; ++k)  // + 32 bytes along K: + 2 in the descriptor's address field
+                    mma_i8(tmem + col_s(t), qd + static_cast<uint64_t>(k * 2), kd + static_cast<uint64_t>(k * 2),
+                           idesc_qk, k > 0 ? 1u : 0u);
                 mma_commit(&s_full[t]);
                 mma_commit(&k_empty[j % kKStages]);
             };
             auto issue_pv = [&](int t, int j) {
-                const uint32_t p_addr = smem_u32(sP + t * kPBytes);
-                const uint32_t v_addr = smem_u32(sV + (j % kVStages) * kVBytes);
+                const uint64_t vd = umma_desc_sw128_kmajor(smem_u32(sV + (j % kVStages) * kVBytes));
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     const uint32_t off = static_cast<uint32_t>((kk >> 2) * kAtomBytes + (kk & 3) * 32);
-                    mma_bf16(tmem + col_o(t), umma_desc_sw128_kmajor(p_addr + off),
-                             umma_desc_sw128_kmajor(v_addr + off), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + static_cast<uint32_t>(kk * 8),
+                                vd + static_cast<uint64_t>(off >> 4), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&pv_done[t]);
                 mma_commit(&v_empty[j % kVStages]);
             };
             bool ok = mbar_wait_bounded(q_full, 0, a.limit_ns, kErrTimeoutAttn, a.err) &&
                       mbar_wait_bounded(&k_full[0], 0, a.limit_ns, kErrTimeoutAttn, a.err);
-            for (int t = 0; t < nq && ok; ++t) {
-                ok = mbar_wait_bounded(&s_free[t], 0, a.limit_ns, kErrTimeoutAttn, a.err);
-                if (ok) {
-                    tc_fence_after_sync();
-                    issue_qk(t, 0);
-                }
+            if (ok) {
+                tc_fence_after_sync();
+                for (int t = 0; t < nq; ++t) issue_qk(t, 0);
             }
             for (int j = 0; j < T && ok; ++j) {
-                if (j + 1 < T)
-                    ok = mbar_wait_bounded(&k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, a.limit_ns,
-                                           kErrTimeoutAttn, a.err);
                 for (int t = 0; t < nq && ok; ++t) {
-                    if (j + 1 < T) {
-                        ok = mbar_wait_bounded(&s_free[t], (j + 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
-                        if (!ok) break;
-                        tc_fence_after_sync();
-                        issue_qk(t, j + 1);
-                    }
                     ok = mbar_wait_bounded(&p_ready[t], j & 1, a.limit_ns, kErrTimeoutAttn, a.err) &&
                          (t > 0 || mbar_wait_bounded(&v_full[j % kVStages], (j / kVStages) & 1, a.limit_ns,
-                                                     kErrTimeoutAttn, a.err));
+                                                     kErrTimeoutAttn, a.err)) &&
+                         (t > 0 || j + 1 >= T ||
+                          mbar_wait_bounded(&k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, a.limit_ns,
+                                            kErrTimeoutAttn, a.err));
                     if (!ok) break;
                     tc_fence_after_sync();
-                    issue_pv(t, j);
+                    issue_pv(t, j);  // reads P_t from S_t's first 64 columns
+                    if (j + 1 < T) issue_qk(t, j + 1);  // in the same in-order pipe: after P V has read P_t
                 }
             }
         }
@@ -317,14 +307,6 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             const uint32_t to = tmem + lane_base + col_o(t);
             const float rs = a.s_q[static_cast<int64_t>(h) * a.Lq + q0 + t * kTile + row] * a.scale_log2;
             const uint64_t rs2 = pk2(rs, rs);
-            uint8_t* prow = sP + t * kPBytes + row * 128;
-            // S_t may be overwritten by the next scores once the warp has read it
-            auto release_scores = [&]() {
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[t]);
-            };
-            release_scores();  // before the first tile's scores
             float m = -INFINITY, l = 0.0f;
             bool ok = true;
             for (int j = 0; j < T; ++j) {
@@ -418,21 +400,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 __syncwarp();  // the warp is done with the stage's key scales
                 if (lane == 0) mbar_arrive(&k_empty[st]);
                 const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf), 1 when m stays
-                // S_t has been read for the last time
-                if (j + 1 < T) release_scores();
-                // P_t is free, and O_t complete, once P V of tile j - 1 is done
-                if (j >= 1) {
-                    ok = mbar_wait_bounded(&pv_done[t], (j - 1) & 1, a.limit_ns, kErrTimeoutAttn, a.err);
-                    ok = __all_sync(0xFFFFFFFFu, ok);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                }
-#pragma unroll
-                for (int chunk16 = 0; chunk16 < kTile / 8; ++chunk16) {  // 8 keys = one 16-byte chunk of P
-                    const int atom = chunk16 >> 3, chunk = chunk16 & 7;
-                    *reinterpret_cast<uint4*>(prow + atom * kAtomBytes + ((chunk ^ (row & 7)) << 4)) =
-                        make_uint4(pw[4 * chunk16], pw[4 * chunk16 + 1], pw[4 * chunk16 + 2], pw[4 * chunk16 + 3]);
-                }
+                // P over S_t's first 64 columns (S_t is read; P V of key tile
+                // j - 1 completed before these scores were committed)
+                tmem_st_32x32b_x32(ts, pw);
+                tmem_st_32x32b_x32(ts + 32u, pw + 32);
                 float s0, s1;
                 upk2(sum2, s0, s1);
                 l = l * alpha + (s0 + s1);
@@ -449,10 +420,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                         for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
                         tmem_st_32x32b_x32(taddr, r);
                     }
-                    tmem_st_wait();
                 }
-                // P (generic-proxy stores) and O are ready for the tensor cores
-                fence_proxy_async_smem();
+                tmem_st_wait();  // P and the rescaled O are in tensor memory
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_ready[t]);

@@ -1,6 +1,7 @@
 // ptx_attn.cuh -- the inline-PTX wrappers only the attention kernels use:
-// kind::f16 MMA and its instruction descriptor, 16-column TMEM loads, TMEM
-// stores, the special-function 2^x and an untiled bulk copy into shared memory.
+// kind::f16 MMA (A from shared or from tensor memory) and its instruction
+// descriptor, 16-column TMEM loads, TMEM stores, the special-function 2^x and
+// an untiled bulk copy into shared memory.
 // Written from the public PTX ISA descriptions of these instructions.
 #pragma once
 
@@ -23,6 +24,19 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+// The same with A read from tensor memory: a_tmem addresses the M x 16 A tile
+// (TMEM lane = row; each 32-bit column holds two consecutive K elements, the
+// lower K index in the low half).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, f32 accumulator,
 // both operands K-major, tile M x N.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
@@ -34,8 +48,8 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
 }
 
 // The store counterpart of tmem_ld_32x32b_x32: lane i writes row
-// (lane base + i), columns [col, col + 32).
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+// (lane base + i), columns [col, col + 32), from r[0..31].
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t* r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
