@@ -142,3 +142,22 @@ def test_attention_int8_with_and_without_the_split_buffer():
     ref, _ = O.attention(bits(q), bits(k), bits(v))
     assert_close_bf16(o_split.float().cpu().numpy(), ref, "attention_int8 split")
     assert_close_bf16(o_whole.float().cpu().numpy(), ref, "attention_int8 whole")
+
+
+def test_attention_int8_split_buffer_16_byte_aligned():
+    # the entry asks only 16-byte alignment of the split buffer: one that is not
+    # 32-byte aligned gives the same output as an aligned one
+    H, Lq, Lk = 2, 256, 2048
+    q, k, v = _qkv(H, Lq, Lk, seed=12)
+    qx, sq = C.quantize_act(q.reshape(H * Lq, 128).to(DEV), 0)
+    kx, sk = C.quantize_act(k.reshape(H * Lk, 128).to(DEV), 0)
+    vt = v.transpose(1, 2).contiguous().to(DEV)
+    nbytes = C.attention_split_bytes(H, Lq, Lk)
+    buf = torch.empty((nbytes + 64,), dtype=torch.uint8, device=DEV)
+    assert buf.data_ptr() % 256 == 0
+    args = (qx.view(H, Lq, 128), sq.view(H, Lq), kx.view(H, Lk, 128), sk.view(H, Lk), vt)
+    o_16 = C.attention_int8(*args, split_ws=buf[16:16 + nbytes])
+    o_256 = C.attention_int8(*args, split_ws=buf[:nbytes])
+    torch.cuda.synchronize()
+    assert C.last_device_status() == (C.OK, 0)
+    assert torch.equal(o_16, o_256)

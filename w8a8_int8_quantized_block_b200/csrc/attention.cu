@@ -435,19 +435,16 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 // a part of the keys: the unnormalised O rows and (m, l) for the combine
                 tc_fence_after_sync();
                 const int64_t slot_row = static_cast<int64_t>(blockIdx.x) * (kQTiles * kTile) + t * kTile + row;
-                float* prow_o = a.o_part + slot_row * kD;
+                float* prow_o = a.o_part + slot_row * kD;  // 16-byte aligned (the entry's contract)
 #pragma unroll 1
                 for (int c4 = 0; c4 < kD / 32; ++c4) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(to + static_cast<uint32_t>(c4 * 32), r);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
-                                         prow_o + c4 * 32 + v * 8),
-                                     "r"(r[8 * v]), "r"(r[8 * v + 1]), "r"(r[8 * v + 2]), "r"(r[8 * v + 3]),
-                                     "r"(r[8 * v + 4]), "r"(r[8 * v + 5]), "r"(r[8 * v + 6]), "r"(r[8 * v + 7])
-                                     : "memory");
+                    for (int v = 0; v < 8; ++v)
+                        reinterpret_cast<uint4*>(prow_o + c4 * 32)[v] =
+                            make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                 }
                 a.ml_part[slot_row] = make_float2(m, l);
             } else if (ok) {
