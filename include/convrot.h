@@ -111,7 +111,8 @@ int convrot_abi_version(void);
  * w: f32 [N][K] row-major.  block: a block value (see above).
  * Writes q: int8 [N][K] (K contiguous, "output-major") and s_w: f32 [N], and
  * fills *desc (HOST pointer) synchronously.  Requires K % 64 == 0,
- * K % b == 0, K <= 32768, N <= 2^31-1, 16-byte aligned pointers.  Weights
+ * K % b == 0, K <= 32768, N <= 2^31-1, w 16-byte aligned, q 32-byte
+ * aligned (the codes are written in 32-byte stores), s_w 4-byte aligned.  Weights
  * must be finite: a row holding inf or NaN is outside the contract (its codes
  * and scale are unspecified; nothing checks them on the device). */
 convrot_status convrot_pack_weight(const float* w, int64_t N, int64_t K, int32_t block, int8_t* q,
@@ -120,7 +121,8 @@ convrot_status convrot_pack_weight(const float* w, int64_t N, int64_t K, int32_t
 /* Steps 1-2: x: bf16 [M][K] with row stride ldx (elements) ->
  * q: int8 [M][K] (contiguous) and s_x: f32 [M].  block: a block value.
  * Requires K % 64 == 0, K % b == 0, K <= 32768, ldx >= K, ldx % 8 == 0,
- * 0 < M <= 2^31-1.  A row of zeros gives s_x = 0 and zero codes.  Inputs
+ * 0 < M <= 2^31-1, x 16-byte aligned, q 32-byte aligned, s_x 4-byte
+ * aligned.  A row of zeros gives s_x = 0 and zero codes.  Inputs
  * must be finite: a row holding inf or NaN is outside the contract (its codes
  * and scale are unspecified; nothing checks them on the device).  The same
  * holds for every entry point that quantises activations. */
@@ -179,7 +181,8 @@ convrot_status convrot_linear_fused(const uint16_t* x, int64_t M, int64_t ldx, c
  * x is computed in f32 and goes straight into the rotation and quantiser of
  * convrot_quantize_act (same block values, same q / s_x); it is never stored.
  * Requires ldh >= K (GELU) or 2K (SwiGLU), ldh % 8 == 0, K % 64 == 0,
- * K % b == 0, K <= 32768.  Any other act is CONVROT_EINVAL. */
+ * K % b == 0, K <= 32768, h 16-byte aligned, q 32-byte aligned.  Any other
+ * act is CONVROT_EINVAL. */
 #define CONVROT_ACT_NONE 0
 #define CONVROT_ACT_GELU 1
 #define CONVROT_ACT_SWIGLU 2

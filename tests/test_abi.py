@@ -158,6 +158,21 @@ def test_misaligned_pointer_rejected():
     assert L.convrot_igemm_s32(FAKE, bad, 1, 4, 4, 16, FAKE, None) == C.EINVAL
 
 
+def test_codes_output_must_be_32_byte_aligned():
+    # the quantisers write the codes in 32-byte stores: a codes pointer that is
+    # only 16-byte aligned is refused before any device work
+    L = C.load()
+    q16 = ctypes.c_void_p(0x100010)
+    assert L.convrot_quantize_act(FAKE, 4, 512, 512, 128, q16, FAKE, None) == C.EINVAL
+    assert L.convrot_pack_weight(FAKE, 4, 512, 128, q16, FAKE, ctypes.byref(C.WDesc()), None) == C.EINVAL
+    assert L.convrot_act_quantize(FAKE, 4, 512, 512, C.ACT_GELU, 128, q16, FAKE, None) == C.EINVAL
+    # a 32-byte aligned codes pointer passes validation: without a GPU the
+    # device query fails (ECUDA); with one, the fake pointers must not launch
+    _skip_if_gpu()
+    q32 = ctypes.c_void_p(0x100020)
+    assert L.convrot_quantize_act(FAKE, 4, 512, 512, 128, q32, FAKE, None) == C.ECUDA
+
+
 def _desc(**kw):
     d = C.WDesc(C.WDESC_MAGIC, C.WDESC_VERSION, C.LAYOUT_OUTPUT_MAJOR, 128, 512, 512)
     for k, v in kw.items():

@@ -156,7 +156,9 @@ convrot_status rotate_quant(const void* x, int in_elem_bytes, int64_t M, int64_t
     const int64_t row_elems = act == CONVROT_ACT_SWIGLU ? 2 * K : K;
     if (K % 64 != 0 || K > 32768 || K % b != 0) return CONVROT_EINVAL;
     if (ldx < row_elems || (ldx * in_elem_bytes) % 16 != 0) return CONVROT_EINVAL;
-    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u) != 0) return CONVROT_EINVAL;
+    // the codes go out in 32-byte stores (each thread's 64 or 128 codes of a row)
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 31u) != 0 || (reinterpret_cast<uintptr_t>(s) & 3u) != 0)
+        return CONVROT_EINVAL;
     const DeviceInfo* d = device_info();
     if (!d) return CONVROT_ECUDA;
     if (!d->supported) return CONVROT_EUNSUPPORTED;
