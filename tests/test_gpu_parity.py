@@ -281,6 +281,31 @@ def test_linear_epilogue_on_identical_codes_is_tight():
     assert (err <= np.abs(yr) * 2.0 ** -8 + 1e-6).all()
 
 
+def test_gelu_epilogue_rounds_like_the_exact_gelu():
+    # Same codes on both sides, pre-activations spread over about [-12, 12] by
+    # the bias, so the negative tail is exercised (there GELU(y) is
+    # 0.5 y erfc(|y| / sqrt 2), many binades below y): nearly every output is
+    # the correctly rounded bf16 of the oracle's fp64 GELU of its fp64
+    # pre-activation, and none is further off than the f32 epilogue allows.
+    # (The f32 rounding of y^2 alone moves 2^(-log2(e) y^2 / 2) by ~6e-6 at
+    # y = -10, so a few in a thousand roundings may go the other way; the form
+    # 0.5 y (1 + erf(y / sqrt 2)) in f32 rounds about a third of them wrongly.)
+    x, w, _ = W.linear_inputs(W.TINY)
+    bias = torch.linspace(-12.0, 12.0, w.shape[0], dtype=torch.float32)
+    pw = C.pack_weight(w.to(DEV), 128)
+    q, s = C.quantize_act(x.to(DEV), 128)
+    y = C.w8a8_linear(q, s, pw, bias.to(DEV), gelu=True)
+    torch.cuda.synchronize()
+    assert C.last_device_status() == (C.OK, 0)
+    acc = O.igemm(q.cpu().numpy(), pw.q.cpu().numpy())
+    yr = O.dequant(acc, s.cpu().numpy(), pw.s.cpu().numpy(), bias.numpy(), 128, gelu=True)
+    got = f32_of_bf16(y).astype(np.float64)
+    nearest = torch.from_numpy(yr).to(torch.bfloat16).double().numpy()
+    assert (yr < -1e-6).mean() > 0.2  # the tail is really there
+    assert np.mean(got == nearest) >= 0.998
+    assert (np.abs(got - yr) <= np.abs(yr) * 2.0 ** -8 + 1e-5).all()
+
+
 # ------------------------------------------------------------------ batched skinny-K GEMM
 
 
