@@ -234,20 +234,27 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                 bulk_load_g2s(sSk + st * kTile, a.s_k + static_cast<int64_t>(h) * a.Lk + (j0 + j) * kTile,
                               kSkBytes, &k_full[st]);
             }
+            if (ok) drain_ring(k_empty, kKStages, T % kKStages, static_cast<uint32_t>(T / kKStages) & 1u, a.limit_ns,
+                               kErrTimeoutAttn, a.err);
         }
     } else if (warp == kWarpV) {
         if (lane == 0) {
             // ---------------------------------------------------------- value producer
+            bool ok = true;
             for (int j = 0; j < T; ++j) {
                 const int st = j % kVStages;
                 if (!mbar_wait_bounded(&v_empty[st], ((j / kVStages) & 1) ^ 1u, a.limit_ns, kErrTimeoutAttn,
-                                       a.err))
+                                       a.err)) {
+                    ok = false;
                     break;
+                }
                 mbar_arrive_expect_tx(&v_full[st], kVBytes);
                 // V^T rows are the 128 d; each 64-key half is one 128-byte swizzle column
                 tma_load_3d(sV + st * kVBytes, &vtmap, &v_full[st], (j0 + j) * kTile, 0, h);
                 tma_load_3d(sV + st * kVBytes + kAtomBytes, &vtmap, &v_full[st], (j0 + j) * kTile + 64, 0, h);
             }
+            if (ok) drain_ring(v_empty, kVStages, T % kVStages, static_cast<uint32_t>(T / kVStages) & 1u, a.limit_ns,
+                               kErrTimeoutAttn, a.err);
         }
     } else if (warp == 1) {
         if (lane == 0) {

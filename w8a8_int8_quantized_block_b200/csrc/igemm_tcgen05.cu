@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
                     }
                 }
             }
+            if (ok) drain_ring(empty_bar, kStages1, stage, phase, p.limit_ns, kErrTimeoutEmpty, p.err);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -320,6 +321,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     }
                 }
             }
+            // the stage-releasing commits reach both CTAs' empty barriers
+            if (ok) drain_ring(empty_bar, kStagesP, stage, phase, p.limit_ns, kErrTimeoutEmpty, p.err);
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {

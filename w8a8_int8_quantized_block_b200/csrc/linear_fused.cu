@@ -263,6 +263,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     }
                 }
             }
+            // the stage-releasing commits reach both CTAs' empty barriers
+            if (ok) drain_ring(empty_bar, kStagesF, stage, phase, p.limit_ns, kErrTimeoutEmpty, p.err);
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {

@@ -91,6 +91,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// A ring producer that is done waits, before it leaves, until the last fill
+// of every stage has been released by its consumer, so that no copy it issued
+// can still be landing when the CTA exits (each stage's next-fill wait in
+// turn, from the next slot (stage, phase) on; a stage never filled passes at
+// once).  It stops at the first time-out: by then a whole wait limit has
+// passed since its last copy was issued.  A producer that itself timed out
+// skips this for the same reason.
+__device__ __forceinline__ void drain_ring(uint64_t* empty_bar, int nstages, int stage, uint32_t phase,
+                                           uint64_t limit_ns, unsigned int code, unsigned int* err) {
+    for (int i = 0; i < nstages; ++i) {
+        if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, limit_ns, code, err)) return;
+        if (++stage == nstages) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
